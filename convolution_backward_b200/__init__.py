@@ -1,0 +1,205 @@
+"""convolution_backward_b200 -- B200 (sm_100a) convolution backward-data (dgrad).
+
+A thin ctypes binding over ``libdgrad.so`` (the C ABI in ``include/dgrad.h``).
+This module only marshals arguments: it checks tensor shapes, dtypes and
+devices, passes raw device pointers and the current CUDA stream, and raises on
+a non-OK status.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback.  If the library is missing the
+calls raise ``DgradUnavailable``.
+
+    dX = pointwise(dY, W)                          # dY (N,H,W,K), W (K,C) -> (N,H,W,C)
+    dX = depthwise(dY, W, H=H, W=W_, stride=1, pad_h=1, pad_w=1)   # W (KH,KW,C)
+
+Tensors are NHWC and contiguous; float32 or bfloat16 (bf16 in, bf16 out,
+fp32 accumulate).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["pointwise", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+           "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libdgrad.so")
+_lock = threading.Lock()
+_lib = None
+
+STATUS = {0: "DGRAD_OK", 1: "DGRAD_ERR_INVALID", 2: "DGRAD_ERR_UNSUPPORTED", 3: "DGRAD_ERR_ALIGNMENT",
+          4: "DGRAD_ERR_CUDA", 5: "DGRAD_ERR_TIMEOUT"}
+DW_MODES = {"auto": 0, "rotated": 1, "rowstream": 2}
+DTYPES = {"f32": 0, "bf16": 1}
+
+
+class DgradUnavailable(RuntimeError):
+    """libdgrad.so could not be loaded (not built, or built for another platform)."""
+
+
+class DgradError(RuntimeError):
+    def __init__(self, status: int, what: str, cuda_error: int = 0):
+        self.status = status
+        self.cuda_error = cuda_error
+        msg = f"{what}: {STATUS.get(status, status)}"
+        if status == 4:
+            msg += f" (cudaError {cuda_error})"
+        super().__init__(msg)
+
+
+class Problem(ctypes.Structure):
+    """dgrad_problem_t: N, H, W, C, K (int64), KH, KW, stride, pad_h, pad_w (int32)."""
+    _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64),
+                ("C", ctypes.c_int64), ("K", ctypes.c_int64), ("KH", ctypes.c_int32),
+                ("KW", ctypes.c_int32), ("stride", ctypes.c_int32), ("pad_h", ctypes.c_int32),
+                ("pad_w", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded libdgrad (ctypes.CDLL) with argument types declared."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise DgradUnavailable(
+                    f"{_LIB_PATH} is missing; build it with `python -m convolution_backward_b200._build` "
+                    "(nvcc, sm_100a)")
+            try:
+                L = ctypes.CDLL(_LIB_PATH)
+            except OSError as e:
+                raise DgradUnavailable(f"cannot load {_LIB_PATH}: {e}") from e
+            P = ctypes.POINTER
+            vp = ctypes.c_void_p
+            L.dgrad_pointwise.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp]
+            L.dgrad_pointwise.restype = ctypes.c_int
+            L.dgrad_depthwise.argtypes = [P(Problem), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+            L.dgrad_depthwise.restype = ctypes.c_int
+            L.dgrad_out_dims.argtypes = [P(Problem), P(ctypes.c_int64), P(ctypes.c_int64)]
+            L.dgrad_out_dims.restype = ctypes.c_int
+            L.dgrad_check_status.argtypes = [vp]
+            L.dgrad_check_status.restype = ctypes.c_int
+            L.dgrad_status_string.argtypes = [ctypes.c_int]
+            L.dgrad_status_string.restype = ctypes.c_char_p
+            L.dgrad_last_cuda_error.argtypes = []
+            L.dgrad_last_cuda_error.restype = ctypes.c_int
+            L.dgrad_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
+            L.dgrad_selftest_timeout.restype = ctypes.c_int
+            L.dgrad_fma_probe.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
+            L.dgrad_fma_probe.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise DgradError(status, what, lib().dgrad_last_cuda_error())
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return 0
+    if t.dtype == torch.bfloat16:
+        return 1
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (NHWC)")
+
+
+def out_dims(H, W, KH, KW, stride=1, pad_h=0, pad_w=-1):
+    """(Ho, Wo) of the forward convolution (host-only C call)."""
+    prob = Problem(1, H, W, 1, 1, KH, KW, stride, pad_h, pad_w)
+    ho, wo = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().dgrad_out_dims(ctypes.byref(prob), ctypes.byref(ho), ctypes.byref(wo)), "dgrad_out_dims")
+    return ho.value, wo.value
+
+
+def pointwise(dY, W, out=None, stream=None):
+    """Pointwise dgrad: dX[n,h,w,:] = dY[n,h,w,:] @ W, dY (N,H,W,K), W (K,C).  Calls dgrad_pointwise."""
+    import torch
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 2 or W.shape[0] != dY.shape[3]:
+        raise ValueError("expected dY (N,H,W,K) and W (K,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
+    N, H, Wd, K = dY.shape
+    C = W.shape[1]
+    if out is None:
+        out = torch.empty((N, H, Wd, C), dtype=dY.dtype, device=dY.device)
+    else:
+        _need_cuda(out)
+        if tuple(out.shape) != (N, H, Wd, C) or out.dtype != dY.dtype:
+            raise ValueError("out has the wrong shape or dtype")
+    prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
+    _check(lib().dgrad_pointwise(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
+                                 out.data_ptr(), _stream_ptr(stream)), "dgrad_pointwise")
+    return out
+
+
+def depthwise(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, mode="auto", out=None,
+              stream=None, **kw):
+    """Depthwise dgrad (groups = C): dY (N,Ho,Wo,C), W (KH,KW,C) -> dX (N,H,W,C).  Calls dgrad_depthwise.
+
+    H and W_out (alias ``Wd``) are dX's spatial extents; pad_w = -1 means pad_h.
+    mode: "auto" (rotated-filter at stride 1, row-streaming otherwise),
+    "rotated" or "rowstream".
+    """
+    import torch
+    if W_out is None:
+        W_out = kw.pop("Wd")
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 3 or W.shape[2] != dY.shape[3]:
+        raise ValueError("expected dY (N,Ho,Wo,C) and W (KH,KW,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
+    N, Ho, Wo, C = dY.shape
+    KH, KW = W.shape[0], W.shape[1]
+    prob = Problem(N, H, W_out, C, C, KH, KW, stride, pad_h, pad_w)
+    eho, ewo = out_dims(H, W_out, KH, KW, stride, pad_h, pad_w)
+    if (eho, ewo) != (Ho, Wo):
+        raise ValueError(f"dY spatial extent {(Ho, Wo)} does not match the geometry ({eho}, {ewo})")
+    if out is None:
+        out = torch.empty((N, H, W_out, C), dtype=dY.dtype, device=dY.device)
+    else:
+        _need_cuda(out)
+        if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
+            raise ValueError("out has the wrong shape or dtype")
+    _check(lib().dgrad_depthwise(ctypes.byref(prob), _dtype_code(dY), DW_MODES[mode], dY.data_ptr(),
+                                 W.data_ptr(), out.data_ptr(), _stream_ptr(stream)), "dgrad_depthwise")
+    return out
+
+
+def check_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel reported a timeout (dgrad_check_status)."""
+    _check(lib().dgrad_check_status(_stream_ptr(stream)), "dgrad_check_status")
+
+
+def selftest_timeout(limit_cycles: int = 20_000_000, stream=None) -> None:
+    """Launch the diagnostic kernel whose bounded wait runs out (dgrad_selftest_timeout)."""
+    _check(lib().dgrad_selftest_timeout(int(limit_cycles), _stream_ptr(stream)), "dgrad_selftest_timeout")
+
+
+def fma_probe(blocks: int, iters: int, packed: bool, sink, stream=None) -> int:
+    """Launch the fp32 FMA-rate probe; returns the FLOP count it performs."""
+    _check(lib().dgrad_fma_probe(int(blocks), int(iters), 1 if packed else 0, sink.data_ptr(),
+                                 _stream_ptr(stream)), "dgrad_fma_probe")
+    return int(blocks) * 256 * int(iters) * 16 * 2

@@ -1,0 +1,337 @@
+// dgrad_abi.cu -- the C ABI of libdgrad (declared in include/dgrad.h).
+//
+// Host side only: argument validation (everything is checked before anything
+// is launched), TMA tensor-map encoding for the tensor-core kernel, the per-device
+// status word the kernels report timeouts into, and dispatch to the kernels.
+// Also two diagnostics: a self-test kernel whose bounded wait is made to run
+// out (it checks the timeout path without hanging anything) and an FMA-rate
+// probe used to measure the fp32 roofline.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "dgrad.h"
+#include "launchers.h"
+
+namespace {
+
+thread_local int t_last_cuda = 0;
+
+// One status word per device: module-scope device variables exist once per
+// device context that loads the library.
+__device__ int g_status_word;
+
+struct DeviceState {
+    bool ready = false;
+    int* status = nullptr;   // device address of g_status_word on that device
+    int sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mu;
+
+dgrad_status_t cuda_fail(cudaError_t e)
+{
+    t_last_cuda = static_cast<int>(e);
+    return DGRAD_ERR_CUDA;
+}
+
+dgrad_status_t device_state(DeviceState** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return DGRAD_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState& st = g_devices[dev];
+    if (!st.ready) {
+        void* addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_status_word);
+        if (e != cudaSuccess) return cuda_fail(e);
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        st.status = static_cast<int*>(addr);
+        st.sms = sms;
+        st.ready = true;
+    }
+    *out = &st;
+    return DGRAD_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box box_cols x box_rows, 128B swizzle.
+bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int env_int(const char* name, int dflt)
+{
+    const char* v = getenv(name);
+    return v && *v ? atoi(v) : dflt;
+}
+
+// Checks shared by both entry points.  Fills the output extents.
+dgrad_status_t validate_common(const dgrad_problem_t* p, dgrad_dtype_t dtype, int64_t* Ho, int64_t* Wo,
+                               int* pad_w)
+{
+    if (!p) return DGRAD_ERR_INVALID;
+    if (dtype != DGRAD_F32 && dtype != DGRAD_BF16) return DGRAD_ERR_INVALID;
+    if (p->N < 0 || p->H < 1 || p->W < 1 || p->C < 1 || p->K < 1) return DGRAD_ERR_INVALID;
+    if (p->KH < 1 || p->KW < 1 || p->stride < 1) return DGRAD_ERR_INVALID;
+    if (p->pad_h < 0 || p->pad_w < -1) return DGRAD_ERR_INVALID;
+    const int pw = p->pad_w == -1 ? p->pad_h : p->pad_w;
+    const int64_t nh = p->H + 2 * static_cast<int64_t>(p->pad_h) - p->KH;
+    const int64_t nw = p->W + 2 * static_cast<int64_t>(pw) - p->KW;
+    if (nh < 0 || nw < 0) return DGRAD_ERR_INVALID;
+    *Ho = nh / p->stride + 1;
+    *Wo = nw / p->stride + 1;
+    *pad_w = pw;
+    return DGRAD_OK;
+}
+
+}  // namespace
+
+namespace dgrad {
+int device_sm_count()
+{
+    DeviceState* st = nullptr;
+    return device_state(&st) == DGRAD_OK ? st->sms : 148;
+}
+}  // namespace dgrad
+
+extern "C" {
+
+dgrad_status_t dgrad_out_dims(const dgrad_problem_t* prob, int64_t* Ho, int64_t* Wo)
+{
+    if (!Ho || !Wo) return DGRAD_ERR_INVALID;
+    int pw = 0;
+    return validate_common(prob, DGRAD_F32, Ho, Wo, &pw);
+}
+
+dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W,
+                               void* dX, void* stream)
+{
+    int64_t Ho = 0, Wo = 0;
+    int pw = 0;
+    dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
+    if (s != DGRAD_OK) return s;
+    if (prob->KH != 1 || prob->KW != 1 || prob->stride != 1 || prob->pad_h != 0 || pw != 0)
+        return DGRAD_ERR_UNSUPPORTED;
+    const int64_t M = prob->N * prob->H * prob->W;
+    if (M == 0) return DGRAD_OK;
+    if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
+    const int64_t esz = dtype == DGRAD_BF16 ? 2 : 4;
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (prob->K * esz) % 16 || (prob->C * esz) % 16)
+        return DGRAD_ERR_ALIGNMENT;
+    if (M > 0x7FFFFFFFLL || prob->K > 65536 || prob->C > 65536) return DGRAD_ERR_UNSUPPORTED;
+
+    DeviceState* st = nullptr;
+    s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    dgrad::PwArgs a{M, prob->K, prob->C, dY, W, dX, st->status};
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (dtype == DGRAD_F32) {
+        e = dgrad::launch_pointwise_f32(a, cs);
+    } else {
+        const int bn = env_int("DGRAD_PW_BN", prob->C <= 64 ? 64 : 128);
+        CUtensorMap map_a, map_b;
+        if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->K), 64, 128) ||
+            !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(prob->K), static_cast<uint64_t>(prob->C), 64, 64))
+            return cuda_fail(cudaErrorInvalidValue);
+        e = dgrad::launch_pointwise_tc(a, map_a, map_b, bn, st->sms, cs);
+    }
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype, dgrad_dw_mode_t mode,
+                               const void* dY, const void* W, void* dX, void* stream)
+{
+    int64_t Ho = 0, Wo = 0;
+    int pw = 0;
+    dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
+    if (s != DGRAD_OK) return s;
+    if (mode != DGRAD_DW_AUTO && mode != DGRAD_DW_ROTATED && mode != DGRAD_DW_ROWSTREAM) return DGRAD_ERR_INVALID;
+    if (prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;
+    if (mode == DGRAD_DW_AUTO) mode = prob->stride == 1 ? DGRAD_DW_ROTATED : DGRAD_DW_ROWSTREAM;
+    if (mode == DGRAD_DW_ROTATED && prob->stride != 1) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->stride > 8) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->H > (1 << 24) || prob->W > (1 << 24) || prob->C > (1 << 24)) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->N == 0) return DGRAD_OK;
+    if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
+    const int64_t esz = dtype == DGRAD_BF16 ? 2 : 4;
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (prob->C * esz) % 16) return DGRAD_ERR_ALIGNMENT;
+
+    DeviceState* st = nullptr;
+    s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    dgrad::DwArgs a{};
+    a.N = static_cast<int>(prob->N);
+    a.H = static_cast<int>(prob->H);
+    a.W = static_cast<int>(prob->W);
+    a.C = static_cast<int>(prob->C);
+    a.Ho = static_cast<int>(Ho);
+    a.Wo = static_cast<int>(Wo);
+    a.KH = prob->KH;
+    a.KW = prob->KW;
+    a.S = prob->stride;
+    a.ph = prob->pad_h;
+    a.pw = pw;
+    a.bf16 = dtype == DGRAD_BF16;
+    a.dY = dY;
+    a.filt = W;
+    a.dX = dX;
+    a.status = st->status;
+    if (prob->N > 0x7FFFFFFFLL) return DGRAD_ERR_UNSUPPORTED;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = mode == DGRAD_DW_ROTATED ? dgrad::launch_dw_rotated(a, cs) : dgrad::launch_dw_rowstream(a, cs);
+    if (e == cudaErrorInvalidConfiguration) return DGRAD_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+dgrad_status_t dgrad_check_status(void* stream)
+{
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    DeviceState* st = nullptr;
+    dgrad_status_t s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    int v = 0;
+    e = cudaMemcpy(&v, st->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (v != 0) {
+        const int zero = 0;
+        e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return v == dgrad::DEV_TIMEOUT ? DGRAD_ERR_TIMEOUT : DGRAD_OK;
+}
+
+const char* dgrad_status_string(dgrad_status_t s)
+{
+    switch (s) {
+    case DGRAD_OK: return "ok";
+    case DGRAD_ERR_INVALID: return "invalid argument";
+    case DGRAD_ERR_UNSUPPORTED: return "unsupported problem for this entry point";
+    case DGRAD_ERR_ALIGNMENT: return "pointer or channel row not 16-byte aligned";
+    case DGRAD_ERR_CUDA: return "CUDA error";
+    case DGRAD_ERR_TIMEOUT: return "a kernel gave up waiting (timeout)";
+    }
+    return "unknown status";
+}
+
+int dgrad_last_cuda_error(void) { return t_last_cuda; }
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ diagnostics
+
+namespace {
+
+// One CTA waits on an mbarrier that nothing will ever complete, with a cycle
+// budget; when the budget runs out it records the timeout exactly as the real
+// kernels do and returns.
+__global__ void selftest_timeout_kernel(long long limit_cycles, int* status)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        dgrad::mbar_init(&bar, 1);
+        dgrad::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        bool ok = dgrad::mbar_try_wait(&bar, 0);
+        const long long t0 = clock64();
+        while (!ok && clock64() - t0 <= limit_cycles) ok = dgrad::mbar_try_wait(&bar, 0);
+        if (!ok) dgrad::report_timeout(status);
+    }
+}
+
+// FMA-rate probe: 8 independent accumulator chains per thread, `iters` rounds.
+// packed = 1 uses fma.rn.f32x2 (two FMAs per instruction).  The result is
+// written so the work cannot be discarded.
+__global__ void __launch_bounds__(256) fma_probe_kernel(int iters, int packed, float* sink)
+{
+    float a = 1.0f + threadIdx.x * 1e-7f, b = 0.999999f;
+    if (packed) {
+        float2 acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = make_float2(a + i, a - i);
+        const float2 m = make_float2(b, b), c = make_float2(1e-7f, -1e-7f);
+        for (int it = 0; it < iters; ++it)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __ffma2_rn(acc[i], m, c);
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s += acc[i].x + acc[i].y;
+        if (s == 12345.678f) sink[blockIdx.x] = s;
+    } else {
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = a + i;
+        for (int it = 0; it < iters; ++it)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] = fmaf(acc[i], b, 1e-7f);
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s += acc[i];
+        if (s == 12345.678f) sink[blockIdx.x] = s;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+dgrad_status_t dgrad_selftest_timeout(long long limit_cycles, void* stream)
+{
+    if (limit_cycles < 0 || limit_cycles > dgrad::kWaitCycles) return DGRAD_ERR_INVALID;
+    DeviceState* st = nullptr;
+    dgrad_status_t s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles, st->status);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+dgrad_status_t dgrad_fma_probe(int blocks, int iters, int packed, float* sink, void* stream)
+{
+    if (blocks < 1 || iters < 1 || !sink) return DGRAD_ERR_INVALID;
+    fma_probe_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(iters, packed, sink);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// launchers.h -- host-side entry points of the individual kernels, called by
+// the C ABI layer (dgrad_abi.cu) after it has validated the problem.  Each
+// launcher only enqueues work on `stream`; none synchronises or allocates.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dgrad {
+
+// Pointwise dgrad as a GEMM: dX[M][C] = dY[M][K] * W[K][C], all row-major.
+struct PwArgs {
+    int64_t M, K, C;
+    const void* dY;
+    const void* W;
+    void* dX;
+    int* status;  // device status word
+};
+
+// fp32 in / fp32 out, fp32 FMA (no reduced-precision tensor-core path).
+cudaError_t launch_pointwise_f32(const PwArgs& a, cudaStream_t stream);
+
+// bf16 in / bf16 out on tcgen05 with TMEM accumulators.  map_a covers dY as a
+// 2-D [M][K] bf16 tensor with a 64 x 128 box (K innermost) and map_b covers W as
+// a 2-D [K][C] bf16 tensor with a 64 x 64 box (C innermost), both with the
+// 128-byte swizzle.  bn is the tile width along C (64, 128 or 256).
+cudaError_t launch_pointwise_tc(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                int bn, int num_sms, cudaStream_t stream);
+
+// Depthwise problem (groups = C = K), NHWC, dense.
+struct DwArgs {
+    int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;
+    bool bf16;  // element type of dY, W and dX: bf16 (true) or f32 (false)
+    const void* dY;
+    const void* filt;  // W[KH][KW][C]
+    void* dX;
+    int* status;
+};
+
+// Stride-1 rotated-filter correlation.  Requires S == 1, KH, KW <= 64.
+cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream);
+
+// Row-streaming kernel with a circular shared-memory accumulator ring (any S <= 8).
+cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace dgrad

@@ -1,0 +1,287 @@
+// pointwise_tc.cu -- pointwise (1x1) dgrad on the Blackwell tensor cores.
+//
+// For a 1x1 filter with stride 1, no padding and one group, dgrad is a plain
+// GEMM: dX[M][C] = dY[M][K] * W[K][C] with M = N*H*W, and every address is an
+// affine function of (m, k, c) -- dY at m*K + k, W at k*C + c, dX at m*C + c
+// ("add the pointwise fast path dgrad was missing", Technical Details and the
+// fast-path commit).  Here the K-loop holds no address arithmetic at all: TMA
+// moves whole tiles by coordinate and the tensor cores consume them from shared
+// memory through descriptors.
+//
+// Kernel structure (persistent, one CTA per SM, 192 threads):
+//   warp 0      TMA producer: dY tile 128 x 64 (K-major) and W tile 64 x BN
+//               (C contiguous, i.e. MN-major for the MMA) into a STAGES-deep ring.
+//   warp 1      allocates 2*BN TMEM columns, then one lane issues
+//               tcgen05.mma (M=128, N=BN, K=16) into one of two accumulators.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp may read the
+//               32 TMEM lanes of its quarter), round to bf16 (nearest even),
+//               16-byte stores to dX.  The second accumulator lets the MMAs of
+//               the next tile run while this one drains.
+// Tiles are taken round-robin in (m-block, n-block) order with n fastest, so
+// the CTAs working at one time share their dY rows through L2.
+//
+// Every wait is bounded (common.cuh); on a timeout the kernel records it in the
+// status word, raises a CTA-wide abort flag, lets in-flight copies and MMAs land
+// and frees its tensor memory before returning.
+#include "common.cuh"
+#include "launchers.h"
+
+namespace dgrad {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+
+template <int BN, int STAGES>
+struct PwTcLayout {
+    static constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+    static constexpr int kBBytes = kBK * BN * 2;    // 8 KB per 64 columns
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kTileBytes = STAGES * kStageBytes;
+    static constexpr int kNumBars = 2 * STAGES + 5;  // full, empty, tmem full x2, tmem empty x2, drain
+    static constexpr int kBytes = kTileBytes + kNumBars * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;     // slack to align the tiles to 1024 bytes
+    static constexpr uint32_t kTmemCols = 2 * BN;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    pw_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                 __nv_bfloat16* __restrict__ dX, int M, int C, int K, int* status)
+{
+    using L = PwTcLayout<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kTileBytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (M + kBM - 1) / kBM;
+    const int num_n = (C + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol_b = policy_evict_last();   // W is re-read by every tile
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                const int m_blk = t / num_n;
+                const int n_blk = t - m_blk * num_n;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+                    uint8_t* a_tile = smem + stage * L::kStageBytes;
+                    uint8_t* b_tile = a_tile + L::kABytes;
+                    tma_load_2d(a_tile, &map_a, &full[stage], kb * kBK, m_blk * kBM);
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tma_load_2d_hint(b_tile + j * 8192, &map_b, &full[stage], n_blk * BN + j * 64, kb * kBK,
+                                         pol_b);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            // Let the last copies land before the CTA may exit.
+            for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
+                const int s = static_cast<int>(i % STAGES);
+                const uint32_t par = static_cast<uint32_t>((i / STAGES) & 1);
+                if (!mbar_wait(&full[s], par)) {
+                    report_timeout(status);
+                    *abort_flag = 1;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
+                    const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        // A: advance 16 k (32 bytes) inside the 128-byte swizzled row.
+                        const uint64_t a_desc = sw128_desc(a_addr + kk * 32, 16, 1024);
+                        // B: advance 16 k-rows (2 groups of 8 rows of 128 bytes).
+                        const uint64_t b_desc = sw128_desc(b_addr + kk * 2048, 8192, 1024);
+                        umma_f16(d_tmem, a_desc, b_desc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty[stage]);   // frees the stage once these MMAs have read it
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);         // accumulator complete
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            umma_commit(drain);                   // all MMAs issued above have finished
+            if (!mbar_wait(drain, 0)) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        // ----------------------------------------------------------- epilogue
+        const int quarter = warp & 3;             // TMEM lanes this warp may read
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const int m_blk = t / num_n;
+            const int n_blk = t - m_blk * num_n;
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int m = m_blk * kBM + row;
+            __nv_bfloat16* out_row = dX + static_cast<int64_t>(m) * C;
+#pragma unroll 1
+            for (int chunk = 0; chunk < BN / 32; ++chunk) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + chunk * 32), v);
+                tmem_wait_ld();
+                const int col0 = n_blk * BN + chunk * 32;
+                if (m < M) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int col = col0 + g * 8;
+                        if (col < C) {
+                            uint4 o;
+                            o.x = float2_to_bf16x2(__uint_as_float(v[g * 8 + 0]), __uint_as_float(v[g * 8 + 1]));
+                            o.y = float2_to_bf16x2(__uint_as_float(v[g * 8 + 2]), __uint_as_float(v[g * 8 + 3]));
+                            o.z = float2_to_bf16x2(__uint_as_float(v[g * 8 + 4]), __uint_as_float(v[g * 8 + 5]));
+                            o.w = float2_to_bf16x2(__uint_as_float(v[g * 8 + 6]), __uint_as_float(v[g * 8 + 7]));
+                            *reinterpret_cast<uint4*>(out_row + col) = o;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) {
+            report_timeout(status);
+            *abort_flag = 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int num_sms,
+                      cudaStream_t stream)
+{
+    using L = PwTcLayout<BN, STAGES>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    auto kern = pw_tc_kernel<BN, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const int num_tiles = static_cast<int>(((a.M + kBM - 1) / kBM) * ((a.C + BN - 1) / BN));
+    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, static_cast<__nv_bfloat16*>(a.dX),
+                                                 static_cast<int>(a.M), static_cast<int>(a.C),
+                                                 static_cast<int>(a.K), a.status);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pointwise_tc(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int bn,
+                                int num_sms, cudaStream_t stream)
+{
+    if (a.M <= 0) return cudaSuccess;
+    switch (bn) {
+    case 64: return launch_bn<64, 8>(a, map_a, map_b, num_sms, stream);
+    case 256: return launch_bn<256, 4>(a, map_a, map_b, num_sms, stream);
+    default: return launch_bn<128, 6>(a, map_a, map_b, num_sms, stream);
+    }
+}
+
+}  // namespace dgrad

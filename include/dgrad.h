@@ -1,0 +1,134 @@
+/*
+ * dgrad.h -- C ABI of libdgrad, a B200 (sm_100a) engine for convolution
+ * backward-data ("dgrad"): dX = dgrad(dY, W) on NHWC activations.
+ *
+ * Operation.  For a forward convolution with dilation 1, stride S, per-axis
+ * padding (pad_h, pad_w) and output extents
+ *     Ho = floor((H + 2*pad_h - KH) / S) + 1,   Wo = floor((W + 2*pad_w - KW) / S) + 1
+ * ("channel-packed and large-filter depthwise dgrad", Technical Details,
+ * per-axis padding: Wo uses PAD_W), dgrad is the adjoint of the forward map in
+ * its input:
+ *     dX[n,h,w,c] = sum over (ho,wo,k,r,s) with h = ho*S - pad_h + r and
+ *                   w = wo*S - pad_w + s of dY[n,ho,wo,k] * Wt(k,r,s,c).
+ * Two shape classes are served:
+ *   - pointwise: 1x1 filter, stride 1, no padding, one group.  dX[M,C] =
+ *     dY[M,K] . W[K,C] with M = N*H*W, dY offset m*K + k, W offset k*C + c and
+ *     dX offset m*C + c ("add the pointwise fast path dgrad was missing",
+ *     Technical Details and the fast-path commit message);
+ *   - depthwise: groups = C = K (depth multiplier 1), W[KH][KW][C].  Stride 1
+ *     runs as a correlation of dY with the 180-degree rotated filter at padding
+ *     KH-1-pad_h rows and KW-1-pad_w columns, filters up to 64 a side, square or
+ *     not; stride > 1 runs as a row-streaming kernel whose accumulator rows sit
+ *     in a circular shared-memory ring ("channel-packed and large-filter
+ *     depthwise dgrad", Technical Details: rotated-filter dgrad and the
+ *     channel-packed row-streaming dgrad).
+ *
+ * Layouts (all dense, channels innermost, no padding between rows):
+ *     dY  [N][Ho][Wo][K]      dX [N][H][W][C]
+ *     W   pointwise [K][C];   depthwise [KH][KW][C]
+ * Element type: DGRAD_F32 (float in, float out) or DGRAD_BF16 (bf16 in, bf16
+ * out).  Accumulation is always fp32; a bf16 dX is rounded once, to nearest even.
+ *
+ * Memory and streams.  Every pointer is device memory the caller owns (for
+ * example a PyTorch CUDA tensor's data pointer) on the current device.  Calls
+ * enqueue work on `stream` (a cudaStream_t; NULL is the legacy default stream)
+ * and return without synchronising; the library allocates no device memory per
+ * call.  dX is written in full (never accumulated into), so it needs no zeroing.
+ * Alignment: every base pointer 16-byte aligned, and K and C multiples of 8
+ * (bf16) or 4 (f32), so that every channel row starts on 16 bytes.
+ *
+ * Errors.  Arguments are validated on the host before anything is launched; a
+ * rejected call launches nothing and leaves dX untouched.  A launch failure is
+ * reported as DGRAD_ERR_CUDA (the CUDA error is kept for dgrad_last_cuda_error).
+ * Kernels never trap: a device-side wait that runs past its limit sets a status
+ * word and the kernel returns; dgrad_check_status reports it.
+ */
+#ifndef DGRAD_H
+#define DGRAD_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem geometry (the pages' DirectConvProblem: extents, filter, stride and
+ * per-axis padding; "channel-packed and large-filter depthwise dgrad",
+ * Technical Details, per-axis padding).  H, W are dX's spatial extents; C is
+ * dX's channel count and K dY's.  Dilation is 1.  pad_w == -1 means "same as
+ * pad_h" (the pages' sentinel); any other negative value is invalid. */
+typedef struct {
+    int64_t N, H, W, C, K;
+    int32_t KH, KW, stride;
+    int32_t pad_h, pad_w;
+} dgrad_problem_t;
+
+typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1 } dgrad_dtype_t;
+
+/* Depthwise kernel choice.  AUTO: rotated-filter for stride 1, row-streaming
+ * otherwise.  ROTATED requires stride 1.  ROWSTREAM serves any stride (at
+ * stride 1 it is a cross-check of the rotated-filter kernel). */
+typedef enum { DGRAD_DW_AUTO = 0, DGRAD_DW_ROTATED = 1, DGRAD_DW_ROWSTREAM = 2 } dgrad_dw_mode_t;
+
+typedef enum {
+    DGRAD_OK = 0,
+    DGRAD_ERR_INVALID = 1,      /* null pointer, non-positive extent, pad_w < -1, Ho or Wo < 1 ... */
+    DGRAD_ERR_UNSUPPORTED = 2,  /* valid geometry this entry point does not serve */
+    DGRAD_ERR_ALIGNMENT = 3,    /* base pointer or channel row not 16-byte aligned */
+    DGRAD_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    DGRAD_ERR_TIMEOUT = 5       /* a kernel gave up waiting (reported by dgrad_check_status) */
+} dgrad_status_t;
+
+/* Pointwise dgrad, dX[M,C] = dY[M,K] . W[K,C] with M = N*H*W.
+ * Requires KH = KW = 1, stride 1, pad_h = pad_w = 0 (else DGRAD_ERR_UNSUPPORTED;
+ * the pointwise page's shape class).  DGRAD_BF16 runs on the tcgen05 tensor
+ * cores (TMA-fed shared-memory tiles, fp32 accumulators in tensor memory);
+ * DGRAD_F32 runs as an fp32 FMA kernel (no reduced-precision inputs). */
+dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
+                               const void* dY, const void* W, void* dX, void* stream);
+
+/* Depthwise dgrad (groups = C; requires K == C, else DGRAD_ERR_UNSUPPORTED).
+ * Rotated-filter mode requires stride 1, KH and KW <= 64 and
+ * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1 (the rotated padding KH-1-pad_h and
+ * KW-1-pad_w is then non-negative).  Row-streaming requires KH, KW <= 64,
+ * stride <= 8, 0 <= pad_h <= KH-1 and 0 <= pad_w <= KW-1. */
+dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
+                               dgrad_dw_mode_t mode,
+                               const void* dY, const void* W, void* dX, void* stream);
+
+/* Output extents of the forward convolution the problem describes (host only,
+ * no CUDA call).  Returns DGRAD_ERR_INVALID for an invalid problem. */
+dgrad_status_t dgrad_out_dims(const dgrad_problem_t* prob, int64_t* Ho, int64_t* Wo);
+
+/* Synchronise `stream`, then report (and clear) the device status word of the
+ * current device: DGRAD_ERR_TIMEOUT if any kernel gave up waiting since the
+ * last check, DGRAD_ERR_CUDA if the stream reported an error, else DGRAD_OK. */
+dgrad_status_t dgrad_check_status(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* dgrad_status_string(dgrad_status_t status);
+
+/* The last CUDA error code the library saw on this thread (0 if none). */
+int dgrad_last_cuda_error(void);
+
+/* ---- Diagnostics (no counterpart on the pages; they support testing and
+ * measurement of the entry points above). ---- */
+
+/* Enqueue one small kernel whose bounded wait is made to run out: it waits on a
+ * barrier nothing completes for `limit_cycles` SM cycles (0 .. 2e9), then
+ * records a timeout in the status word exactly as the dgrad kernels do and
+ * returns.  dgrad_check_status then reports DGRAD_ERR_TIMEOUT and clears it.
+ * Used to test the failure path without faulting or hanging the GPU. */
+dgrad_status_t dgrad_selftest_timeout(long long limit_cycles, void* stream);
+
+/* Enqueue an fp32 FMA-rate probe: `blocks` CTAs of 256 threads, each thread
+ * running `iters` rounds of 16 independent FMAs (packed != 0: as 8 fma.rn.f32x2).
+ * Work = blocks * 256 * iters * 16 FMAs.  `sink` is a device buffer of at least
+ * `blocks` floats that keeps the work live (normally left untouched). */
+dgrad_status_t dgrad_fma_probe(int blocks, int iters, int packed, float* sink, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DGRAD_H */

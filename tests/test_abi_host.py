@@ -1,0 +1,151 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+- libdgrad.so loads and exports every function include/dgrad.h declares;
+- dgrad_out_dims computes the forward extents (per-axis padding, pad_w = -1);
+- every validation rule rejects before anything touches the GPU (the pointers
+  passed here are never dereferenced: a rejected call launches nothing);
+- an empty batch is a no-op.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import convolution_backward_b200 as cb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+OK, INVALID, UNSUPPORTED, ALIGNMENT = 0, 1, 2, 3
+FAKE = 0x10000   # 16-byte aligned, never dereferenced
+BF16, F32 = 1, 0
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(dgrad_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = cb.lib()
+    names = declared_functions()
+    assert "dgrad_pointwise" in names and "dgrad_depthwise" in names
+    for n in names:
+        assert hasattr(L, n), f"libdgrad.so does not export {n}"
+
+
+def test_status_strings():
+    L = cb.lib()
+    for code in range(6):
+        s = L.dgrad_status_string(code)
+        assert s and isinstance(s, bytes)
+    assert L.dgrad_status_string(0) == b"ok"
+
+
+@pytest.mark.parametrize("geom,expect", [
+    ((56, 56, 3, 3, 1, 1, 1), (56, 56)),
+    ((112, 112, 7, 7, 2, 3, 3), (56, 56)),
+    ((64, 64, 51, 5, 1, 25, 2), (64, 64)),
+    ((64, 64, 5, 51, 1, 2, 25), (64, 64)),
+    ((10, 9, 3, 3, 1, 1, -1), (10, 9)),        # pad_w = -1 means pad_h
+    ((10, 9, 3, 3, 1, 1, 0), (10, 7)),
+    ((28, 28, 1, 1, 1, 0, 0), (28, 28)),
+])
+def test_out_dims(geom, expect):
+    assert cb.out_dims(*geom) == expect
+
+
+def _prob(N=1, H=8, W=8, C=16, K=16, KH=3, KW=3, S=1, ph=1, pw=1):
+    return cb.Problem(N, H, W, C, K, KH, KW, S, ph, pw)
+
+
+def _dw(prob, dtype=BF16, mode=0, ptrs=(FAKE, FAKE, FAKE)):
+    return cb.lib().dgrad_depthwise(ctypes.byref(prob), dtype, mode, *ptrs, None)
+
+
+def _pw(prob, dtype=BF16, ptrs=(FAKE, FAKE, FAKE)):
+    return cb.lib().dgrad_pointwise(ctypes.byref(prob), dtype, *ptrs, None)
+
+
+def test_null_problem_is_invalid():
+    L = cb.lib()
+    assert L.dgrad_pointwise(None, BF16, FAKE, FAKE, FAKE, None) == INVALID
+    assert L.dgrad_depthwise(None, BF16, 0, FAKE, FAKE, FAKE, None) == INVALID
+    ho = ctypes.c_int64()
+    assert L.dgrad_out_dims(None, ctypes.byref(ho), ctypes.byref(ho)) == INVALID
+
+
+@pytest.mark.parametrize("kw", [
+    dict(H=0), dict(W=-1), dict(C=0), dict(K=0), dict(N=-1), dict(KH=0), dict(S=0),
+    dict(ph=-1), dict(pw=-2), dict(pw=-7), dict(H=2, KH=7, ph=1),   # Ho < 1
+])
+def test_invalid_geometry(kw):
+    assert _dw(_prob(**kw)) == INVALID
+
+
+def test_bad_dtype_and_mode():
+    assert _dw(_prob(), dtype=7) == INVALID
+    assert _dw(_prob(), mode=9) == INVALID
+
+
+def test_null_pointers_invalid():
+    assert _dw(_prob(), ptrs=(0, FAKE, FAKE)) == INVALID
+    assert _pw(_prob(KH=1, KW=1, ph=0, pw=0), ptrs=(FAKE, 0, FAKE)) == INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(KH=3, KW=3, ph=1, pw=1), dict(KH=1, KW=1, S=2, ph=0, pw=0),
+                                dict(KH=1, KW=1, ph=1, pw=1), dict(KH=1, KW=1, ph=0, pw=1)])
+def test_pointwise_refuses_other_shapes(kw):
+    assert _pw(_prob(**kw)) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,mode", [
+    (dict(K=32, C=16), 0),                           # depth multiplier 2
+    (dict(KH=65, ph=1, H=70), 0),                    # filter over 64 rows
+    (dict(KW=65, pw=1, W=70), 0),
+    (dict(S=2), 1),                                  # rotated mode at stride 2
+    (dict(KH=3, ph=3, H=8), 0),                      # pad beyond KH-1
+    (dict(KW=3, pw=3), 0),
+    (dict(S=9, H=40, W=40), 2),                      # stride over 8
+])
+def test_depthwise_refusals(kw, mode):
+    assert _dw(_prob(**kw), mode=mode) == UNSUPPORTED
+
+
+def test_alignment():
+    assert _dw(_prob(), ptrs=(FAKE + 2, FAKE, FAKE)) == ALIGNMENT
+    assert _dw(_prob(), ptrs=(FAKE, FAKE, FAKE + 8)) == ALIGNMENT
+    assert _dw(_prob(C=12, K=12)) == ALIGNMENT                  # 24-byte bf16 rows
+    assert _dw(_prob(C=12, K=12), dtype=F32) != ALIGNMENT       # 48-byte f32 rows are fine
+    p = _prob(KH=1, KW=1, ph=0, pw=0, K=20, C=16)
+    assert _pw(p) == ALIGNMENT                                  # K*2 = 40 bytes
+    assert _pw(_prob(KH=1, KW=1, ph=0, pw=0), ptrs=(FAKE, FAKE + 4, FAKE)) == ALIGNMENT
+
+
+def test_empty_batch_is_noop():
+    assert _dw(_prob(N=0), ptrs=(0, 0, 0)) == OK
+    assert _pw(_prob(N=0, KH=1, KW=1, ph=0, pw=0), ptrs=(0, 0, 0)) == OK
+
+
+def test_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 4, 4, 8, dtype=torch.bfloat16)
+    w = torch.zeros(8, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        cb.pointwise(x, w)
+    with pytest.raises(ValueError):
+        cb.depthwise(x, torch.zeros(3, 3, 8, dtype=torch.bfloat16), H=4, Wd=4, pad_h=1)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(cb, "_LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(cb, "_lib", None)
+    with pytest.raises(cb.DgradUnavailable):
+        cb.lib()

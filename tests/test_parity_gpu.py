@@ -1,0 +1,219 @@
+"""GPU parity: the CUDA kernels, called through the C ABI, against the fp64 oracle.
+
+Small cases are compared element by element with the oracle over the whole
+output; they span several tiles and ragged tails (M, K and C not multiples of
+the tile sizes, channel counts not multiples of 32, odd image sizes).  The five
+workloads run at full size with the launch configuration the benchmark times;
+there the oracle evaluates a sample of outputs one by one (random points plus
+corners and edges), and every element is also checked against cuDNN in fp32.
+Tolerances are written out in gpu_helpers.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from convolution_backward_b200 import synthetic
+from convolution_backward_b200.synthetic import Problem
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _h():
+    import gpu_helpers
+    return gpu_helpers
+
+
+def P(name, kind, dtype, N, H, W, C, K, KH=1, KW=1, S=1, ph=0, pw=0, seed=11):
+    return Problem(name, kind, dtype, N=N, H=H, W=W, C=C, K=K, KH=KH, KW=KW, stride=S, pad_h=ph,
+                   pad_w=pw, seed=seed, w_var=1.0 / (KH * KW) if kind == "depthwise" else 1.0 / K)
+
+
+SMALL = [
+    # pointwise bf16 (tcgen05): ragged M (598 = 4 tiles + 86), ragged K (200 = 3*64 + 8), ragged C
+    P("pw_bf16_ragged", "pointwise", "bf16", 2, 13, 23, 264, 200, seed=21),
+    P("pw_bf16_c40", "pointwise", "bf16", 1, 9, 15, 40, 72, seed=22),
+    P("pw_bf16_k8_c8", "pointwise", "bf16", 3, 5, 7, 8, 8, seed=23),
+    P("pw_bf16_one_row", "pointwise", "bf16", 1, 1, 1, 128, 64, seed=24),
+    P("pw_bf16_256", "pointwise", "bf16", 4, 16, 20, 256, 512, seed=25),
+    # pointwise f32
+    P("pw_f32_ragged", "pointwise", "f32", 1, 7, 11, 20, 12, seed=26),
+    P("pw_f32_wide", "pointwise", "f32", 2, 10, 9, 132, 100, seed=27),
+    # depthwise stride 1 (rotated filter)
+    P("dw3x3", "depthwise", "bf16", 2, 19, 23, 40, 40, 3, 3, 1, 1, 1, seed=31),
+    P("dw31x31", "depthwise", "bf16", 1, 37, 45, 32, 32, 31, 31, 1, 15, 15, seed=32),
+    P("dw51x5", "depthwise", "bf16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=33),
+    P("dw5x51", "depthwise", "bf16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=34),
+    P("dw7x7_nonsame", "depthwise", "bf16", 2, 17, 18, 16, 16, 7, 7, 1, 1, 5, seed=35),
+    P("dw5x5_pw0", "depthwise", "bf16", 1, 12, 14, 48, 48, 5, 5, 1, 2, 0, seed=36),
+    P("dw4x6_even", "depthwise", "bf16", 1, 11, 13, 8, 8, 4, 6, 1, 3, 0, seed=37),
+    P("dw64x64_max", "depthwise", "bf16", 1, 70, 66, 8, 8, 64, 64, 1, 32, 31, seed=38),
+    P("dw1x1", "depthwise", "bf16", 2, 5, 6, 16, 16, 1, 1, 1, 0, 0, seed=39),
+    P("dw13x13", "depthwise", "bf16", 1, 33, 35, 64, 64, 13, 13, 1, 6, 6, seed=40),
+    P("dw3x3_f32", "depthwise", "f32", 2, 9, 10, 12, 12, 3, 3, 1, 1, 1, seed=41),
+    P("dw31x31_f32", "depthwise", "f32", 1, 20, 21, 8, 8, 31, 31, 1, 15, 15, seed=42),
+    P("dw3x3_tiny_image", "depthwise", "bf16", 1, 1, 1, 8, 8, 3, 3, 1, 1, 1, seed=43),
+    # depthwise strided (row streaming)
+    P("dw7x7s2", "depthwise", "bf16", 2, 29, 27, 40, 40, 7, 7, 2, 3, 3, seed=51),
+    P("dw3x3s2", "depthwise", "bf16", 1, 20, 21, 32, 32, 3, 3, 2, 1, 1, seed=52),
+    P("dw5x3s3", "depthwise", "bf16", 1, 22, 19, 16, 16, 5, 3, 3, 2, 1, seed=53),
+    P("dw2x2s3_gaps", "depthwise", "bf16", 1, 14, 13, 8, 8, 2, 2, 3, 0, 0, seed=54),
+    P("dw31x31s2", "depthwise", "bf16", 1, 70, 66, 16, 16, 31, 31, 2, 15, 15, seed=55),
+    P("dw7x7s2_f32", "depthwise", "f32", 1, 15, 16, 12, 12, 7, 7, 2, 3, 3, seed=56),
+    P("dw64x64s1_rowstream", "depthwise", "bf16", 1, 66, 65, 8, 8, 64, 64, 1, 30, 33, seed=57),
+]
+
+ROWSTREAM_AT_S1 = {"dw3x3", "dw7x7_nonsame", "dw51x5", "dw5x5_pw0", "dw4x6_even", "dw64x64s1_rowstream",
+                   "dw3x3_f32", "dw31x31"}
+
+
+def _modes(p):
+    if p.kind == "pointwise":
+        return ["auto"]
+    if p.stride > 1:
+        return ["auto"]
+    if p.name == "dw64x64s1_rowstream":
+        return ["rowstream"]
+    return ["auto", "rowstream"] if p.name in ROWSTREAM_AT_S1 else ["auto"]
+
+
+CASES = [(p, m) for p in SMALL for m in _modes(p)]
+
+
+@pytest.mark.parametrize("p,mode", CASES, ids=[f"{p.name}-{m}" for p, m in CASES])
+def test_small_against_oracle(p, mode):
+    h = _h()
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w, mode=mode))
+    torch.cuda.synchronize()
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/{mode}")
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
+@pytest.mark.parametrize("bn", ["64", "128", "256"])
+def test_pointwise_tile_widths(bn, monkeypatch):
+    """Every tcgen05 tile width (BN = 64, 128, 256) on a ragged problem."""
+    h = _h()
+    monkeypatch.setenv("DGRAD_PW_BN", bn)
+    p = P("pw_bf16_bn", "pointwise", "bf16", 1, 23, 17, 328, 136, seed=60)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"BN={bn}")
+
+
+def _torch_fp32_reference(p, dy, w):
+    """dgrad by cuDNN / cuBLAS in fp32 with TF32 off (full-tensor property check)."""
+    torch.backends.cudnn.allow_tf32 = False
+    torch.backends.cuda.matmul.allow_tf32 = False
+    dyf = dy.float()
+    wf = w.float()
+    if p.kind == "pointwise":
+        return (dyf.reshape(-1, p.K) @ wf).reshape(p.N, p.H, p.W, p.C)
+    wt = wf.permute(2, 0, 1).reshape(p.C, 1, p.KH, p.KW).contiguous()
+    out = torch.nn.grad.conv2d_input((p.N, p.C, p.H, p.W), wt, dyf.permute(0, 3, 1, 2).contiguous(),
+                                     stride=p.stride, padding=(p.pad_h, p.pad_w), groups=p.C)
+    return out.permute(0, 2, 3, 1)
+
+
+FULL = synthetic.all_problems()
+
+
+@pytest.mark.parametrize("p", FULL, ids=[p.name for p in FULL])
+def test_full_size_workloads(p):
+    h = _h()
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = h.run_gpu(p, dy, w)
+    torch.cuda.synchronize()
+    if p.name == "pw_f32_small":
+        got = h.gpu_to_np(out)
+        ref = h.oracle_full(p, inp.dy, inp.w)
+        absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+        h.check(p, got, ref, absref, what=p.name)
+        return
+    pts = h.sample_points(p, 3000)
+    got = out.float()[pts[:, 0], pts[:, 1], pts[:, 2], pts[:, 3]].cpu().numpy().astype(np.float64)
+    ref = h.oracle_points(p, inp.dy, inp.w, pts)
+    absref = h.oracle_points(p, np.abs(inp.dy), np.abs(inp.w), pts)
+    h.check(p, got, ref, absref, what=f"{p.name} sampled")
+    # every element against cuDNN/cuBLAS fp32 with the normwise bar
+    tref = _torch_fp32_reference(p, dy, w)
+    err = (out.float() - tref).abs().max().item()
+    assert err / (tref.abs().max().item() + 1e-6) <= 1e-2
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
+def test_guard_bands_untouched():
+    """dX sits between NaN canary bands; the kernels must write exactly dX."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    for p, mode in [(SMALL[0], "auto"), (SMALL[7], "auto"), (SMALL[7], "rowstream"), (SMALL[20], "auto"),
+                    (SMALL[5], "auto")]:
+        inp = synthetic.make_inputs(p)
+        dy, w = h.to_dev(inp)
+        n = int(np.prod(p.dx_shape))
+        band = 4096
+        dt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+        buf = torch.full((band + n + band,), float("nan"), dtype=dt, device="cuda")
+        out = buf[band:band + n].view(p.dx_shape)
+        h.run_gpu(p, dy, w, mode=mode, out=out)
+        torch.cuda.synchronize()
+        assert torch.isnan(buf[:band]).all() and torch.isnan(buf[band + n:]).all(), p.name
+        assert not torch.isnan(out).any(), p.name
+        cb.check_status()
+
+
+def test_empty_batch_gpu():
+    import convolution_backward_b200 as cb
+    dy = torch.empty((0, 8, 8, 16), dtype=torch.bfloat16, device="cuda")
+    w = torch.randn(3, 3, 16, device="cuda").to(torch.bfloat16)
+    out = cb.depthwise(dy, w, H=8, Wd=8, pad_h=1)
+    assert out.shape == (0, 8, 8, 16)
+    out = cb.pointwise(torch.empty((0, 4, 4, 16), dtype=torch.bfloat16, device="cuda"),
+                       torch.randn(16, 8, device="cuda").to(torch.bfloat16))
+    assert out.shape == (0, 4, 4, 8)
+    cb.check_status()
+
+
+def test_timeout_is_reported_not_hung():
+    """A bounded wait that runs out is reported by dgrad_check_status, and the context stays usable."""
+    import convolution_backward_b200 as cb
+    cb.check_status()
+    cb.selftest_timeout(20_000_000)
+    with pytest.raises(cb.DgradError) as ei:
+        cb.check_status()
+    assert ei.value.status == 5
+    cb.check_status()     # cleared
+    h = _h()
+    p = SMALL[7]
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    h.run_gpu(p, dy, w)
+    cb.check_status()
+
+
+def test_streams_are_respected():
+    """Work enqueued on a side stream is ordered on that stream."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    p = SMALL[4]
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        out = cb.pointwise(dy, w)
+    s.synchronize()
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, h.gpu_to_np(out), ref, absref, what="side stream")
