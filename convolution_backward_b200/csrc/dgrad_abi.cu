@@ -92,6 +92,22 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+// 4-D bf16 NHWC tensor (C innermost), box[4] inner first, no swizzle, zero fill.
+bool encode_nhwc_bf16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H, uint64_t W, uint64_t C,
+                      const unsigned box[4])
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {C, W, H, N};
+    const cuuint64_t strides[3] = {C * 2, W * C * 2, H * W * C * 2};
+    const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int env_int(const char* name, int dflt)
@@ -216,7 +232,19 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     a.status = st->status;
     if (prob->N > 0x7FFFFFFFLL) return DGRAD_ERR_UNSUPPORTED;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    cudaError_t e = mode == DGRAD_DW_ROTATED ? dgrad::launch_dw_rotated(a, cs) : dgrad::launch_dw_rowstream(a, cs);
+    cudaError_t e;
+    unsigned box[4];
+    if (mode == DGRAD_DW_ROTATED) {
+        e = dgrad::launch_dw_rotated(a, cs);
+    } else if (env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box)) {
+        CUtensorMap map;
+        if (!encode_nhwc_bf16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
+                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box))
+            return cuda_fail(cudaErrorInvalidValue);
+        e = dgrad::launch_dw_rowstream_fast(a, map, 0, cs);
+    } else {
+        e = dgrad::launch_dw_rowstream(a, cs);
+    }
     if (e == cudaErrorInvalidConfiguration) return DGRAD_ERR_UNSUPPORTED;
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }

@@ -27,6 +27,7 @@
 // KA is a compile-time parameter; a filter whose A extent has no exact
 // instantiation runs in the next larger one with zero taps appended.
 #include "common.cuh"
+#include "host_util.h"
 #include "launchers.h"
 
 namespace dgrad {
@@ -245,7 +246,7 @@ cudaError_t launch_one(RotParams& p, long long blocks, cudaStream_t stream)
     constexpr int TAT = tat_for<KAI>();
     const size_t smem = static_cast<size_t>(p.RING * p.LA + 2 * KAI) * kPairs * sizeof(float2);
     auto kern = dw_rot_kernel<KAI, TAT, BF16>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p);
     return cudaGetLastError();

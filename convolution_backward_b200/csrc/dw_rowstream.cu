@@ -23,6 +23,7 @@
 // filter, converted to fp32 pairs, sits in shared memory when it fits and is
 // read through the read-only cache otherwise.
 #include "common.cuh"
+#include "host_util.h"
 #include "launchers.h"
 
 namespace dgrad {
@@ -217,7 +218,7 @@ template <bool BF16>
 cudaError_t launch_t(const RsParams& p, long long blocks, size_t smem, cudaStream_t stream)
 {
     auto kern = dw_rowstream_kernel<BF16>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p);
     return cudaGetLastError();

@@ -1,0 +1,334 @@
+// dw_rowstream_fast.cu -- row-streaming depthwise dgrad, register-blocked (bf16).
+//
+// The row-streaming schedule of "channel-packed and large-filter depthwise
+// dgrad" (Technical Details, channel-packed row-streaming dgrad) for strided
+// filters with compile-time KH, KW, S (KH >= S, KW >= S):
+//   - dY rows stream through the kernel in order; dY row ho adds
+//     dY[ho][wo] * W[r][s] into dX row h = ho*S - pad_h + r, column
+//     x = wo*S - pad_w + s;
+//   - once no later dY row can reach a dX row it is final and is written out;
+//     the rows still open are carried in a circular accumulator buffer in
+//     shared memory;
+//   - after the last dY row the open rows are flushed (rows no dY row reaches
+//     come out as zeros).
+//
+// B200 design.
+//   * Work unit (one CTA): image n, 32 channels (16 pairs), a strip of TX dX
+//     columns and a band of BH dX rows.  The band's dY rows (plus the
+//     (KH-S)/S rows of halo above it) stream through a 3-deep TMA ring: each
+//     stage is a 4-D tile [G dY rows][LW dY columns][32 channels] whose
+//     out-of-image part the TMA fills with zeros, which is exactly the padding.
+//   * Thread (pair cp, slot): a slot owns Q dX columns of one column phase
+//     (x + pad_w) mod S, spaced S apart.  All taps reaching that phase have
+//     the same parity s = s0, s0+S, ..., so the thread keeps just those
+//     KH * ceil((KW-s0)/S) filter taps in registers, and Q + NT - 1 dY values
+//     per row feed Q * KH * NT packed FMAs (fma.rn.f32x2 on channel pairs).
+//   * G dY rows are applied per step, all in registers: they touch
+//     (G-1)*S + KH dX rows, of which the first KH-S come in from the shared
+//     accumulator ring (the rows left open by the previous step), the first
+//     G*S are final afterwards and are rounded to bf16 and stored, and the last
+//     KH-S go back to the ring.  Ring entries are private to their thread, so
+//     the ring needs no barriers; one __syncthreads per step recycles the TMA
+//     stage.
+//   * Waits on the TMA barriers are bounded and report a timeout instead of
+//     hanging.
+#include "common.cuh"
+#include "host_util.h"
+#include "launchers.h"
+
+namespace dgrad {
+namespace {
+
+constexpr int kStages = 3;
+constexpr int kMaxThreads = 256;
+
+struct FastParams {
+    __nv_bfloat16* dX;
+    const __nv_bfloat16* filt;
+    int* status;
+    int N, H, W, C, Ho, Wo, ph, pw;
+    int nslot;    // slots per CTA (threads = 16 * nslot), a multiple of 2*S
+    int TX;       // dX columns per strip = nslot * Q
+    int LW;       // dY columns per staged row
+    int BH;       // dX rows per band (multiple of G*S)
+    int nX, nC, nB;
+};
+
+template <int KH, int KW, int S, int Q, int G>
+struct RsGeom {
+    static constexpr int RB = (G - 1) * S + KH;   // dX rows one step touches
+    static constexpr int NF = G * S;              // rows final after a step
+    static constexpr int NC = KH - S;             // rows carried to the next step
+    static constexpr int NTMAX = (KW + S - 1) / S;
+    static_assert(KH >= S && KW >= S, "filter must be at least the stride");
+    static_assert(Q % 2 == 0, "carried rows are stored as column pairs");
+};
+
+// One step with a fixed tap count NT (the thread's column phase has NT taps).
+template <int KH, int KW, int S, int Q, int G, int NT>
+__device__ __forceinline__ void rs_step(float2 (&acc)[RsGeom<KH, KW, S, Q, G>::RB][Q],
+                                        const float2 (&wr)[KH][RsGeom<KH, KW, S, Q, G>::NTMAX],
+                                        const uint32_t* stage, int LW, int cp, int col0)
+{
+    // stage: [G][LW][32 channels] bf16 -> as uint32 pairs: [G][LW][16]
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float2 dv[Q + NT - 1];
+        const uint32_t* row = stage + (g * LW + col0) * 16 + cp;
+#pragma unroll
+        for (int m = 0; m < Q + NT - 1; ++m) dv[m] = bf16x2_to_float2(row[m * 16]);
+#pragma unroll
+        for (int r = 0; r < KH; ++r)
+#pragma unroll
+            for (int q = 0; q < Q; ++q)
+#pragma unroll
+                for (int i = 0; i < NT; ++i)
+                    acc[g * S + r][q] = ffma2(dv[q - i + NT - 1], wr[r][i], acc[g * S + r][q]);
+    }
+}
+
+template <int KH, int KW, int S, int Q, int G>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+    dw_rs_fast_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
+{
+    using Geo = RsGeom<KH, KW, S, Q, G>;
+    constexpr int RB = Geo::RB, NF = Geo::NF, NC = Geo::NC, NTMAX = Geo::NTMAX;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);   // TMA destinations 128-byte aligned
+    const int nthreads = 16 * p.nslot;
+    const int stage_bytes = G * p.LW * 64;                       // 32 bf16 channels = 64 bytes
+    uint32_t* stages = reinterpret_cast<uint32_t*>(smem);
+    float4* carry = reinterpret_cast<float4*>(smem + kStages * stage_bytes);   // [NC][Q/2][nthreads]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes +
+                                                 NC * (Q / 2) * nthreads * sizeof(float4));
+
+    int u = blockIdx.x;
+    const int xblk = u % p.nX;
+    u /= p.nX;
+    const int band = u % p.nB;
+    u /= p.nB;
+    const int cblk = u % p.nC;
+    const int n = u / p.nC;
+
+    const int tid = threadIdx.x;
+    const int cp = tid & 15;
+    const int slot = tid >> 4;
+    const int warp = slot >> 1;
+    const int t = warp % S;                          // column offset of this slot's phase
+    const int j = (warp / S) * 2 + (slot & 1);       // column group within the phase
+    const int x0 = xblk * p.TX;
+    const int c0 = cblk * 32;
+    const int c = c0 + 2 * cp;
+    const bool c_ok = c < p.C;
+    const int s0 = ((x0 + t + p.pw) % S + S) % S;    // first tap reaching this phase
+    const int nt = (KW - s0 + S - 1) / S;            // taps reaching it
+    // dY column of tap (q = 0, i = 0) for this slot, and the strip's first staged column
+    const int e = (x0 + t + p.pw - s0) / S + j * Q;
+    const int wo_start = (x0 + p.pw - (KW - 1)) >= 0 ? (x0 + p.pw - (KW - 1)) / S
+                                                       : -((-(x0 + p.pw - (KW - 1)) + S - 1) / S);
+    const int col0 = e - (nt - 1) - wo_start;        // staged column of dv[0]
+
+    const int h0 = band * p.BH;
+    const int h1 = min(h0 + p.BH, p.H);
+    // first dY row reaching the band (halo rows above it contribute only to discarded rows)
+    int ho_lo = h0 + p.ph - KH + 1;
+    ho_lo = ho_lo <= 0 ? 0 : (ho_lo + S - 1) / S;
+    const int hb0 = ho_lo * S - p.ph;                // first dX row of the first step
+    const int nsteps = (h1 - hb0 + NF - 1) / NF;
+
+    // filter taps of this phase, in registers: wr[r][i] = W[r][s0 + S*i]
+    float2 wr[KH][NTMAX];
+#pragma unroll
+    for (int r = 0; r < KH; ++r)
+#pragma unroll
+        for (int i = 0; i < NTMAX; ++i) {
+            const int s = s0 + S * i;
+            float2 v = make_float2(0.f, 0.f);
+            if (s < KW && c_ok)
+                v = bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + s) * p.C + c)));
+            wr[r][i] = v;
+        }
+    // clear this thread's carried rows
+#pragma unroll
+    for (int r = 0; r < NC; ++r)
+#pragma unroll
+        for (int qh = 0; qh < Q / 2; ++qh) carry[(r * (Q / 2) + qh) * nthreads + tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int step) {
+        const int sidx = step % kStages;
+        mbar_arrive_expect_tx(&full[sidx], stage_bytes);
+        // coordinates (channel, wo, ho, n); out-of-range parts are zero-filled
+        asm volatile(
+            "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(reinterpret_cast<uint8_t*>(stages) +
+                                                                   sidx * stage_bytes)),
+            "l"(reinterpret_cast<uint64_t>(&dy_map)), "r"(smem_u32(&full[sidx])), "r"(c0), "r"(wo_start),
+            "r"(ho_lo + step * G), "r"(n)
+            : "memory");
+    };
+    int issued = 0;   // steps whose tile has been requested (thread 0's count)
+    if (tid == 0) {
+        tma_prefetch_desc(&dy_map);
+        for (; issued < kStages - 1 && issued < nsteps; ++issued) issue(issued);
+    }
+
+    for (int step = 0; step < nsteps; ++step) {
+        if (tid == 0 && issued < nsteps) issue(issued++);
+        float2 acc[RB][Q];
+#pragma unroll
+        for (int r = 0; r < NC; ++r)
+#pragma unroll
+            for (int qh = 0; qh < Q / 2; ++qh) {
+                const float4 v = carry[(r * (Q / 2) + qh) * nthreads + tid];
+                acc[r][2 * qh] = make_float2(v.x, v.y);
+                acc[r][2 * qh + 1] = make_float2(v.z, v.w);
+            }
+#pragma unroll
+        for (int r = NC; r < RB; ++r)
+#pragma unroll
+            for (int q = 0; q < Q; ++q) acc[r][q] = make_float2(0.f, 0.f);
+
+        const int sidx = step % kStages;
+        const bool ok = mbar_wait(&full[sidx], static_cast<uint32_t>((step / kStages) & 1));
+        // every thread leaves together if any of them gave up waiting
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) report_timeout(p.status);
+            break;
+        }
+        const uint32_t* stage = reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(stages) +
+                                                                  sidx * stage_bytes);
+        if (nt == NTMAX)
+            rs_step<KH, KW, S, Q, G, NTMAX>(acc, wr, stage, p.LW, cp, col0);
+        else
+            rs_step<KH, KW, S, Q, G, NTMAX - 1>(acc, wr, stage, p.LW, cp, col0);
+
+        // rows hb .. hb+NF-1 are final
+        const int hb = hb0 + step * NF;
+#pragma unroll
+        for (int i = 0; i < NF; ++i) {
+            const int h = hb + i;
+            if (h >= h0 && h < h1 && c_ok) {
+                __nv_bfloat16* orow = p.dX + ((static_cast<long long>(n) * p.H + h) * p.W) * p.C + c;
+#pragma unroll
+                for (int q = 0; q < Q; ++q) {
+                    const int x = x0 + t + S * (j * Q + q);
+                    if (x < p.W)
+                        *reinterpret_cast<uint32_t*>(orow + static_cast<long long>(x) * p.C) =
+                            float2_to_bf16x2(acc[i][q].x, acc[i][q].y);
+                }
+            }
+        }
+        // rows hb+NF .. hb+RB-1 stay open: back to the ring
+#pragma unroll
+        for (int r = 0; r < NC; ++r)
+#pragma unroll
+            for (int qh = 0; qh < Q / 2; ++qh)
+                carry[(r * (Q / 2) + qh) * nthreads + tid] =
+                    make_float4(acc[NF + r][2 * qh].x, acc[NF + r][2 * qh].y, acc[NF + r][2 * qh + 1].x,
+                                acc[NF + r][2 * qh + 1].y);
+        __syncthreads();   // every thread is done with this stage before it is refilled
+    }
+    // Let every requested tile land before the CTA's shared memory can be reused.
+    if (tid == 0)
+        for (int s = (issued > kStages ? issued - kStages : 0); s < issued; ++s)
+            if (!mbar_wait(&full[s % kStages], static_cast<uint32_t>((s / kStages) & 1))) report_timeout(p.status);
+}
+
+template <int KH, int KW, int S, int Q, int G>
+FastParams plan_fast(const DwArgs& a)
+{
+    using Geo = RsGeom<KH, KW, S, Q, G>;
+    FastParams p{};
+    p.dX = static_cast<__nv_bfloat16*>(a.dX);
+    p.filt = static_cast<const __nv_bfloat16*>(a.filt);
+    p.status = a.status;
+    p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.Ho = a.Ho; p.Wo = a.Wo; p.ph = a.ph; p.pw = a.pw;
+    // strip width: pick the slot count (multiple of 2*S, at most 16) that wastes the fewest columns
+    int best = -1, best_waste = 1 << 30;
+    for (int ns = 16; ns >= 2 * S; ns -= 2 * S) {
+        const int tx = ns * Q;
+        const int strips = (a.W + tx - 1) / tx;
+        const int waste = strips * tx - a.W;
+        if (waste < best_waste) {
+            best_waste = waste;
+            best = ns;
+        }
+    }
+    p.nslot = best;
+    p.TX = best * Q;
+    p.LW = (p.TX - 1 + KW - 1) / S + 2;
+    p.nX = (a.W + p.TX - 1) / p.TX;
+    p.nC = (a.C + 31) / 32;
+    // bands: enough CTAs to fill the machine several times over, rows a multiple of G*S
+    const int nf = Geo::NF;
+    const long long base = static_cast<long long>(a.N) * p.nC * p.nX;
+    const int sms = device_sm_count();
+    const int blocks_per_sm = 4;
+    int nb = static_cast<int>((static_cast<long long>(sms) * blocks_per_sm * 2 + base - 1) / base);
+    nb = max(1, min(nb, (a.H + nf - 1) / nf));
+    int bh = (a.H + nb - 1) / nb;
+    bh = ((bh + nf - 1) / nf) * nf;
+    p.BH = bh;
+    p.nB = (a.H + bh - 1) / bh;
+    return p;
+}
+
+template <int KH, int KW, int S, int Q, int G>
+cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
+{
+    using Geo = RsGeom<KH, KW, S, Q, G>;
+    const FastParams p = plan_fast<KH, KW, S, Q, G>(a);
+    const long long blocks = static_cast<long long>(a.N) * p.nC * p.nX * p.nB;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const int nthreads = 16 * p.nslot;
+    const size_t smem = static_cast<size_t>(kStages) * G * p.LW * 64 +
+                        static_cast<size_t>(Geo::NC) * (Q / 2) * nthreads * sizeof(float4) + kStages * 8 + 128;
+    auto kern = dw_rs_fast_kernel<KH, KW, S, Q, G>;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// The compiled set: (KH, KW, S) -> (Q, G).
+#define DGRAD_RS_FAST_SET(X) \
+    X(7, 7, 2, 4, 2)         \
+    X(5, 5, 2, 4, 2)         \
+    X(3, 3, 2, 4, 4)
+
+bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4])
+{
+    if (!a.bf16) return false;
+#define DGRAD_RS_BOX(kh, kw, s, q, g)                                  \
+    if (a.KH == kh && a.KW == kw && a.S == s) {                         \
+        const FastParams p = plan_fast<kh, kw, s, q, g>(a);            \
+        box[0] = 32; box[1] = static_cast<unsigned>(p.LW); box[2] = g; box[3] = 1; \
+        return true;                                                   \
+    }
+    DGRAD_RS_FAST_SET(DGRAD_RS_BOX)
+#undef DGRAD_RS_BOX
+    return false;
+}
+
+// Returns cudaErrorNotSupported when no specialised instantiation serves the problem.
+cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, int G, cudaStream_t stream)
+{
+    (void)G;
+    if (!a.bf16) return cudaErrorNotSupported;
+#define DGRAD_RS_LAUNCH(kh, kw, s, q, g) \
+    if (a.KH == kh && a.KW == kw && a.S == s) return launch_fast<kh, kw, s, q, g>(a, dy_map, stream);
+    DGRAD_RS_FAST_SET(DGRAD_RS_LAUNCH)
+#undef DGRAD_RS_LAUNCH
+    return cudaErrorNotSupported;
+}
+
+}  // namespace dgrad

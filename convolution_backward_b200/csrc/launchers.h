@@ -44,6 +44,15 @@ cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream);
 // Row-streaming kernel with a circular shared-memory accumulator ring (any S <= 8).
 cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);
 
+// Register-blocked row-streaming kernel for the compiled (KH, KW, S) set, bf16
+// only.  dy_map covers dY as a 4-D bf16 tensor (C, Wo, Ho, N innermost first)
+// with no swizzle.  Returns cudaErrorNotSupported when no instantiation fits.
+cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, int G, cudaStream_t stream);
+
+// Box (inner first) the fast row-streaming kernel loads from dY, or false when
+// the problem has no fast instantiation.
+bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4]);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 

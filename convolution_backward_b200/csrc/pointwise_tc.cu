@@ -24,6 +24,7 @@
 // status word, raises a CTA-wide abort flag, lets in-flight copies and MMAs land
 // and frees its tensor memory before returning.
 #include "common.cuh"
+#include "host_util.h"
 #include "launchers.h"
 
 namespace dgrad {
@@ -261,7 +262,7 @@ cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorM
     using L = PwTcLayout<BN, STAGES>;
     static_assert(L::kAlloc <= 232448, "shared memory budget");
     auto kern = pw_tc_kernel<BN, STAGES>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::kAlloc);
     if (e != cudaSuccess) return e;
     const int num_tiles = static_cast<int>(((a.M + kBM - 1) / kBM) * ((a.C + BN - 1) / BN));
     const int grid = num_tiles < num_sms ? num_tiles : num_sms;

@@ -110,6 +110,35 @@ def test_pointwise_tile_widths(bn, monkeypatch):
     h.check(p, got, ref, absref, what=f"BN={bn}")
 
 
+RS_FAST = [
+    P("rs7x7s2_p3", "depthwise", "bf16", 2, 29, 27, 40, 40, 7, 7, 2, 3, 3, seed=71),
+    P("rs7x7s2_p0", "depthwise", "bf16", 1, 30, 31, 32, 32, 7, 7, 2, 0, 0, seed=72),
+    P("rs7x7s2_p6x1", "depthwise", "bf16", 1, 23, 40, 16, 16, 7, 7, 2, 6, 1, seed=73),
+    P("rs7x7s2_wide", "depthwise", "bf16", 1, 12, 130, 64, 64, 7, 7, 2, 3, 3, seed=74),
+    P("rs7x7s2_tall", "depthwise", "bf16", 1, 117, 9, 8, 8, 7, 7, 2, 3, 2, seed=75),
+    P("rs5x5s2", "depthwise", "bf16", 2, 25, 26, 48, 48, 5, 5, 2, 2, 2, seed=76),
+    P("rs3x3s2_p1", "depthwise", "bf16", 1, 33, 34, 96, 96, 3, 3, 2, 1, 1, seed=77),
+    P("rs3x3s2_p0", "depthwise", "bf16", 1, 16, 17, 32, 32, 3, 3, 2, 0, 0, seed=78),
+    P("rs7x7s2_tiny", "depthwise", "bf16", 1, 2, 3, 8, 8, 7, 7, 2, 3, 3, seed=79),
+]
+
+
+@pytest.mark.parametrize("generic", ["0", "1"])
+@pytest.mark.parametrize("p", RS_FAST, ids=[p.name for p in RS_FAST])
+def test_rowstream_paths(p, generic, monkeypatch):
+    """Strided depthwise through the register-blocked row-streaming kernel and the generic one."""
+    h = _h()
+    monkeypatch.setenv("DGRAD_RS_GENERIC", generic)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/generic={generic}")
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
 def _torch_fp32_reference(p, dy, w):
     """dgrad by cuDNN / cuBLAS in fp32 with TF32 off (full-tensor property check)."""
     torch.backends.cudnn.allow_tf32 = False
