@@ -8,6 +8,7 @@
 // probe used to measure the fp32 roofline.
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -180,12 +181,22 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     if (dtype == DGRAD_F32) {
         e = dgrad::launch_pointwise_f32(a, cs);
     } else {
-        const int bn = env_int("DGRAD_PW_BN", prob->C <= 64 ? 64 : 128);
         CUtensorMap map_a, map_b;
         if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->K), 64, 128) ||
             !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(prob->K), static_cast<uint64_t>(prob->C), 64, 64))
             return cuda_fail(cudaErrorInvalidValue);
-        e = dgrad::launch_pointwise_tc(a, map_a, map_b, bn, st->sms, cs);
+        // Resident-W kernel when it applies (DGRAD_PW_MODE=stream forces the streaming kernel).
+        const char* mode = getenv("DGRAD_PW_MODE");
+        const bool want_stream = mode && strcmp(mode, "stream") == 0;
+        if (!want_stream && dgrad::pointwise_tc_resident_ok(a, st->sms)) {
+            CUtensorMap map_d;
+            if (!encode_2d_bf16(&map_d, dX, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->C), 64, 128))
+                return cuda_fail(cudaErrorInvalidValue);
+            e = dgrad::launch_pointwise_tc_resident(a, map_a, map_b, map_d, st->sms, cs);
+        } else {
+            const int bn = env_int("DGRAD_PW_BN", prob->C <= 64 ? 64 : 128);
+            e = dgrad::launch_pointwise_tc(a, map_a, map_b, bn, st->sms, cs);
+        }
     }
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
@@ -234,7 +245,16 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     unsigned box[4];
-    if (mode == DGRAD_DW_ROTATED) {
+    const char* rk = getenv("DGRAD_ROT_KERNEL");
+    const bool force_line = rk && strcmp(rk, "line") == 0;
+    if (mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box)) {
+        // small filters: one halo tile per CTA
+        CUtensorMap map;
+        if (!encode_nhwc_bf16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
+                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box))
+            return cuda_fail(cudaErrorInvalidValue);
+        e = dgrad::launch_dw_tile(a, map, cs);
+    } else if (mode == DGRAD_DW_ROTATED) {
         e = dgrad::launch_dw_rotated(a, cs);
     } else if (env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box)) {
         CUtensorMap map;

@@ -30,6 +30,8 @@
 #include "host_util.h"
 #include "launchers.h"
 
+#include <cstdlib>
+
 namespace dgrad {
 namespace {
 
@@ -109,68 +111,74 @@ __global__ void __launch_bounds__(kThreads)
     const T* __restrict__ wg = static_cast<const T*>(p.filt);
     T* __restrict__ dx = static_cast<T*>(p.dX) + static_cast<long long>(n) * p.out_sN;
 
+    // Fill plan, fixed for the whole CTA: item k of this thread is dY position
+    // pos = it / kPerPos of a line, channel chunk ch = it % kPerPos (it = tid + k*256).
+    // Only the line index changes from step to step.
     const int line_items = p.LA * Ch::kPerPos;
+    int goff[kMaxPF];        // element offset inside a dY line (position and channel)
+    int soff[kMaxPF];        // float2 offset inside a ring line
+    uint32_t vmask = 0;      // bit k: item k lies inside the image along A and inside C
+    uint32_t imask = 0;      // bit k: item k exists
+#pragma unroll
+    for (int k = 0; k < kMaxPF; ++k) {
+        const int it = tid + k * kThreads;
+        const int pos = it / Ch::kPerPos;
+        const int ch = it - pos * Ch::kPerPos;
+        const int ia = ia0 + pos;
+        const int c = c0 + ch * Ch::kElems;
+        goff[k] = static_cast<int>(ia * p.in_sA) + c;
+        soff[k] = pos * kPairs + ch * Ch::kPairs;
+        if (it < line_items) {
+            imask |= 1u << k;
+            if (ia >= 0 && ia < p.IA && c < p.C) vmask |= 1u << k;
+        }
+    }
+    constexpr int kWItems = KAI * Ch::kPerPos;
+    constexpr int kWPF = (kWItems + kThreads - 1) / kThreads;
+    int wgoff[kWPF];
+    int wsoff[kWPF];
+    uint32_t wvmask = 0, wimask = 0;
+#pragma unroll
+    for (int k = 0; k < kWPF; ++k) {
+        const int it = tid + k * kThreads;
+        const int ia = it / Ch::kPerPos;
+        const int ch = it - ia * Ch::kPerPos;
+        const int c = c0 + ch * Ch::kElems;
+        // tap ia of a rotated filter line is W[B index KB-1-jb][A index KA-1-ia]
+        wgoff[k] = (p.KA - 1 - ia) * p.w_sA + c;
+        wsoff[k] = ia * kPairs + ch * Ch::kPairs;
+        if (it < kWItems) {
+            wimask |= 1u << k;
+            if (ia < p.KA && c < p.C) wvmask |= 1u << k;
+        }
+    }
 
     auto fetch_line = [&](int i, uint4 (&pf)[kMaxPF]) {
         const int ib = ib0 + i;
-        const bool row_ok = ib >= 0 && ib < p.IB;
+        const uint32_t m = (ib >= 0 && ib < p.IB) ? vmask : 0u;
+        const T* base = dy + static_cast<long long>(ib) * p.in_sB;
 #pragma unroll
-        for (int k = 0; k < kMaxPF; ++k) {
-            const int it = tid + k * kThreads;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (it < line_items && row_ok) {
-                const int pos = it / Ch::kPerPos;
-                const int ch = it - pos * Ch::kPerPos;
-                const int ia = ia0 + pos;
-                const int c = c0 + ch * Ch::kElems;
-                if (ia >= 0 && ia < p.IA && c < p.C)
-                    v = __ldg(reinterpret_cast<const uint4*>(dy + ib * p.in_sB + ia * p.in_sA + c));
-            }
-            pf[k] = v;
-        }
+        for (int k = 0; k < kMaxPF; ++k)
+            pf[k] = (m >> k) & 1u ? __ldg(reinterpret_cast<const uint4*>(base + goff[k])) : make_uint4(0u, 0u, 0u, 0u);
     };
-    auto store_line = [&](int i, const uint4 (&pf)[kMaxPF]) {
-        float2* dst = ring + (i % p.RING) * p.LA * kPairs;
+    auto store_line = [&](int slot_idx, const uint4 (&pf)[kMaxPF]) {
+        float2* dst = ring + slot_idx * p.LA * kPairs;
 #pragma unroll
-        for (int k = 0; k < kMaxPF; ++k) {
-            const int it = tid + k * kThreads;
-            if (it < line_items) {
-                const int pos = it / Ch::kPerPos;
-                const int ch = it - pos * Ch::kPerPos;
-                chunk_to_pairs<BF16>(pf[k], dst + pos * kPairs + ch * Ch::kPairs);
-            }
-        }
+        for (int k = 0; k < kMaxPF; ++k)
+            if ((imask >> k) & 1u) chunk_to_pairs<BF16>(pf[k], dst + soff[k]);
     };
-    // Rotated filter line jb: tap ia of the line is W[B index KB-1-jb][A index KA-1-ia].
-    constexpr int kWItems = KAI * Ch::kPerPos;
-    constexpr int kWPF = (kWItems + kThreads - 1) / kThreads;
     auto fetch_wline = [&](int jb, uint4 (&pw)[kWPF]) {
+        const T* base = wg + (p.KB - 1 - jb) * p.w_sB;
 #pragma unroll
-        for (int k = 0; k < kWPF; ++k) {
-            const int it = tid + k * kThreads;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (it < kWItems) {
-                const int ia = it / Ch::kPerPos;
-                const int ch = it - ia * Ch::kPerPos;
-                const int c = c0 + ch * Ch::kElems;
-                if (ia < p.KA && c < p.C)
-                    v = __ldg(reinterpret_cast<const uint4*>(wg + (p.KB - 1 - jb) * p.w_sB +
-                                                             (p.KA - 1 - ia) * p.w_sA + c));
-            }
-            pw[k] = v;
-        }
+        for (int k = 0; k < kWPF; ++k)
+            pw[k] = (wvmask >> k) & 1u ? __ldg(reinterpret_cast<const uint4*>(base + wgoff[k]))
+                                       : make_uint4(0u, 0u, 0u, 0u);
     };
     auto store_wline = [&](int jb, const uint4 (&pw)[kWPF]) {
         float2* dst = wbuf + (jb & 1) * KAI * kPairs;
 #pragma unroll
-        for (int k = 0; k < kWPF; ++k) {
-            const int it = tid + k * kThreads;
-            if (it < kWItems) {
-                const int ia = it / Ch::kPerPos;
-                const int ch = it - ia * Ch::kPerPos;
-                chunk_to_pairs<BF16>(pw[k], dst + ia * kPairs + ch * Ch::kPairs);
-            }
-        }
+        for (int k = 0; k < kWPF; ++k)
+            if ((wimask >> k) & 1u) chunk_to_pairs<BF16>(pw[k], dst + wsoff[k]);
     };
 
     // Prologue: the first TB dY lines and filter line 0.
@@ -190,6 +198,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int j = 0; j < TAT; ++j) acc[j] = make_float2(0.f, 0.f);
 
+    int read_slot = line;              // ring slot of dY line (line + jb)
+    int fill_slot = p.TB;              // ring slot of dY line (TB + jb), the one fetched during step jb
     for (int jb = 0; jb < p.KB; ++jb) {
         const bool more = jb + 1 < p.KB;
         uint4 pf[kMaxPF];
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kThreads)
         const float2* wsrc = wbuf + (jb & 1) * KAI * kPairs + cp;
 #pragma unroll
         for (int ia = 0; ia < KAI; ++ia) wr[ia] = wsrc[ia * kPairs];
-        const float2* src = ring + (((line + jb) % p.RING) * p.LA + strip * TAT) * kPairs + cp;
+        const float2* src = ring + (read_slot * p.LA + strip * TAT) * kPairs + cp;
 #pragma unroll
         for (int q = 0; q < TAT + KAI - 1; ++q) {
             const float2 x = src[q * kPairs];
@@ -213,9 +223,11 @@ __global__ void __launch_bounds__(kThreads)
             }
         }
         if (more) {
-            store_line(p.TB + jb, pf);
+            store_line(fill_slot, pf);
             store_wline(jb + 1, pw);
         }
+        if (++read_slot == p.RING) read_slot = 0;
+        if (++fill_slot == p.RING) fill_slot = 0;
         __syncthreads();
     }
 
@@ -239,11 +251,12 @@ constexpr int kInstKA[] = {1, 3, 5, 7, 9, 11, 13, 15, 17, 21, 25, 31, 33, 41, 51
 
 template <int KAI>
 constexpr int tat_for() { return KAI <= 7 ? 8 : 16; }
+template <int KAI>
+constexpr int tat_alt() { return KAI <= 7 ? 16 : 32; }
 
-template <int KAI, bool BF16>
+template <int KAI, int TAT, bool BF16>
 cudaError_t launch_one(RotParams& p, long long blocks, cudaStream_t stream)
 {
-    constexpr int TAT = tat_for<KAI>();
     const size_t smem = static_cast<size_t>(p.RING * p.LA + 2 * KAI) * kPairs * sizeof(float2);
     auto kern = dw_rot_kernel<KAI, TAT, BF16>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
@@ -252,10 +265,9 @@ cudaError_t launch_one(RotParams& p, long long blocks, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-template <int KAI>
+template <int TAT, int KAI>
 void plan_tiles(RotParams& p)
 {
-    constexpr int TAT = tat_for<KAI>();
     int need = (p.OA + TAT - 1) / TAT;
     int ns = 1;
     while (ns < need && ns < 16) ns *= 2;
@@ -269,16 +281,25 @@ void plan_tiles(RotParams& p)
     p.nC = (p.C + kCB - 1) / kCB;
 }
 
-template <int KAI>
-cudaError_t dispatch(RotParams& p, int N, bool bf16, cudaStream_t stream)
+template <int KAI, int TAT>
+cudaError_t dispatch_t(RotParams& p, int N, bool bf16, cudaStream_t stream)
 {
-    plan_tiles<KAI>(p);
+    plan_tiles<TAT, KAI>(p);
     const long long blocks = static_cast<long long>(N) * p.nC * p.nB * p.nA;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const int per_pos = bf16 ? Chunk<true>::kPerPos : Chunk<false>::kPerPos;
     if (p.LA * per_pos > kMaxPF * kThreads) return cudaErrorInvalidConfiguration;
-    return bf16 ? launch_one<KAI, true>(p, blocks, stream) : launch_one<KAI, false>(p, blocks, stream);
+    return bf16 ? launch_one<KAI, TAT, true>(p, blocks, stream) : launch_one<KAI, TAT, false>(p, blocks, stream);
+}
+
+// Outputs per thread along A: tat_for<KAI>() by default; DGRAD_ROT_TAT may select tat_alt<KAI>().
+template <int KAI>
+cudaError_t dispatch(RotParams& p, int N, bool bf16, cudaStream_t stream)
+{
+    const char* e = getenv("DGRAD_ROT_TAT");
+    if (e && atoi(e) == tat_alt<KAI>()) return dispatch_t<KAI, tat_alt<KAI>()>(p, N, bf16, stream);
+    return dispatch_t<KAI, tat_for<KAI>()>(p, N, bf16, stream);
 }
 
 }  // namespace

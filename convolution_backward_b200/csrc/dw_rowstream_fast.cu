@@ -15,7 +15,7 @@
 // B200 design.
 //   * Work unit (one CTA): image n, 32 channels (16 pairs), a strip of TX dX
 //     columns and a band of BH dX rows.  The band's dY rows (plus the
-//     (KH-S)/S rows of halo above it) stream through a 3-deep TMA ring: each
+//     (KH-S)/S rows of halo above it) stream through a 6-deep TMA ring: each
 //     stage is a 4-D tile [G dY rows][LW dY columns][32 channels] whose
 //     out-of-image part the TMA fills with zeros, which is exactly the padding.
 //   * Thread (pair cp, slot): a slot owns Q dX columns of one column phase
@@ -36,10 +36,12 @@
 #include "host_util.h"
 #include "launchers.h"
 
+#include <cstdlib>
+
 namespace dgrad {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStages = 6;
 constexpr int kMaxThreads = 256;
 
 struct FastParams {
@@ -77,12 +79,13 @@ __device__ __forceinline__ void rs_step(float2 (&acc)[RsGeom<KH, KW, S, Q, G>::R
         const uint32_t* row = stage + (g * LW + col0) * 16 + cp;
 #pragma unroll
         for (int m = 0; m < Q + NT - 1; ++m) dv[m] = bf16x2_to_float2(row[m * 16]);
+        // taps outermost: consecutive FMAs update different accumulators
 #pragma unroll
-        for (int r = 0; r < KH; ++r)
+        for (int i = 0; i < NT; ++i)
 #pragma unroll
-            for (int q = 0; q < Q; ++q)
+            for (int r = 0; r < KH; ++r)
 #pragma unroll
-                for (int i = 0; i < NT; ++i)
+                for (int q = 0; q < Q; ++q)
                     acc[g * S + r][q] = ffma2(dv[q - i + NT - 1], wr[r][i], acc[g * S + r][q]);
     }
 }
@@ -98,9 +101,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);   // TMA destinations 128-byte aligned
     const int nthreads = 16 * p.nslot;
     const int stage_bytes = G * p.LW * 64;                       // 32 bf16 channels = 64 bytes
+    const int stage_stride = (stage_bytes + 127) & ~127;         // TMA destinations are 128-byte aligned
     uint32_t* stages = reinterpret_cast<uint32_t*>(smem);
-    float4* carry = reinterpret_cast<float4*>(smem + kStages * stage_bytes);   // [NC][Q/2][nthreads]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes +
+    float4* carry = reinterpret_cast<float4*>(smem + kStages * stage_stride);  // [NC][Q/2][nthreads]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * stage_stride +
                                                  NC * (Q / 2) * nthreads * sizeof(float4));
 
     int u = blockIdx.x;
@@ -128,6 +132,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int wo_start = (x0 + p.pw - (KW - 1)) >= 0 ? (x0 + p.pw - (KW - 1)) / S
                                                        : -((-(x0 + p.pw - (KW - 1)) + S - 1) / S);
     const int col0 = e - (nt - 1) - wo_start;        // staged column of dv[0]
+    // store addressing: dX row h of this thread's columns is obase + h*row_elems + xoff[q]
+    const long long row_elems = static_cast<long long>(p.W) * p.C;
+    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+    int xoff[Q];
+    uint32_t xmask = 0;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        const int x = x0 + t + S * (j * Q + q);
+        xoff[q] = x * p.C;
+        if (x < p.W && c_ok) xmask |= 1u << q;
+    }
 
     const int h0 = band * p.BH;
     const int h1 = min(h0 + p.BH, p.H);
@@ -167,7 +182,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         asm volatile(
             "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(reinterpret_cast<uint8_t*>(stages) +
-                                                                   sidx * stage_bytes)),
+                                                                   sidx * stage_stride)),
             "l"(reinterpret_cast<uint64_t>(&dy_map)), "r"(smem_u32(&full[sidx])), "r"(c0), "r"(wo_start),
             "r"(ho_lo + step * G), "r"(n)
             : "memory");
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             break;
         }
         const uint32_t* stage = reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(stages) +
-                                                                  sidx * stage_bytes);
+                                                                  sidx * stage_stride);
         if (nt == NTMAX)
             rs_step<KH, KW, S, Q, G, NTMAX>(acc, wr, stage, p.LW, cp, col0);
         else
@@ -213,15 +228,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 #pragma unroll
         for (int i = 0; i < NF; ++i) {
             const int h = hb + i;
-            if (h >= h0 && h < h1 && c_ok) {
-                __nv_bfloat16* orow = p.dX + ((static_cast<long long>(n) * p.H + h) * p.W) * p.C + c;
+            if (h >= h0 && h < h1) {
+                __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
-                for (int q = 0; q < Q; ++q) {
-                    const int x = x0 + t + S * (j * Q + q);
-                    if (x < p.W)
-                        *reinterpret_cast<uint32_t*>(orow + static_cast<long long>(x) * p.C) =
-                            float2_to_bf16x2(acc[i][q].x, acc[i][q].y);
-                }
+                for (int q = 0; q < Q; ++q)
+                    if ((xmask >> q) & 1u)
+                        *reinterpret_cast<uint32_t*>(orow + xoff[q]) = float2_to_bf16x2(acc[i][q].x, acc[i][q].y);
             }
         }
         // rows hb+NF .. hb+RB-1 stay open: back to the ring
@@ -265,12 +277,18 @@ FastParams plan_fast(const DwArgs& a)
     p.LW = (p.TX - 1 + KW - 1) / S + 2;
     p.nX = (a.W + p.TX - 1) / p.TX;
     p.nC = (a.C + 31) / 32;
-    // bands: enough CTAs to fill the machine several times over, rows a multiple of G*S
+    // bands: split the rows only as far as needed to fill one wave of resident
+    // CTAs (longer streams amortise the filter load and the pipeline fill, and
+    // every band re-reads (KH-S)/S halo rows); band rows are a multiple of G*S
     const int nf = Geo::NF;
     const long long base = static_cast<long long>(a.N) * p.nC * p.nX;
     const int sms = device_sm_count();
-    const int blocks_per_sm = 4;
-    int nb = static_cast<int>((static_cast<long long>(sms) * blocks_per_sm * 2 + base - 1) / base);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dw_rs_fast_kernel<KH, KW, S, Q, G>, 16 * p.nslot,
+                                                      0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const long long slots = static_cast<long long>(sms) * per_sm;
+    int nb = static_cast<int>(slots / base);
     nb = max(1, min(nb, (a.H + nf - 1) / nf));
     int bh = (a.H + nb - 1) / nb;
     bh = ((bh + nf - 1) / nf) * nf;
@@ -288,7 +306,7 @@ cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const int nthreads = 16 * p.nslot;
-    const size_t smem = static_cast<size_t>(kStages) * G * p.LW * 64 +
+    const size_t smem = static_cast<size_t>(kStages) * ((G * p.LW * 64 + 127) & ~127) +
                         static_cast<size_t>(Geo::NC) * (Q / 2) * nthreads * sizeof(float4) + kStages * 8 + 128;
     auto kern = dw_rs_fast_kernel<KH, KW, S, Q, G>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
@@ -305,15 +323,29 @@ cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     X(5, 5, 2, 4, 2)         \
     X(3, 3, 2, 4, 4)
 
+// Alternative step depths (G), selected with DGRAD_RS_G for tuning.
+#define DGRAD_RS_ALT_SET(X) \
+    X(7, 7, 2, 4, 1)         \
+    X(5, 5, 2, 4, 1)         \
+    X(3, 3, 2, 4, 2)
+
+static int alt_g()
+{
+    const char* e = getenv("DGRAD_RS_G");
+    return e && *e ? atoi(e) : 0;
+}
+
 bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4])
 {
     if (!a.bf16) return false;
+    const int ga = alt_g();
 #define DGRAD_RS_BOX(kh, kw, s, q, g)                                  \
-    if (a.KH == kh && a.KW == kw && a.S == s) {                         \
+    if (a.KH == kh && a.KW == kw && a.S == s && (ga == 0 || ga == g)) { \
         const FastParams p = plan_fast<kh, kw, s, q, g>(a);            \
         box[0] = 32; box[1] = static_cast<unsigned>(p.LW); box[2] = g; box[3] = 1; \
         return true;                                                   \
     }
+    if (ga != 0) { DGRAD_RS_ALT_SET(DGRAD_RS_BOX) }
     DGRAD_RS_FAST_SET(DGRAD_RS_BOX)
 #undef DGRAD_RS_BOX
     return false;
@@ -324,8 +356,10 @@ cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map,
 {
     (void)G;
     if (!a.bf16) return cudaErrorNotSupported;
+    const int ga = alt_g();
 #define DGRAD_RS_LAUNCH(kh, kw, s, q, g) \
-    if (a.KH == kh && a.KW == kw && a.S == s) return launch_fast<kh, kw, s, q, g>(a, dy_map, stream);
+    if (a.KH == kh && a.KW == kw && a.S == s && (ga == 0 || ga == g)) return launch_fast<kh, kw, s, q, g>(a, dy_map, stream);
+    if (ga != 0) { DGRAD_RS_ALT_SET(DGRAD_RS_LAUNCH) }
     DGRAD_RS_FAST_SET(DGRAD_RS_LAUNCH)
 #undef DGRAD_RS_LAUNCH
     return cudaErrorNotSupported;

@@ -1,0 +1,221 @@
+// dw_tile.cu -- stride-1 depthwise dgrad for small filters (up to 7 x 7), bf16.
+//
+// The rotated-filter correlation of "channel-packed and large-filter depthwise
+// dgrad" (Technical Details, rotated-filter dgrad):
+//     dX[n,h,w,c] = sum_{r'<KH, s'<KW} dY[n, h-P'h+r', w-P'w+s', c] * W[KH-1-r'][KW-1-s'][c],
+// P'h = KH-1-pad_h, P'w = KW-1-pad_w, dY zero off the image.
+//
+// Small filters make this HBM-bound (a few FMAs per byte), so the kernel is
+// built for one memory round trip per CTA and many CTAs in flight:
+//   * a CTA owns an output tile of TH rows x TW columns x 32 channels; one TMA
+//     load brings its whole halo tile [TH+KH-1][TW+KW-1][32] of dY into shared
+//     memory, the out-of-image part zero-filled by the TMA (that is the padding);
+//   * thread (channel pair, row slot, column slot) computes R rows x TAT columns;
+//     it walks the R+KH-1 input rows it needs once, converting each bf16 pair
+//     to fp32 once, and applies every filter row that input row reaches
+//     (packed fma.rn.f32x2, the rotated filter held in registers);
+//   * results are rounded to bf16 and stored straight to dX (16 threads write
+//     64 contiguous bytes).
+#include "common.cuh"
+#include "host_util.h"
+#include "launchers.h"
+
+namespace dgrad {
+namespace {
+
+struct TileParams {
+    __nv_bfloat16* dX;
+    const __nv_bfloat16* filt;
+    int* status;
+    int N, H, W, C, ph, pw;
+    int CS, RS;       // column and row slots per CTA (threads = 16 * CS * RS)
+    int TH, TW;       // output tile
+    int nX, nY, nC;
+};
+
+template <int KH, int KW, int R, int TAT>
+__global__ void __launch_bounds__(256)
+    dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const TileParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
+    const int LWt = p.TW + KW - 1;                        // staged columns
+    const int LHt = p.TH + KH - 1;                        // staged rows
+    const uint32_t tile_bytes = static_cast<uint32_t>(LWt * LHt * 64);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ((tile_bytes + 15u) & ~15u));
+    const uint32_t* tile = reinterpret_cast<const uint32_t*>(smem);   // [LHt][LWt][16] bf16 pairs
+
+    int u = blockIdx.x;
+    const int xblk = u % p.nX;
+    u /= p.nX;
+    const int yblk = u % p.nY;
+    u /= p.nY;
+    const int cblk = u % p.nC;
+    const int n = u / p.nC;
+    const int tid = threadIdx.x;
+    const int cp = tid & 15;
+    const int slot = tid >> 4;
+    const int cs = slot % p.CS;
+    const int rs = slot / p.CS;
+    const int c0 = cblk * 32;
+    const int c = c0 + 2 * cp;
+    const int h0 = yblk * p.TH;
+    const int w0 = xblk * p.TW;
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        tma_prefetch_desc(&dy_map);
+        mbar_arrive_expect_tx(bar, tile_bytes);
+        asm volatile(
+            "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem)),
+            "l"(reinterpret_cast<uint64_t>(&dy_map)), "r"(smem_u32(bar)), "r"(c0),
+            "r"(w0 - (KW - 1 - p.pw)), "r"(h0 - (KH - 1 - p.ph)), "r"(n)
+            : "memory");
+    }
+    // rotated filter taps of this channel pair: wr[r'][s'] = W[KH-1-r'][KW-1-s']
+    float2 wr[KH][KW];
+    const bool c_ok = c < p.C;
+#pragma unroll
+    for (int r = 0; r < KH; ++r)
+#pragma unroll
+        for (int s = 0; s < KW; ++s)
+            wr[r][s] = c_ok ? bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(
+                                  p.filt + ((KH - 1 - r) * KW + (KW - 1 - s)) * p.C + c)))
+                            : make_float2(0.f, 0.f);
+
+    const bool ok = mbar_wait(bar, 0);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) {
+            report_timeout(p.status);
+            mbar_wait(bar, 0);   // let the copy land before the shared memory is released
+        }
+        return;
+    }
+
+    float2 acc[R][TAT];
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < TAT; ++j) acc[i][j] = make_float2(0.f, 0.f);
+
+    const int row0 = rs * R;          // first output row of this thread inside the tile
+    const int col0 = cs * TAT;
+#pragma unroll
+    for (int i = 0; i < R + KH - 1; ++i) {
+        // staged input row row0 + i feeds output rows row0 + ro with filter row r' = i - ro
+        float2 x[TAT + KW - 1];
+        const uint32_t* src = tile + ((row0 + i) * LWt + col0) * 16 + cp;
+#pragma unroll
+        for (int m = 0; m < TAT + KW - 1; ++m) x[m] = bf16x2_to_float2(src[m * 16]);
+        // taps outermost: consecutive FMAs update different accumulators
+#pragma unroll
+        for (int s = 0; s < KW; ++s)
+#pragma unroll
+            for (int ro = 0; ro < R; ++ro) {
+                const int rr = i - ro;
+                if (rr < 0 || rr >= KH) continue;
+#pragma unroll
+                for (int j = 0; j < TAT; ++j) acc[ro][j] = ffma2(x[j + s], wr[rr][s], acc[ro][j]);
+            }
+    }
+
+    if (!c_ok) return;
+    const long long row_elems = static_cast<long long>(p.W) * p.C;
+    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+#pragma unroll
+    for (int ro = 0; ro < R; ++ro) {
+        const int h = h0 + row0 + ro;
+        if (h >= p.H || row0 + ro >= p.TH) continue;
+        __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
+#pragma unroll
+        for (int j = 0; j < TAT; ++j) {
+            const int w = w0 + col0 + j;
+            if (w < p.W && col0 + j < p.TW)
+                *reinterpret_cast<uint32_t*>(orow + static_cast<long long>(w) * p.C) =
+                    float2_to_bf16x2(acc[ro][j].x, acc[ro][j].y);
+        }
+    }
+}
+
+template <int KH, int KW, int R, int TAT>
+TileParams plan_tile(const DwArgs& a)
+{
+    TileParams p{};
+    p.dX = static_cast<__nv_bfloat16*>(a.dX);
+    p.filt = static_cast<const __nv_bfloat16*>(a.filt);
+    p.status = a.status;
+    p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.ph = a.ph; p.pw = a.pw;
+    // columns: as few column slots as cover the row (at most 16), balanced
+    int cs = (a.W + TAT - 1) / TAT;
+    if (cs > 16) {
+        const int strips = (cs + 15) / 16;
+        cs = (cs + strips - 1) / strips;
+    }
+    p.CS = cs;
+    p.TW = cs * TAT;
+    // rows: fill up to 256 threads, but keep enough CTAs in flight
+    int rs = 16 / cs;
+    if (rs < 1) rs = 1;
+    p.RS = rs;
+    p.TH = rs * R;
+    p.nX = (a.W + p.TW - 1) / p.TW;
+    p.nY = (a.H + p.TH - 1) / p.TH;
+    p.nC = (a.C + 31) / 32;
+    return p;
+}
+
+template <int KH, int KW, int R, int TAT>
+cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
+{
+    const TileParams p = plan_tile<KH, KW, R, TAT>(a);
+    const long long blocks = static_cast<long long>(a.N) * p.nC * p.nY * p.nX;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const size_t tile = static_cast<size_t>(p.TW + KW - 1) * (p.TH + KH - 1) * 64;
+    const size_t smem = ((tile + 15) & ~static_cast<size_t>(15)) + 16 + 128;
+    auto kern = dw_tile_kernel<KH, KW, R, TAT>;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(blocks), 16 * p.CS * p.RS, smem, stream>>>(map, p);
+    return cudaGetLastError();
+}
+
+#define DGRAD_TILE_SET(X) \
+    X(3, 3, 2, 8)         \
+    X(5, 5, 2, 8)         \
+    X(7, 7, 2, 8)
+
+}  // namespace
+
+bool dw_tile_box(const DwArgs& a, unsigned box[4])
+{
+    if (!a.bf16 || a.S != 1) return false;
+#define DGRAD_TILE_BOX(kh, kw, r, tat)                                                              \
+    if (a.KH == kh && a.KW == kw) {                                                                 \
+        const TileParams p = plan_tile<kh, kw, r, tat>(a);                                          \
+        box[0] = 32; box[1] = static_cast<unsigned>(p.TW + kw - 1);                                  \
+        box[2] = static_cast<unsigned>(p.TH + kh - 1); box[3] = 1;                                   \
+        return true;                                                                                \
+    }
+    DGRAD_TILE_SET(DGRAD_TILE_BOX)
+#undef DGRAD_TILE_BOX
+    return false;
+}
+
+cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream)
+{
+    if (!a.bf16 || a.S != 1) return cudaErrorNotSupported;
+#define DGRAD_TILE_LAUNCH(kh, kw, r, tat) \
+    if (a.KH == kh && a.KW == kw) return launch_tile<kh, kw, r, tat>(a, dy_map, stream);
+    DGRAD_TILE_SET(DGRAD_TILE_LAUNCH)
+#undef DGRAD_TILE_LAUNCH
+    return cudaErrorNotSupported;
+}
+
+}  // namespace dgrad

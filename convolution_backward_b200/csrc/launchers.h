@@ -28,6 +28,14 @@ cudaError_t launch_pointwise_f32(const PwArgs& a, cudaStream_t stream);
 cudaError_t launch_pointwise_tc(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                 int bn, int num_sms, cudaStream_t stream);
 
+// Resident-W tcgen05 variant: each CTA keeps its 128-column slice of W in
+// shared memory (needs K <= 512 and ceil(C/128) <= num_sms/2) and writes dX
+// through map_d, a 2-D [M][C] bf16 map with a 64 x 128 box and the 128-byte
+// swizzle.  map_b must have a 64 x 64 box as above.
+bool pointwise_tc_resident_ok(const PwArgs& a, int num_sms);
+cudaError_t launch_pointwise_tc_resident(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                         const CUtensorMap& map_d, int num_sms, cudaStream_t stream);
+
 // Depthwise problem (groups = C = K), NHWC, dense.
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;
@@ -40,6 +48,12 @@ struct DwArgs {
 
 // Stride-1 rotated-filter correlation.  Requires S == 1, KH, KW <= 64.
 cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream);
+
+// Stride-1 depthwise for small filters (3x3, 5x5, 7x7; bf16): one TMA halo tile
+// per CTA.  dy_map covers dY as a 4-D bf16 tensor (C, Wo, Ho, N innermost first)
+// with the box dw_tile_box returns.  cudaErrorNotSupported when not compiled.
+bool dw_tile_box(const DwArgs& a, unsigned box[4]);
+cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream);
 
 // Row-streaming kernel with a circular shared-memory accumulator ring (any S <= 8).
 cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);

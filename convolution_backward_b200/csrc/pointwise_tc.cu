@@ -255,6 +255,242 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Resident-W variant (K <= 512).  Each CTA is pinned to one 128-column slice of
+// C and keeps that slice of W (K x 128 bf16, at most 128 KB) in shared memory for
+// its whole life, loaded alongside the first tile's k-blocks; after that only dY
+// streams through the ring (16 KB per k-block), so the L2->SM traffic per tile is
+// the dY tile alone.  The epilogue stages each 128 x 64 bf16 half of the tile in
+// shared memory (128-byte swizzle, conflict-free) and writes it with one TMA
+// bulk tensor store; the store clips the M and C tails.
+constexpr int kResStages = 4;
+constexpr int kResMaxKb = 8;   // K <= 512
+
+struct PwResLayout {
+    static constexpr int kW = 0;                                  // [kb][2 atoms][64 k][128 B]
+    static constexpr int kA = kW + kResMaxKb * 16384;             // [stage][128 rows][128 B]
+    static constexpr int kEpi = kA + kResStages * 16384;          // [2][128 rows][128 B]
+    static constexpr int kBars = kEpi + 2 * 16384;
+    static constexpr int kNumBars = 2 * kResStages + kResMaxKb + 5;
+    static constexpr int kBytes = kBars + kNumBars * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    pw_tc_res_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                     const __grid_constant__ CUtensorMap map_d, int M, int C, int K, int* status)
+{
+    using L = PwResLayout;
+    constexpr int BN = 128;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kResStages;
+    uint64_t* wfull = bars + 2 * kResStages;
+    uint64_t* tfull = wfull + kResMaxKb;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (M + kBM - 1) / kBM;
+    const int num_n = (C + BN - 1) / BN;
+    const int num_kb = (K + kBK - 1) / kBK;
+    const int n_blk = blockIdx.x % num_n;
+    const int first_m = blockIdx.x / num_n;
+    const int m_step = gridDim.x / num_n;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kResStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int k = 0; k < kResMaxKb; ++k) mbar_init(&wfull[k], 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+        tma_prefetch_desc(&map_d);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 2 * BN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_first();   // each dY tile is read by num_n CTAs, then dead
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true, first = true;
+            for (int m = first_m; m < num_m && ok; m += m_step) {
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], 16384);
+                    tma_load_2d_hint(smem + L::kA + stage * 16384, &map_a, &full[stage], kb * kBK, m * kBM,
+                                     num_n > 1 ? policy_evict_last() : pol_a);
+                    if (first) {
+                        mbar_arrive_expect_tx(&wfull[kb], 16384);
+                        tma_load_2d(smem + L::kW + kb * 16384, &map_b, &wfull[kb], n_blk * BN, kb * kBK);
+                        tma_load_2d(smem + L::kW + kb * 16384 + 8192, &map_b, &wfull[kb], n_blk * BN + 64,
+                                    kb * kBK);
+                    }
+                    ++issued;
+                    if (++stage == kResStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                first = false;
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            for (long long i = (issued > kResStages ? issued - kResStages : 0); i < issued; ++i)
+                if (!mbar_wait(&full[i % kResStages], static_cast<uint32_t>((i / kResStages) & 1))) {
+                    report_timeout(status);
+                    *abort_flag = 1;
+                }
+            if (!first)
+                for (int kb = 0; kb < num_kb; ++kb)
+                    if (!mbar_wait(&wfull[kb], 0)) {
+                        report_timeout(status);
+                        *abort_flag = 1;
+                    }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, first = true;
+            for (int m = first_m; m < num_m && ok; m += m_step) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag) || (first && !mbar_wait(&wfull[kb], 0, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + L::kA + stage * 16384);
+                    const uint32_t b_addr = smem_u32(smem + L::kW + kb * 16384);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_f16(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                                 sw128_desc(b_addr + kk * 2048, 8192, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
+                    umma_commit(&empty[stage]);
+                    if (++stage == kResStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                first = false;
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            umma_commit(drain);
+            if (!mbar_wait(drain, 0)) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        // Epilogue: 4 warps; warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows.
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        const bool issuer = warp == 2 && lane == 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int m = first_m; m < num_m; m += m_step) {
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint8_t* buf = smem + L::kEpi + half * 16384;
+                if (issuer) bulk_wait_group_read<1>();     // the last store out of this buffer has read it
+                named_barrier_sync(1, 128);
+                uint32_t v[64];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * 64),
+                                   *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + half * 64 + 32),
+                                   *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tmem_wait_ld();
+                uint8_t* rowp = buf + row * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 o;
+                    o.x = float2_to_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                    o.y = float2_to_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                    o.z = float2_to_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                    o.w = float2_to_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                    *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1, 128);
+                if (issuer) {
+                    tma_store_2d(&map_d, buf, n_blk * BN + half * 64, m * kBM);
+                    bulk_commit_group();
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) {
+            report_timeout(status);
+            *abort_flag = 1;
+        }
+        if (issuer) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, 2 * BN);
+    }
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int num_sms,
                       cudaStream_t stream)
@@ -272,7 +508,38 @@ cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorM
     return cudaGetLastError();
 }
 
+cudaError_t launch_res(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                       const CUtensorMap& map_d, int num_sms, cudaStream_t stream)
+{
+    using L = PwResLayout;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(pw_tc_res_kernel), L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const int num_m = static_cast<int>((a.M + kBM - 1) / kBM);
+    const int num_n = static_cast<int>((a.C + 127) / 128);
+    int per_n = num_sms / num_n;
+    if (per_n > num_m) per_n = num_m;
+    const int grid = per_n * num_n;
+    pw_tc_res_kernel<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, map_d, static_cast<int>(a.M),
+                                                            static_cast<int>(a.C), static_cast<int>(a.K),
+                                                            a.status);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+bool pointwise_tc_resident_ok(const PwArgs& a, int num_sms)
+{
+    return a.K <= 64 * kResMaxKb && (a.C + 127) / 128 <= num_sms / 2;
+}
+
+cudaError_t launch_pointwise_tc_resident(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                         const CUtensorMap& map_d, int num_sms, cudaStream_t stream)
+{
+    if (a.M <= 0) return cudaSuccess;
+    if (!pointwise_tc_resident_ok(a, num_sms)) return cudaErrorInvalidValue;
+    return launch_res(a, map_a, map_b, map_d, num_sms, stream);
+}
 
 cudaError_t launch_pointwise_tc(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int bn,
                                 int num_sms, cudaStream_t stream)

@@ -96,18 +96,54 @@ def test_small_against_oracle(p, mode):
     cb.check_status()
 
 
-@pytest.mark.parametrize("bn", ["64", "128", "256"])
-def test_pointwise_tile_widths(bn, monkeypatch):
-    """Every tcgen05 tile width (BN = 64, 128, 256) on a ragged problem."""
+PW_VARIANTS = [("resident", None), ("stream", "64"), ("stream", "128"), ("stream", "256")]
+
+
+@pytest.mark.parametrize("mode,bn", PW_VARIANTS, ids=[f"{m}-{b}" for m, b in PW_VARIANTS])
+@pytest.mark.parametrize("shape", [(1, 23, 17, 328, 136), (2, 13, 23, 264, 200), (1, 9, 11, 64, 512),
+                                   (3, 7, 5, 8, 8)], ids=["c328k136", "c264k200", "c64k512", "c8k8"])
+def test_pointwise_kernels(mode, bn, shape, monkeypatch):
+    """Both tcgen05 kernels (resident W; streaming W with BN = 64, 128, 256) on ragged problems."""
     h = _h()
-    monkeypatch.setenv("DGRAD_PW_BN", bn)
-    p = P("pw_bf16_bn", "pointwise", "bf16", 1, 23, 17, 328, 136, seed=60)
+    monkeypatch.setenv("DGRAD_PW_MODE", mode)
+    if bn:
+        monkeypatch.setenv("DGRAD_PW_BN", bn)
+    N, H, W, C, K = shape
+    p = P("pw_bf16_var", "pointwise", "bf16", N, H, W, C, K, seed=60)
     inp = synthetic.make_inputs(p)
     dy, w = h.to_dev(inp)
     got = h.gpu_to_np(h.run_gpu(p, dy, w))
     ref = h.oracle_full(p, inp.dy, inp.w)
     absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
-    h.check(p, got, ref, absref, what=f"BN={bn}")
+    h.check(p, got, ref, absref, what=f"{mode}/BN={bn}")
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
+ROT_SMALL = [
+    P("tile3x3", "depthwise", "bf16", 2, 19, 23, 40, 40, 3, 3, 1, 1, 1, seed=81),
+    P("tile3x3_wide", "depthwise", "bf16", 1, 9, 150, 32, 32, 3, 3, 1, 0, 2, seed=82),
+    P("tile5x5", "depthwise", "bf16", 1, 12, 14, 48, 48, 5, 5, 1, 2, 0, seed=83),
+    P("tile7x7", "depthwise", "bf16", 2, 17, 18, 16, 16, 7, 7, 1, 1, 5, seed=84),
+    P("tile7x7_same", "depthwise", "bf16", 1, 33, 31, 72, 72, 7, 7, 1, 3, 3, seed=85),
+    P("tile3x3_1px", "depthwise", "bf16", 1, 1, 1, 8, 8, 3, 3, 1, 1, 1, seed=86),
+]
+
+
+@pytest.mark.parametrize("kernel", ["tile", "line"])
+@pytest.mark.parametrize("p", ROT_SMALL, ids=[p.name for p in ROT_SMALL])
+def test_rotated_small_filter_kernels(p, kernel, monkeypatch):
+    """Small stride-1 filters through the halo-tile kernel and the line kernel."""
+    h = _h()
+    monkeypatch.setenv("DGRAD_ROT_KERNEL", kernel)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/{kernel}")
+    import convolution_backward_b200 as cb
+    cb.check_status()
 
 
 RS_FAST = [
@@ -123,12 +159,18 @@ RS_FAST = [
 ]
 
 
-@pytest.mark.parametrize("generic", ["0", "1"])
+RS_VARIANTS = [("0", ""), ("0", "alt"), ("1", "")]
+
+
+@pytest.mark.parametrize("generic,g", RS_VARIANTS, ids=["fast", "fast-altG", "generic"])
 @pytest.mark.parametrize("p", RS_FAST, ids=[p.name for p in RS_FAST])
-def test_rowstream_paths(p, generic, monkeypatch):
-    """Strided depthwise through the register-blocked row-streaming kernel and the generic one."""
+def test_rowstream_paths(p, generic, g, monkeypatch):
+    """Strided depthwise through the register-blocked row-streaming kernel (both
+    step depths G) and the generic one."""
     h = _h()
     monkeypatch.setenv("DGRAD_RS_GENERIC", generic)
+    if g == "alt":
+        monkeypatch.setenv("DGRAD_RS_G", {7: "1", 5: "1", 3: "2"}[p.KH])
     inp = synthetic.make_inputs(p)
     dy, w = h.to_dev(inp)
     got = h.gpu_to_np(h.run_gpu(p, dy, w))
