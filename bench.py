@@ -247,16 +247,21 @@ KERNEL_SOURCE = {"pointwise": {"bf16": "convolution_backward_b200/csrc/pointwise
                                "f32": "convolution_backward_b200/csrc/pointwise_f32.cu"},
                  "rotated": "convolution_backward_b200/csrc/dw_rotated.cu",
                  "rowstream": "convolution_backward_b200/csrc/dw_rowstream.cu",
-                 "rowstream_fast": "convolution_backward_b200/csrc/dw_rowstream_fast.cu"}
+                 "rowstream_fast": "convolution_backward_b200/csrc/dw_rowstream_fast.cu",
+                 "tile": "convolution_backward_b200/csrc/dw_tile.cu"}
 
 
 def kernel_of(p):
     if p.kind == "pointwise":
         return ("pw_tc_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
+
+    if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
+            and p.KH >= 3:
+        return "dw_tile_kernel", KERNEL_SOURCE["tile"]
     if p.stride == 1:
         return "dw_rot_kernel", KERNEL_SOURCE["rotated"]
     if p.dtype == "bf16" and (p.KH, p.KW, p.stride) in ((7, 7, 2), (5, 5, 2), (3, 3, 2)):
-        return "dw_rs_fast_kernel", KERNEL_SOURCE["rowstream_fast"]
+        return "dw_rs_reg_kernel", KERNEL_SOURCE["rowstream_fast"]
     return "dw_rowstream_kernel", KERNEL_SOURCE["rowstream"]
 
 

@@ -79,7 +79,7 @@ __device__ __forceinline__ void chunk_to_pairs(const uint4& v, float2* dst)
 }
 
 template <int KAI, int TAT, bool BF16>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
     dw_rot_kernel(const RotParams p)
 {
     using Ch = Chunk<BF16>;

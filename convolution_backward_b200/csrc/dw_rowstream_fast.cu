@@ -37,6 +37,7 @@
 #include "launchers.h"
 
 #include <cstdlib>
+#include <cstring>
 
 namespace dgrad {
 namespace {
@@ -252,6 +253,183 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             if (!mbar_wait(&full[s % kStages], static_cast<uint32_t>((s / kStages) & 1))) report_timeout(p.status);
 }
 
+// ---------------------------------------------------------------------------
+// Register-ring variant.  The circular accumulator slots live in registers, as
+// in the pages' design (their accumulator-slot budget is a register budget):
+// acc[RS][Q] with RS >= KH slots, dX row h in slot (h - hb0) mod RS.  Each TMA
+// stage carries GT dY rows and S*GT is a multiple of RS, so inside a stage every
+// slot index is a compile-time constant and the ring "rotates" by renaming;
+// nothing is carried through shared memory and there is one barrier per stage.
+// After dY row t of the band the S rows in slots (S*t .. S*t+S-1) mod RS are
+// final: they are stored (if inside the band) and cleared.
+template <int KH, int KW, int S, int Q, int RS, int GT, int NT>
+__device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 (&wr)[KH][(KW + S - 1) / S],
+                                             const uint32_t* stage, int LW, int cp, int col0, int hb, int h0,
+                                             int h1, __nv_bfloat16* obase, long long row_elems,
+                                             const int (&xoff)[Q], uint32_t xmask)
+{
+    static_assert((S * GT) % RS == 0 && RS >= KH && KH >= S, "ring geometry");
+    // dY row k of the stage, converted to fp32 pairs; row k+1 is loaded while row k computes
+    float2 dv[Q + NT - 1];
+    auto load_row = [&](int k, float2 (&d)[Q + NT - 1]) {
+        const uint32_t* row = stage + (k * LW + col0) * 16 + cp;
+#pragma unroll
+        for (int m = 0; m < Q + NT - 1; ++m) d[m] = bf16x2_to_float2(row[m * 16]);
+    };
+    load_row(0, dv);
+#pragma unroll
+    for (int k = 0; k < GT; ++k) {
+        float2 nx[Q + NT - 1];
+        if (k + 1 < GT) load_row(k + 1, nx);
+        // Filter rows in order r = 0 .. KH-1: rows 0 .. S-1 are the ones that become
+        // final after this dY row, so their last FMAs are issued first.  Rows
+        // r >= KH-S are touched for the first time (their slot was flushed earlier),
+        // so their first tap is a multiply, not an add onto a cleared slot.
+#pragma unroll
+        for (int r = 0; r < KH; ++r)
+#pragma unroll
+            for (int i = 0; i < NT; ++i)
+#pragma unroll
+                for (int q = 0; q < Q; ++q) {
+                    float2& a = acc[(S * k + r) % RS][q];
+                    const float2 x = dv[q - i + NT - 1];
+                    if (r >= KH - S && i == 0)
+                        a = make_float2(x.x * wr[r][0].x, x.y * wr[r][0].y);
+                    else
+                        a = ffma2(x, wr[r][i], a);
+                }
+#pragma unroll
+        for (int i = 0; i < S; ++i) {
+            const int slot = (S * k + i) % RS;
+            const int h = hb + S * k + i;
+            if (h >= h0 && h < h1) {
+                __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
+#pragma unroll
+                for (int q = 0; q < Q; ++q)
+                    if ((xmask >> q) & 1u)
+                        *reinterpret_cast<uint32_t*>(orow + xoff[q]) =
+                            float2_to_bf16x2(acc[slot][q].x, acc[slot][q].y);
+            }
+        }
+        if (k + 1 < GT)
+#pragma unroll
+            for (int m = 0; m < Q + NT - 1; ++m) dv[m] = nx[m];
+    }
+}
+
+template <int KH, int KW, int S, int Q, int RS, int GT>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+    dw_rs_reg_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
+{
+    constexpr int NTMAX = (KW + S - 1) / S;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
+    const int stage_bytes = GT * p.LW * 64;
+    const int stage_stride = (stage_bytes + 127) & ~127;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * stage_stride);
+
+    int u = blockIdx.x;
+    const int xblk = u % p.nX;
+    u /= p.nX;
+    const int band = u % p.nB;
+    u /= p.nB;
+    const int cblk = u % p.nC;
+    const int n = u / p.nC;
+    const int tid = threadIdx.x;
+    const int cp = tid & 15;
+    const int slot = tid >> 4;
+    const int warp = slot >> 1;
+    const int t = warp % S;
+    const int j = (warp / S) * 2 + (slot & 1);
+    const int x0 = xblk * p.TX;
+    const int c0 = cblk * 32;
+    const int c = c0 + 2 * cp;
+    const bool c_ok = c < p.C;
+    const int s0 = (x0 + t + p.pw) % S;
+    const int nt = (KW - s0 + S - 1) / S;
+    const int e = (x0 + t + p.pw - s0) / S + j * Q;
+    const int wo_start = (x0 + p.pw - (KW - 1)) >= 0 ? (x0 + p.pw - (KW - 1)) / S
+                                                       : -((-(x0 + p.pw - (KW - 1)) + S - 1) / S);
+    const int col0 = e - (nt - 1) - wo_start;
+    const long long row_elems = static_cast<long long>(p.W) * p.C;
+    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+    int xoff[Q];
+    uint32_t xmask = 0;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        const int x = x0 + t + S * (j * Q + q);
+        xoff[q] = x * p.C;
+        if (x < p.W && c_ok) xmask |= 1u << q;
+    }
+    const int h0 = band * p.BH;
+    const int h1 = min(h0 + p.BH, p.H);
+    int ho_lo = h0 + p.ph - KH + 1;
+    ho_lo = ho_lo <= 0 ? 0 : (ho_lo + S - 1) / S;
+    const int hb0 = ho_lo * S - p.ph;
+    const int nrows = (h1 - hb0 + S - 1) / S;          // dY rows until every band row is final
+    const int nstages = (nrows + GT - 1) / GT;
+
+    float2 wr[KH][NTMAX];
+#pragma unroll
+    for (int r = 0; r < KH; ++r)
+#pragma unroll
+        for (int i = 0; i < NTMAX; ++i) {
+            const int sx = s0 + S * i;
+            wr[r][i] = (sx < KW && c_ok)
+                           ? bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + sx) * p.C + c)))
+                           : make_float2(0.f, 0.f);
+        }
+    if (tid == 0) {
+        for (int sidx = 0; sidx < kStages; ++sidx) mbar_init(&full[sidx], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int st) {
+        const int sidx = st % kStages;
+        mbar_arrive_expect_tx(&full[sidx], stage_bytes);
+        asm volatile(
+            "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem + sidx * stage_stride)),
+            "l"(reinterpret_cast<uint64_t>(&dy_map)), "r"(smem_u32(&full[sidx])), "r"(c0), "r"(wo_start),
+            "r"(ho_lo + st * GT), "r"(n)
+            : "memory");
+    };
+    int issued = 0;
+    if (tid == 0) {
+        tma_prefetch_desc(&dy_map);
+        for (; issued < kStages - 1 && issued < nstages; ++issued) issue(issued);
+    }
+
+    float2 acc[RS][Q];
+#pragma unroll
+    for (int i = 0; i < RS; ++i)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) acc[i][q] = make_float2(0.f, 0.f);
+
+    for (int st = 0; st < nstages; ++st) {
+        if (tid == 0 && issued < nstages) issue(issued++);
+        const int sidx = st % kStages;
+        const bool ok = mbar_wait(&full[sidx], static_cast<uint32_t>((st / kStages) & 1));
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) report_timeout(p.status);
+            break;
+        }
+        const uint32_t* stage = reinterpret_cast<const uint32_t*>(smem + sidx * stage_stride);
+        const int hb = hb0 + st * GT * S;
+        if (nt == NTMAX)
+            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
+                                                      row_elems, xoff, xmask);
+        else
+            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX - 1>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
+                                                          row_elems, xoff, xmask);
+        __syncthreads();
+    }
+    if (tid == 0)
+        for (int sx = (issued > kStages ? issued - kStages : 0); sx < issued; ++sx)
+            if (!mbar_wait(&full[sx % kStages], static_cast<uint32_t>((sx / kStages) & 1))) report_timeout(p.status);
+}
+
 template <int KH, int KW, int S, int Q, int G>
 FastParams plan_fast(const DwArgs& a)
 {
@@ -315,7 +493,36 @@ cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     return cudaGetLastError();
 }
 
+template <int KH, int KW, int S, int Q, int RS, int GT>
+cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
+{
+    // plan as the shared-ring kernel with G = GT (band rows a multiple of S*GT)
+    FastParams p = plan_fast<KH, KW, S, Q, GT>(a);
+    const long long blocks = static_cast<long long>(a.N) * p.nC * p.nX * p.nB;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const int nthreads = 16 * p.nslot;
+    const size_t smem = static_cast<size_t>(kStages) * ((GT * p.LW * 64 + 127) & ~127) + kStages * 8 + 128;
+    auto kern = dw_rs_reg_kernel<KH, KW, S, Q, RS, GT>;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+// Register-ring set: (KH, KW, S) -> (Q, ring slots RS, dY rows per stage GT).
+#define DGRAD_RS_REG_SET(X) \
+    X(7, 7, 2, 4, 8, 4)     \
+    X(5, 5, 2, 4, 8, 4)     \
+    X(3, 3, 2, 4, 4, 4)
+
+static bool use_reg_ring()
+{
+    const char* e = getenv("DGRAD_RS_KERNEL");
+    return !(e && strcmp(e, "smem") == 0);
+}
 
 // The compiled set: (KH, KW, S) -> (Q, G).
 #define DGRAD_RS_FAST_SET(X) \
@@ -338,6 +545,17 @@ static int alt_g()
 bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4])
 {
     if (!a.bf16) return false;
+    if (use_reg_ring()) {
+#define DGRAD_RS_REG_BOX(kh, kw, s, q, rs, gt)                                                     \
+        if (a.KH == kh && a.KW == kw && a.S == s) {                                                 \
+            const FastParams p = plan_fast<kh, kw, s, q, gt>(a);                                    \
+            box[0] = 32; box[1] = static_cast<unsigned>(p.LW); box[2] = gt; box[3] = 1;            \
+            return true;                                                                            \
+        }
+        DGRAD_RS_REG_SET(DGRAD_RS_REG_BOX)
+#undef DGRAD_RS_REG_BOX
+        return false;
+    }
     const int ga = alt_g();
 #define DGRAD_RS_BOX(kh, kw, s, q, g)                                  \
     if (a.KH == kh && a.KW == kw && a.S == s && (ga == 0 || ga == g)) { \
@@ -356,6 +574,13 @@ cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map,
 {
     (void)G;
     if (!a.bf16) return cudaErrorNotSupported;
+    if (use_reg_ring()) {
+#define DGRAD_RS_REG_LAUNCH(kh, kw, s, q, rs, gt) \
+        if (a.KH == kh && a.KW == kw && a.S == s) return launch_reg<kh, kw, s, q, rs, gt>(a, dy_map, stream);
+        DGRAD_RS_REG_SET(DGRAD_RS_REG_LAUNCH)
+#undef DGRAD_RS_REG_LAUNCH
+        return cudaErrorNotSupported;
+    }
     const int ga = alt_g();
 #define DGRAD_RS_LAUNCH(kh, kw, s, q, g) \
     if (a.KH == kh && a.KW == kw && a.S == s && (ga == 0 || ga == g)) return launch_fast<kh, kw, s, q, g>(a, dy_map, stream);

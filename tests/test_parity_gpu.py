@@ -159,16 +159,18 @@ RS_FAST = [
 ]
 
 
-RS_VARIANTS = [("0", ""), ("0", "alt"), ("1", "")]
+RS_VARIANTS = [("0", "reg", ""), ("0", "smem", ""), ("0", "smem", "alt"), ("1", "", "")]
 
 
-@pytest.mark.parametrize("generic,g", RS_VARIANTS, ids=["fast", "fast-altG", "generic"])
+@pytest.mark.parametrize("generic,kern,g", RS_VARIANTS, ids=["reg-ring", "smem-ring", "smem-ring-altG", "generic"])
 @pytest.mark.parametrize("p", RS_FAST, ids=[p.name for p in RS_FAST])
-def test_rowstream_paths(p, generic, g, monkeypatch):
-    """Strided depthwise through the register-blocked row-streaming kernel (both
-    step depths G) and the generic one."""
+def test_rowstream_paths(p, generic, kern, g, monkeypatch):
+    """Strided depthwise through every row-streaming kernel: accumulator ring in
+    registers, ring in shared memory (both step depths G), and the generic one."""
     h = _h()
     monkeypatch.setenv("DGRAD_RS_GENERIC", generic)
+    if kern:
+        monkeypatch.setenv("DGRAD_RS_KERNEL", kern)
     if g == "alt":
         monkeypatch.setenv("DGRAD_RS_G", {7: "1", 5: "1", 3: "2"}[p.KH])
     inp = synthetic.make_inputs(p)
