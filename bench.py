@@ -253,8 +253,7 @@ KERNEL_SOURCE = {"pointwise": {"bf16": "convolution_backward_b200/csrc/pointwise
 
 def kernel_of(p):
     if p.kind == "pointwise":
-        return ("pw_tc_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
-
+        return ("pw_tc_pair_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
     if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
             and p.KH >= 3:
         return "dw_tile_kernel", KERNEL_SOURCE["tile"]

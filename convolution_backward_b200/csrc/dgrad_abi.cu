@@ -185,10 +185,18 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
         if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->K), 64, 128) ||
             !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(prob->K), static_cast<uint64_t>(prob->C), 64, 64))
             return cuda_fail(cudaErrorInvalidValue);
-        // Resident-W kernel when it applies (DGRAD_PW_MODE=stream forces the streaming kernel).
+        // Kernel choice: the SM-pair kernel by default (256-column pair tiles when C > 128);
+        // DGRAD_PW_MODE = resident | stream selects the one-SM kernels.
         const char* mode = getenv("DGRAD_PW_MODE");
         const bool want_stream = mode && strcmp(mode, "stream") == 0;
-        if (!want_stream && dgrad::pointwise_tc_resident_ok(a, st->sms)) {
+        const bool want_resident = mode && strcmp(mode, "resident") == 0;
+        if (!want_stream && !want_resident) {
+            CUtensorMap map_d;
+            if (!encode_2d_bf16(&map_d, dX, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->C), 64, 128))
+                return cuda_fail(cudaErrorInvalidValue);
+            const int bn = env_int("DGRAD_PW_BN", prob->C > 128 ? 256 : 128);
+            e = dgrad::launch_pointwise_tc_pair(a, map_a, map_b, map_d, bn, st->sms, cs);
+        } else if (want_resident && dgrad::pointwise_tc_resident_ok(a, st->sms)) {
             CUtensorMap map_d;
             if (!encode_2d_bf16(&map_d, dX, static_cast<uint64_t>(M), static_cast<uint64_t>(prob->C), 64, 128))
                 return cuda_fail(cudaErrorInvalidValue);

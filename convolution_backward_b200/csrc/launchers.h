@@ -36,6 +36,12 @@ bool pointwise_tc_resident_ok(const PwArgs& a, int num_sms);
 cudaError_t launch_pointwise_tc_resident(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                          const CUtensorMap& map_d, int num_sms, cudaStream_t stream);
 
+// SM-pair tcgen05 variant (cta_group::2, clusters of two CTAs): 256 x bn tiles
+// (bn = 256 or 128), each CTA holding 128 dY rows and bn/2 W columns per
+// k-block.  Maps as for the resident variant.
+cudaError_t launch_pointwise_tc_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                     const CUtensorMap& map_d, int bn, int num_sms, cudaStream_t stream);
+
 // Depthwise problem (groups = C = K), NHWC, dense.
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;

@@ -491,6 +491,248 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// SM-pair variant (cta_group::2).  Two CTAs of a cluster compute one 256 x 256
+// tile of dX: each holds 128 rows of the dY tile and 128 columns of the W tile
+// in its own shared memory, the rank-0 CTA issues tcgen05.mma.cta_group::2
+// (M = 256, N = 256, K = 16), and each CTA's tensor memory receives its 128 rows
+// x 256 columns of the accumulator.  Per k-block each SM loads 32 KB for a
+// 128 x 256 slab of output, half the operand bytes per output of a one-SM tile,
+// which is what bounds this memory-streaming GEMM.
+//   * both CTAs' TMA loads complete on the rank-0 CTA's "full" barrier, whose
+//     expected byte count (both halves) the rank-0 producer posts;
+//   * the MMA commit is multicast to the "empty" and "tmem full" barriers of
+//     both CTAs; both epilogues arrive on the rank-0 "tmem empty" barrier;
+//   * the epilogue stages 128 x 64 bf16 chunks in shared memory (128-byte
+//     swizzle) and stores them with TMA, which clips the M and C tails;
+//   * cluster barriers order barrier initialisation before any remote arrive
+//     and keep both CTAs alive until all cross-CTA traffic has landed.
+// BN is the pair tile width (256 or 128); each CTA holds BN/2 columns of W.
+template <int BN, int STAGES>
+struct PwPairLayout {
+    static constexpr int kBHalf = (BN / 2) * kBK * 2;         // this CTA's W columns, one k-block
+    static constexpr int kStage = 16384 + kBHalf;            // A 16 KB + W half
+    static constexpr int kA = 0;
+    static constexpr int kEpi = STAGES * kStage;             // 2 x 16 KB staging
+    static constexpr int kBars = kEpi + 2 * 16384;
+    static constexpr int kNumBars = 2 * STAGES + 5;
+    static constexpr int kBytes = kBars + kNumBars * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    pw_tc_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_d, int M, int C, int K, int* status)
+{
+    using L = PwPairLayout<BN, STAGES>;
+    constexpr int kPairStages = STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* full = bars;                      // used in the rank-0 CTA
+    uint64_t* empty = bars + kPairStages;       // each CTA's own
+    uint64_t* tfull = bars + 2 * kPairStages;   // each CTA's own
+    uint64_t* tempty = tfull + 2;               // used in the rank-0 CTA (256 arrivals)
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const uint32_t rank = cluster_ctarank();
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (M + 255) / 256;
+    const int num_n = (C + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + kBK - 1) / kBK;
+    const int pair = blockIdx.x >> 1;
+    const int num_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 256);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+        tma_prefetch_desc(&map_d);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 2 * BN);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();                              // barriers of both CTAs exist before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t full0 = leader_addr(&full[0]);
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                const int m_blk = t / num_n;
+                const int n_blk = t - m_blk * num_n;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStage);
+                    uint8_t* a_tile = smem + L::kA + stage * L::kStage;
+                    uint8_t* b_tile = a_tile + 16384;
+                    const uint32_t fb = full0 + static_cast<uint32_t>(stage * 8);
+                    tma_load_2d_pair(a_tile, &map_a, fb, kb * kBK, m_blk * 256 + static_cast<int>(rank) * 128);
+                    const int ncol = n_blk * BN + static_cast<int>(rank) * (BN / 2);
+#pragma unroll
+                    for (int j = 0; j < BN / 128; ++j)
+                        tma_load_2d_pair(b_tile + j * 8192, &map_b, fb, ncol + j * 64, kb * kBK);
+                    ++issued;
+                    if (++stage == kPairStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            // the last loads of this CTA land before it may exit: wait until the MMAs
+            // that read them have released the stages (multicast commit)
+            for (long long i = (issued > kPairStages ? issued - kPairStages : 0); i < issued; ++i)
+                if (!mbar_wait(&empty[i % kPairStages], static_cast<uint32_t>((i / kPairStages) & 1))) {
+                    report_timeout(status);
+                    *abort_flag = 1;
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(256, BN, /*b_mn_major=*/true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+                if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + L::kA + stage * L::kStage);
+                    const uint32_t b_addr = a_addr + 16384;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_f16_pair(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                                      sw128_desc(b_addr + kk * 2048, 8192, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
+                    umma_commit_pair(&empty[stage]);
+                    if (++stage == kPairStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit_pair(&tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            umma_commit_pair(drain);             // same CTA-group as the MMAs it tracks
+            if (!mbar_wait(drain, 0)) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        const bool issuer = warp == 2 && lane == 0;
+        const uint32_t tempty0 = leader_addr(&tempty[0]);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles; t += num_pairs) {
+            const int m_blk = t / num_n;
+            const int n_blk = t - m_blk * num_n;
+            if (!mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int chunk = 0; chunk < BN / 64; ++chunk) {
+                uint8_t* buf = smem + L::kEpi + (chunk & 1) * 16384;
+                if (issuer) bulk_wait_group_read<1>();
+                named_barrier_sync(1, 128);
+                uint32_t v[64];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + chunk * 64),
+                                   *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + chunk * 64 + 32),
+                                   *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tmem_wait_ld();
+                uint8_t* rowp = buf + row * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 o;
+                    o.x = float2_to_bf16x2(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+                    o.y = float2_to_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+                    o.z = float2_to_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+                    o.w = float2_to_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+                    *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1, 128);
+                if (issuer) {
+                    tma_store_2d(&map_d, buf, n_blk * BN + chunk * 64, m_blk * 256 + static_cast<int>(rank) * 128);
+                    bulk_commit_group();
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(acc * 8));   // rank-0 CTA's tmem-empty barrier
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) {
+            report_timeout(status);
+            *abort_flag = 1;
+        }
+        if (issuer) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    cluster_sync();                              // no CTA leaves while its pair still needs it
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, 2 * BN);
+    }
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int num_sms,
                       cudaStream_t stream)
@@ -526,7 +768,50 @@ cudaError_t launch_res(const PwArgs& a, const CUtensorMap& map_a, const CUtensor
     return cudaGetLastError();
 }
 
+template <int BN, int STAGES>
+cudaError_t launch_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                        const CUtensorMap& map_d, int num_sms, cudaStream_t stream)
+{
+    using L = PwPairLayout<BN, STAGES>;
+    static_assert(L::kAlloc <= 232448, "shared memory budget");
+    auto kern = pw_tc_pair_kernel<BN, STAGES>;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const int num_tiles = static_cast<int>(((a.M + 255) / 256) * ((a.C + BN - 1) / BN));
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (at most one per tile)
+    static int max_clusters = 0;
+    if (max_clusters == 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms / 2;
+        max_clusters = n;
+    }
+    int pairs = max_clusters < num_tiles ? max_clusters : num_tiles;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    return cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_d, static_cast<int>(a.M),
+                              static_cast<int>(a.C), static_cast<int>(a.K), a.status);
+}
+
 }  // namespace
+
+cudaError_t launch_pointwise_tc_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                     const CUtensorMap& map_d, int bn, int num_sms, cudaStream_t stream)
+{
+    if (a.M <= 0) return cudaSuccess;
+    if (bn == 256) return launch_pair<256, 6>(a, map_a, map_b, map_d, num_sms, stream);
+    return launch_pair<128, 8>(a, map_a, map_b, map_d, num_sms, stream);
+}
 
 bool pointwise_tc_resident_ok(const PwArgs& a, int num_sms)
 {

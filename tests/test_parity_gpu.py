@@ -96,14 +96,17 @@ def test_small_against_oracle(p, mode):
     cb.check_status()
 
 
-PW_VARIANTS = [("resident", None), ("stream", "64"), ("stream", "128"), ("stream", "256")]
+PW_VARIANTS = [("pair", None), ("resident", None), ("pair", "128"), ("pair", "256"), ("stream", "64"),
+               ("stream", "128"), ("stream", "256")]
 
 
 @pytest.mark.parametrize("mode,bn", PW_VARIANTS, ids=[f"{m}-{b}" for m, b in PW_VARIANTS])
 @pytest.mark.parametrize("shape", [(1, 23, 17, 328, 136), (2, 13, 23, 264, 200), (1, 9, 11, 64, 512),
-                                   (3, 7, 5, 8, 8)], ids=["c328k136", "c264k200", "c64k512", "c8k8"])
+                                   (3, 7, 5, 8, 8), (4, 16, 20, 256, 512)],
+                         ids=["c328k136", "c264k200", "c64k512", "c8k8", "c256k512"])
 def test_pointwise_kernels(mode, bn, shape, monkeypatch):
-    """Both tcgen05 kernels (resident W; streaming W with BN = 64, 128, 256) on ragged problems."""
+    """Every tcgen05 kernel (resident W; SM pair with 256 x 128 and 256 x 256 tiles; streaming W with
+    BN = 64, 128, 256) on ragged problems."""
     h = _h()
     monkeypatch.setenv("DGRAD_PW_MODE", mode)
     if bn:
