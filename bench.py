@@ -56,6 +56,8 @@ def workload_problems(name: str):
         return synthetic.all_problems()
     if name in synthetic.WORKLOADS:
         return synthetic.WORKLOADS[name]
+    if name in synthetic.EXTRA_WORKLOADS:
+        return synthetic.EXTRA_WORKLOADS[name]
     return [synthetic.problem(name)]
 
 
@@ -252,6 +254,8 @@ KERNEL_SOURCE = {"pointwise": {"bf16": "convolution_backward_b200/csrc/pointwise
 
 
 def kernel_of(p):
+    if p.variant == "splitk":
+        return "pw_tc_splitk_kernel", KERNEL_SOURCE["pointwise"]["bf16"]
     if p.kind == "pointwise":
         return ("pw_tc_pair_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
     if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
@@ -277,6 +281,7 @@ def run_ours(args, world, rank, local):
 
     inputs = {p.name: synthetic.make_inputs(p) for p in problems}
     sets = {}
+    workspaces = {}
     for p in problems:
         inp = inputs[p.name]
         if p.dtype == "bf16":
@@ -288,10 +293,15 @@ def run_ours(args, world, rank, local):
         copies = max(2, math.ceil(2 * l2 / p.algorithmic_bytes()) + 1)
         sets[p.name] = [(dy.clone(), w.clone(), torch.empty(p.dx_shape, dtype=dy.dtype, device=dev))
                         for _ in range(copies)]
+        if p.variant == "splitk":
+            nb, _ = cb.splitk_workspace_bytes(p.N, p.H, p.W, p.K, p.C, 0)
+            workspaces[p.name] = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def call(p, dy, w, out):
-        if p.kind == "pointwise":
+        if p.variant == "splitk":
+            cb.pointwise_splitk(dy, w, splits=0, workspace=workspaces[p.name], out=out)
+        elif p.kind == "pointwise":
             cb.pointwise(dy, w, out=out)
         else:
             cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)

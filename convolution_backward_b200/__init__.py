@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["pointwise", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+__all__ = ["pointwise", "pointwise_splitk", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +90,12 @@ def lib():
             L.dgrad_selftest_timeout.restype = ctypes.c_int
             L.dgrad_fma_probe.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
             L.dgrad_fma_probe.restype = ctypes.c_int
+            L.dgrad_pointwise_splitk.argtypes = [P(Problem), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp,
+                                                 ctypes.c_size_t, vp]
+            L.dgrad_pointwise_splitk.restype = ctypes.c_int
+            L.dgrad_pointwise_splitk_workspace.argtypes = [P(Problem), ctypes.c_int, P(ctypes.c_size_t),
+                                                           P(ctypes.c_int)]
+            L.dgrad_pointwise_splitk_workspace.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -150,6 +156,39 @@ def pointwise(dY, W, out=None, stream=None):
     prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
     _check(lib().dgrad_pointwise(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
                                  out.data_ptr(), _stream_ptr(stream)), "dgrad_pointwise")
+    return out
+
+
+def splitk_workspace_bytes(N, H, W, K, C, splits=0):
+    """(bytes, splits) of workspace pointwise_splitk needs (dgrad_pointwise_splitk_workspace)."""
+    prob = Problem(N, H, W, C, K, 1, 1, 1, 0, 0)
+    nb, used = ctypes.c_size_t(), ctypes.c_int()
+    _check(lib().dgrad_pointwise_splitk_workspace(ctypes.byref(prob), int(splits), ctypes.byref(nb),
+                                                  ctypes.byref(used)), "dgrad_pointwise_splitk_workspace")
+    return nb.value, used.value
+
+
+def pointwise_splitk(dY, W, splits=0, workspace=None, out=None, stream=None):
+    """Split-K pointwise dgrad for small M (bf16; dgrad_pointwise_splitk).
+
+    workspace: a caller-owned CUDA tensor of at least splitk_workspace_bytes(...)
+    bytes; allocated here with torch when None."""
+    import torch
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 2 or W.shape[0] != dY.shape[3]:
+        raise ValueError("expected dY (N,H,W,K) and W (K,C)")
+    N, H, Wd, K = dY.shape
+    C = W.shape[1]
+    nbytes, used = splitk_workspace_bytes(N, H, Wd, K, C, splits)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dY.device)
+    if out is None:
+        out = torch.empty((N, H, Wd, C), dtype=dY.dtype, device=dY.device)
+    prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
+    _check(lib().dgrad_pointwise_splitk(ctypes.byref(prob), _dtype_code(dY), int(used), dY.data_ptr(),
+                                        W.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "dgrad_pointwise_splitk")
     return out
 
 

@@ -209,6 +209,76 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 
+// Shared checks for the split-K entry points: pointwise shape class, bf16, the
+// problem extents the kernels index with 32-bit integers.
+static dgrad_status_t splitk_prepare(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
+                                     dgrad::PwArgs* a, int* sms)
+{
+    int64_t Ho = 0, Wo = 0;
+    int pw = 0;
+    dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
+    if (s != DGRAD_OK) return s;
+    if (prob->KH != 1 || prob->KW != 1 || prob->stride != 1 || prob->pad_h != 0 || pw != 0)
+        return DGRAD_ERR_UNSUPPORTED;
+    if (dtype != DGRAD_BF16) return DGRAD_ERR_UNSUPPORTED;
+    if (splits < 0 || splits > 64) return DGRAD_ERR_INVALID;
+    const int64_t M = prob->N * prob->H * prob->W;
+    if (M > 0x7FFFFFFFLL || prob->K > 65536 || prob->C > 65536) return DGRAD_ERR_UNSUPPORTED;
+    if ((prob->K * 2) % 16 || (prob->C * 2) % 16) return DGRAD_ERR_ALIGNMENT;
+    *a = dgrad::PwArgs{M, prob->K, prob->C, nullptr, nullptr, nullptr, nullptr};
+    *sms = 0;
+    return DGRAD_OK;
+}
+
+dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int splits, size_t* bytes,
+                                                int* splits_used)
+{
+    if (!bytes) return DGRAD_ERR_INVALID;
+    dgrad::PwArgs a{};
+    int sms = 0;
+    dgrad_status_t s = splitk_prepare(prob, DGRAD_BF16, splits, &a, &sms);
+    if (s != DGRAD_OK) return s;
+    if (splits == 0) {
+        DeviceState* st = nullptr;
+        s = device_state(&st);
+        if (s != DGRAD_OK) return s;
+        splits = dgrad::pointwise_splitk_auto(a, st->sms);
+    }
+    *bytes = dgrad::pointwise_splitk_workspace_bytes(a, splits);
+    if (splits_used) *splits_used = splits;
+    return DGRAD_OK;
+}
+
+dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits, const void* dY,
+                                      const void* W, void* dX, void* workspace, size_t workspace_bytes,
+                                      void* stream)
+{
+    dgrad::PwArgs a{};
+    int sms = 0;
+    dgrad_status_t s = splitk_prepare(prob, dtype, splits, &a, &sms);
+    if (s != DGRAD_OK) return s;
+    if (a.M == 0) return DGRAD_OK;
+    if (!dY || !W || !dX || !workspace) return DGRAD_ERR_INVALID;
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || !aligned16(workspace)) return DGRAD_ERR_ALIGNMENT;
+    if (splits > 0 && workspace_bytes < dgrad::pointwise_splitk_workspace_bytes(a, splits)) return DGRAD_ERR_INVALID;
+    DeviceState* st = nullptr;
+    s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    if (splits == 0) splits = dgrad::pointwise_splitk_auto(a, st->sms);
+    if (workspace_bytes < dgrad::pointwise_splitk_workspace_bytes(a, splits)) return DGRAD_ERR_INVALID;
+    a.dY = dY;
+    a.W = W;
+    a.dX = dX;
+    a.status = st->status;
+    CUtensorMap map_a, map_b;
+    if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), 64, 128) ||
+        !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.C), 64, 64))
+        return cuda_fail(cudaErrorInvalidValue);
+    cudaError_t e = dgrad::launch_pointwise_tc_splitk(a, map_a, map_b, splits, static_cast<float*>(workspace),
+                                                       st->sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
 dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype, dgrad_dw_mode_t mode,
                                const void* dY, const void* W, void* dX, void* stream)
 {

@@ -271,6 +271,9 @@ void plan_tiles(RotParams& p)
     int need = (p.OA + TAT - 1) / TAT;
     int ns = 1;
     while (ns < need && ns < 16) ns *= 2;
+    // DGRAD_ROT_NS caps the strips per CTA (fewer strips, more lines: less fill per output)
+    const char* e = getenv("DGRAD_ROT_NS");
+    if (e && atoi(e) >= 1 && atoi(e) < ns) ns = atoi(e);
     p.NS = ns;
     p.TB = 16 / ns;
     p.TAC = ns * TAT;

@@ -42,6 +42,14 @@ cudaError_t launch_pointwise_tc_resident(const PwArgs& a, const CUtensorMap& map
 cudaError_t launch_pointwise_tc_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                      const CUtensorMap& map_d, int bn, int num_sms, cudaStream_t stream);
 
+// Split-K tcgen05 variant for small M: partial tiles go to ws (fp32,
+// [splits][M][C]), then a reduction kernel sums them in split order and writes
+// bf16 dX.  pointwise_splitk_auto picks a split count that fills the SMs.
+int pointwise_splitk_auto(const PwArgs& a, int num_sms);
+size_t pointwise_splitk_workspace_bytes(const PwArgs& a, int splits);
+cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                       int splits, float* ws, int num_sms, cudaStream_t stream);
+
 // Depthwise problem (groups = C = K), NHWC, dense.
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;

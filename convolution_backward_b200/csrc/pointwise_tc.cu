@@ -733,6 +733,239 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Split-K variant for small M (few tiles): the K-loop of every (m, n) tile is
+// split into S contiguous ranges of k-blocks.  Work unit (m-block, n-block,
+// split) computes a partial tile and writes it as fp32 to the workspace
+// ws[split][m][c]; a second kernel sums the S partials in split order
+// (deterministic: no atomics, nothing to zero) and rounds to bf16.  Structure
+// as the streaming kernel: TMA producer, MMA issuer, 4 epilogue warps, two TMEM
+// accumulators.
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    pw_tc_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                        float* __restrict__ ws, int M, int C, int K, int S, int* status)
+{
+    using L = PwTcLayout<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kTileBytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (M + kBM - 1) / kBM;
+    const int num_n = (C + BN - 1) / BN;
+    const int num_units = num_m * num_n * S;
+    const int num_kb = (K + kBK - 1) / kBK;
+    const int kb_per = (num_kb + S - 1) / S;
+    auto unit_range = [&](int u, int& m_blk, int& n_blk, int& kb0, int& kb1) {
+        const int ks = u % S;
+        const int t = u / S;
+        m_blk = t / num_n;
+        n_blk = t - m_blk * num_n;
+        kb0 = ks * kb_per;
+        kb1 = min(num_kb, kb0 + kb_per);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, L::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                int m_blk, n_blk, kb0, kb1;
+                unit_range(u, m_blk, n_blk, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+                    uint8_t* a_tile = smem + stage * L::kStageBytes;
+                    uint8_t* b_tile = a_tile + L::kABytes;
+                    tma_load_2d(a_tile, &map_a, &full[stage], kb * kBK, m_blk * kBM);
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tma_load_2d(b_tile + j * 8192, &map_b, &full[stage], n_blk * BN + j * 64, kb * kBK);
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+                if (!mbar_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1))) {
+                    report_timeout(status);
+                    *abort_flag = 1;
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+                int m_blk, n_blk, kb0, kb1;
+                unit_range(u, m_blk, n_blk, kb0, kb1);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
+                    const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_f16(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                                 sw128_desc(b_addr + kk * 2048, 8192, 1024), idesc,
+                                 (kb > kb0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (!ok) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+            umma_commit(drain);
+            if (!mbar_wait(drain, 0)) {
+                report_timeout(status);
+                *abort_flag = 1;
+            }
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            int m_blk, n_blk, kb0, kb1;
+            unit_range(u, m_blk, n_blk, kb0, kb1);
+            const int ks = u % S;
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int m = m_blk * kBM + row;
+            float* out_row = ws + (static_cast<long long>(ks) * M + m) * C;
+#pragma unroll 1
+            for (int chunk = 0; chunk < BN / 32; ++chunk) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(acc * BN + chunk * 32), v);
+                tmem_wait_ld();
+                const int col0 = n_blk * BN + chunk * 32;
+                if (m < M) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int col = col0 + g * 4;
+                        if (col < C)
+                            *reinterpret_cast<uint4*>(out_row + col) =
+                                make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+        if (!ok) {
+            report_timeout(status);
+            *abort_flag = 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, L::kTmemCols);
+    }
+}
+
+// dX[m][c] = bf16(sum over s of ws[s][m][c]), s in increasing order; 8 channels per thread.
+__global__ void __launch_bounds__(256)
+    splitk_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ dX, long long MC, int S)
+{
+    const long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
+    if (i >= MC) return;
+    float4 a = *reinterpret_cast<const float4*>(ws + i);
+    float4 b = *reinterpret_cast<const float4*>(ws + i + 4);
+    for (int s = 1; s < S; ++s) {
+        const float4 x = *reinterpret_cast<const float4*>(ws + s * MC + i);
+        const float4 y = *reinterpret_cast<const float4*>(ws + s * MC + i + 4);
+        a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+        b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    }
+    uint4 o;
+    o.x = float2_to_bf16x2(a.x, a.y);
+    o.y = float2_to_bf16x2(a.z, a.w);
+    o.z = float2_to_bf16x2(b.x, b.y);
+    o.w = float2_to_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4*>(dX + i) = o;
+}
+
 template <int BN, int STAGES>
 cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b, int num_sms,
                       cudaStream_t stream)
@@ -804,6 +1037,45 @@ cudaError_t launch_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtenso
 }
 
 }  // namespace
+
+int pointwise_splitk_auto(const PwArgs& a, int num_sms)
+{
+    const int tiles = static_cast<int>(((a.M + kBM - 1) / kBM) * ((a.C + 127) / 128));
+    const int num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
+    int s = (num_sms + tiles - 1) / tiles;
+    if (s > num_kb) s = num_kb;
+    if (s > 32) s = 32;
+    return s < 1 ? 1 : s;
+}
+
+size_t pointwise_splitk_workspace_bytes(const PwArgs& a, int splits)
+{
+    return static_cast<size_t>(splits) * static_cast<size_t>(a.M) * static_cast<size_t>(a.C) * sizeof(float);
+}
+
+cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                       int splits, float* ws, int num_sms, cudaStream_t stream)
+{
+    if (a.M <= 0) return cudaSuccess;
+    using L = PwTcLayout<128, 6>;
+    auto kern = pw_tc_splitk_kernel<128, 6>;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::kAlloc);
+    if (e != cudaSuccess) return e;
+    const int num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
+    const int kb_per = (num_kb + splits - 1) / splits;
+    const int S = (num_kb + kb_per - 1) / kb_per;   // no empty split
+    const long long units = ((a.M + kBM - 1) / kBM) * ((a.C + 127) / 128) * S;
+    const int grid = static_cast<int>(units < num_sms ? units : num_sms);
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, ws, static_cast<int>(a.M), static_cast<int>(a.C),
+                                                static_cast<int>(a.K), S, a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long MC = a.M * a.C;
+    const long long threads = (MC + 7) / 8;
+    splitk_reduce_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        ws, static_cast<__nv_bfloat16*>(a.dX), MC, S);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pointwise_tc_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                      const CUtensorMap& map_d, int bn, int num_sms, cudaStream_t stream)

@@ -44,6 +44,7 @@ class Problem:
     dy_var: float = 1.0
     w_dist: str = "normal"
     w_var: float = 1.0
+    variant: str = ""    # "splitk": run through the split-K pointwise entry point
 
     @property
     def Ho(self) -> int:
@@ -112,13 +113,22 @@ WORKLOADS: dict[str, list[Problem]] = {
 WORKLOAD_ORDER = ["pw_f32_small", "dw3x3_bf16", "pw_bf16", "dw31x31_bf16",
                   "dw_nonsquare_strided_bf16"]
 
+# Extra workloads outside the benchmark suite (run with --workload NAME).
+EXTRA_WORKLOADS: dict[str, list[Problem]] = {
+    # small M, long K: 16 output tiles, split-K fills the GPU
+    "pw_bf16_smallm_splitk": [Problem("pw_bf16_smallm_splitk", "pointwise", "bf16", N=2, H=14, W=14, C=512,
+                                      K=2048, seed=5, w_var=1.0 / 2048, variant="splitk")],
+    "pw_bf16_smallm": [Problem("pw_bf16_smallm", "pointwise", "bf16", N=2, H=14, W=14, C=512, K=2048,
+                               seed=5, w_var=1.0 / 2048)],
+}
+
 
 def all_problems() -> list[Problem]:
     return [p for name in WORKLOAD_ORDER for p in WORKLOADS[name]]
 
 
 def problem(name: str) -> Problem:
-    for p in all_problems():
+    for p in all_problems() + [q for v in EXTRA_WORKLOADS.values() for q in v]:
         if p.name == name:
             return p
     raise KeyError(name)

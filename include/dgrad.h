@@ -19,7 +19,7 @@
  *     runs as a correlation of dY with the 180-degree rotated filter at padding
  *     KH-1-pad_h rows and KW-1-pad_w columns, filters up to 64 a side, square or
  *     not; stride > 1 runs as a row-streaming kernel whose accumulator rows sit
- *     in a circular shared-memory ring ("channel-packed and large-filter
+ *     in circular slots (registers, or a shared-memory ring) ("channel-packed and large-filter
  *     depthwise dgrad", Technical Details: rotated-filter dgrad and the
  *     channel-packed row-streaming dgrad).
  *
@@ -46,6 +46,7 @@
 #ifndef DGRAD_H
 #define DGRAD_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -86,6 +87,30 @@ typedef enum {
  * DGRAD_F32 runs as an fp32 FMA kernel (no reduced-precision inputs). */
 dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
                                const void* dY, const void* W, void* dX, void* stream);
+
+/* Split-K pointwise dgrad for problems with few output tiles (small M = N*H*W,
+ * long K): each 128 x 128 tile's K-loop is split into `splits` ranges that run
+ * on different SMs; partial tiles are written as fp32 to `workspace` and then
+ * summed in split order (deterministic: no atomics, nothing to zero) and
+ * rounded once to bf16 into dX.  Same shape class and layouts as
+ * dgrad_pointwise; DGRAD_BF16 only (else DGRAD_ERR_UNSUPPORTED).  The pages'
+ * implicit-GEMM dgrad has a split-K mode ("add the pointwise fast path dgrad
+ * was missing", review-fix commit: split-K sub-GEMMs, dX accumulated
+ * atomically).
+ * splits: 1 .. 64, or 0 to let the library choose one that fills the GPU.
+ * workspace: caller-owned device memory, 16-byte aligned, at least the size
+ * dgrad_pointwise_splitk_workspace reports for the same problem and splits;
+ * its contents on entry do not matter and are clobbered.  Too small or null:
+ * DGRAD_ERR_INVALID. */
+dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
+                                      const void* dY, const void* W, void* dX,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes dgrad_pointwise_splitk needs for `splits` (0: the automatic
+ * choice, which is returned in *splits_used when that pointer is non-null).
+ * Queries the current device's SM count for the automatic choice. */
+dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int splits, size_t* bytes,
+                                                int* splits_used);
 
 /* Depthwise dgrad (groups = C; requires K == C, else DGRAD_ERR_UNSUPPORTED).
  * Rotated-filter mode requires stride 1, KH and KW <= 64 and

@@ -149,3 +149,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(cb, "_lib", None)
     with pytest.raises(cb.DgradUnavailable):
         cb.lib()
+
+
+def test_splitk_validation_and_workspace_size():
+    L = cb.lib()
+    p = _prob(N=2, H=14, W=14, C=64, K=256, KH=1, KW=1, ph=0, pw=0)
+    nb = ctypes.c_size_t()
+    used = ctypes.c_int()
+    assert L.dgrad_pointwise_splitk_workspace(ctypes.byref(p), 4, ctypes.byref(nb), ctypes.byref(used)) == OK
+    assert nb.value == 4 * 2 * 14 * 14 * 64 * 4 and used.value == 4
+    assert L.dgrad_pointwise_splitk_workspace(ctypes.byref(p), 65, ctypes.byref(nb), None) == INVALID
+    call = lambda prob, dtype=BF16, splits=4, ws_bytes=1 << 30: L.dgrad_pointwise_splitk(
+        ctypes.byref(prob), dtype, splits, FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+    assert call(p, dtype=F32) == UNSUPPORTED
+    assert call(_prob()) == UNSUPPORTED                     # 3x3 is not pointwise
+    assert call(p, splits=-1) == INVALID
+    assert call(p, ws_bytes=nb.value - 16) == INVALID        # workspace too small
+    assert L.dgrad_pointwise_splitk(ctypes.byref(p), BF16, 4, FAKE, FAKE, FAKE, 0, 1 << 30, None) == INVALID
+    assert L.dgrad_pointwise_splitk(ctypes.byref(p), BF16, 4, FAKE, FAKE, FAKE, FAKE + 4, 1 << 30, None) == ALIGNMENT

@@ -149,6 +149,34 @@ def test_rotated_small_filter_kernels(p, kernel, monkeypatch):
     cb.check_status()
 
 
+SPLITK = [
+    (P("sk_small_m", "pointwise", "bf16", 2, 14, 14, 512, 2048, seed=91), [1, 2, 5, 0]),
+    (P("sk_ragged", "pointwise", "bf16", 1, 7, 9, 136, 1000, seed=92), [3, 16, 0]),
+    (P("sk_one_tile", "pointwise", "bf16", 1, 4, 4, 64, 4096, seed=93), [8, 64, 0]),
+    (P("sk_k_lt_64", "pointwise", "bf16", 3, 5, 5, 264, 40, seed=94), [1, 0]),
+]
+SPLITK_CASES = [(p, s) for p, ss in SPLITK for s in ss]
+
+
+@pytest.mark.parametrize("p,splits", SPLITK_CASES, ids=[f"{p.name}-s{s}" for p, s in SPLITK_CASES])
+def test_pointwise_splitk(p, splits):
+    """Split-K tcgen05 pointwise (NEXT-4): partial tiles in a caller workspace, deterministic reduction."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    nbytes, used = cb.splitk_workspace_bytes(p.N, p.H, p.W, p.K, p.C, splits)
+    ws = torch.full((nbytes // 4 + 4,), float("nan"), dtype=torch.float32, device="cuda")   # contents must not matter
+    out = cb.pointwise_splitk(dy, w, splits=splits, workspace=ws)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/splits={splits}({used})")
+    again = cb.pointwise_splitk(dy, w, splits=splits, workspace=ws)
+    assert torch.equal(out, again)                      # deterministic
+    cb.check_status()
+
+
 RS_FAST = [
     P("rs7x7s2_p3", "depthwise", "bf16", 2, 29, 27, 40, 40, 7, 7, 2, 3, 3, seed=71),
     P("rs7x7s2_p0", "depthwise", "bf16", 1, 30, 31, 32, 32, 7, 7, 2, 0, 0, seed=72),
