@@ -1042,6 +1042,7 @@ int pointwise_splitk_auto(const PwArgs& a, int num_sms)
 {
     const int tiles = static_cast<int>(((a.M + kBM - 1) / kBM) * ((a.C + 127) / 128));
     const int num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
+    if (tiles <= 0) return 1;   // empty batch: nothing to split
     int s = (num_sms + tiles - 1) / tiles;
     if (s > num_kb) s = num_kb;
     if (s > 32) s = 32;

@@ -167,3 +167,11 @@ def test_splitk_validation_and_workspace_size():
     assert call(p, ws_bytes=nb.value - 16) == INVALID        # workspace too small
     assert L.dgrad_pointwise_splitk(ctypes.byref(p), BF16, 4, FAKE, FAKE, FAKE, 0, 1 << 30, None) == INVALID
     assert L.dgrad_pointwise_splitk(ctypes.byref(p), BF16, 4, FAKE, FAKE, FAKE, FAKE + 4, 1 << 30, None) == ALIGNMENT
+
+
+def test_splitk_workspace_empty_batch():
+    L = cb.lib()
+    nb = ctypes.c_size_t(99)
+    p = _prob(N=0, H=14, W=14, C=64, K=256, KH=1, KW=1, ph=0, pw=0)
+    assert L.dgrad_pointwise_splitk_workspace(ctypes.byref(p), 3, ctypes.byref(nb), None) == OK
+    assert nb.value == 0

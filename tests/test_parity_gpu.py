@@ -286,6 +286,9 @@ def test_empty_batch_gpu():
     out = cb.pointwise(torch.empty((0, 4, 4, 16), dtype=torch.bfloat16, device="cuda"),
                        torch.randn(16, 8, device="cuda").to(torch.bfloat16))
     assert out.shape == (0, 4, 4, 8)
+    out = cb.pointwise_splitk(torch.empty((0, 4, 4, 16), dtype=torch.bfloat16, device="cuda"),
+                              torch.randn(16, 8, device="cuda").to(torch.bfloat16))   # automatic split count
+    assert out.shape == (0, 4, 4, 8)
     cb.check_status()
 
 
