@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["pointwise", "pointwise_splitk", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +31,7 @@ STATUS = {0: "DGRAD_OK", 1: "DGRAD_ERR_INVALID", 2: "DGRAD_ERR_UNSUPPORTED", 3: 
           4: "DGRAD_ERR_CUDA", 5: "DGRAD_ERR_TIMEOUT"}
 DW_MODES = {"auto": 0, "rotated": 1, "rowstream": 2}
 DTYPES = {"f32": 0, "bf16": 1}
+SPLITK_SCRATCH_BYTES = 8 << 20   # DGRAD_SPLITK_SCRATCH_BYTES: the fixed per-device split-K buffer
 
 
 class DgradUnavailable(RuntimeError):
@@ -96,6 +97,8 @@ def lib():
             L.dgrad_pointwise_splitk_workspace.argtypes = [P(Problem), ctypes.c_int, P(ctypes.c_size_t),
                                                            P(ctypes.c_int)]
             L.dgrad_pointwise_splitk_workspace.restype = ctypes.c_int
+            L.dgrad_pointwise_splitk_noalloc.argtypes = [P(Problem), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+            L.dgrad_pointwise_splitk_noalloc.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -189,6 +192,30 @@ def pointwise_splitk(dY, W, splits=0, workspace=None, out=None, stream=None):
                                         W.data_ptr(), out.data_ptr(), workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
            "dgrad_pointwise_splitk")
+    return out
+
+
+def pointwise_splitk_noalloc(dY, W, out, splits=0, stream=None):
+    """Split-K pointwise dgrad that allocates nothing (dgrad_pointwise_splitk_noalloc).
+
+    For callers that must not allocate device memory at call time: the partial
+    tiles go to the library's fixed per-device scratch buffer of
+    SPLITK_SCRATCH_BYTES, so ``out`` (N,H,W,C, dY's dtype) is required.  Calls
+    that overlap in time on one device share that buffer and race; calls ordered
+    on one stream do not.  The first call on a device sets the buffer up: make
+    it before any stream capture begins.  A problem whose partial tiles do not
+    fit the buffer raises DgradError (status 2, unsupported)."""
+    _need_cuda(dY, W, out)
+    if dY.dim() != 4 or W.dim() != 2 or W.shape[0] != dY.shape[3]:
+        raise ValueError("expected dY (N,H,W,K) and W (K,C)")
+    N, H, Wd, K = dY.shape
+    C = W.shape[1]
+    if tuple(out.shape) != (N, H, Wd, C) or out.dtype != dY.dtype:
+        raise ValueError("out must be (N,H,W,C) with dY's dtype")
+    prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
+    _check(lib().dgrad_pointwise_splitk_noalloc(ctypes.byref(prob), _dtype_code(dY), int(splits), dY.data_ptr(),
+                                                W.data_ptr(), out.data_ptr(), _stream_ptr(stream)),
+           "dgrad_pointwise_splitk_noalloc")
     return out
 
 

@@ -382,6 +382,8 @@ int dgrad_last_cuda_error(void) { return t_last_cuda; }
 
 }  // extern "C"
 
+void dgrad::record_cuda_error(cudaError_t e) { t_last_cuda = static_cast<int>(e); }
+
 // ------------------------------------------------------------------ diagnostics
 
 namespace {

@@ -50,6 +50,10 @@ size_t pointwise_splitk_workspace_bytes(const PwArgs& a, int splits);
 cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                        int splits, float* ws, int num_sms, cudaStream_t stream);
 
+// Keep a CUDA error code for dgrad_last_cuda_error (entry points defined
+// outside the ABI file report their failures through this).
+void record_cuda_error(cudaError_t e);
+
 // Depthwise problem (groups = C = K), NHWC, dense.
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;

@@ -112,6 +112,40 @@ dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t
 dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int splits, size_t* bytes,
                                                 int* splits_used);
 
+/* ---- A variant for callers that cannot allocate (no counterpart on the
+ * pages: their kernels take whatever workspace their host framework gives). ---- */
+
+/* Size of the fixed split-K scratch buffer built into the library: 8 MiB, one
+ * buffer per device. */
+#define DGRAD_SPLITK_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* dgrad_pointwise_splitk with no workspace argument: the fp32 partial tiles go
+ * to a fixed buffer of DGRAD_SPLITK_SCRATCH_BYTES that is part of the
+ * library's device image (CUDA reserves it when it loads the library's code on
+ * a device), so the call allocates nothing: no cudaMalloc, no framework
+ * allocator.  It serves callers that have no workspace to pass and must not
+ * allocate at call time, for example a plugin or callback running inside a
+ * framework that owns all device memory, or code that runs while a caching
+ * allocator is reclaiming memory and so cannot call back into it.
+ * Same shape class, dtype, layouts, kernels and results as
+ * dgrad_pointwise_splitk with the same split count.
+ * splits: 1 .. 64, or 0 for the automatic count, lowered as far as needed for
+ * the partial tiles to fit the buffer.  When the partial tiles still need more
+ * than DGRAD_SPLITK_SCRATCH_BYTES (splits * M * C * 4 bytes, M = N*H*W; with
+ * splits 0, even one split's M * C * 4), the call returns
+ * DGRAD_ERR_UNSUPPORTED and launches nothing.
+ * Nothing in the buffer has to start at zero and nothing clears it: each split
+ * writes its whole partial tile before the reduction reads it.
+ * Set-up: the first call on each device (with that device current) looks up
+ * the buffer's device address and keeps it; make that first call before any
+ * stream capture begins.
+ * Races: there is ONE buffer per device.  Calls whose work may overlap on the
+ * same device (issued to different streams, or from several host threads
+ * without ordering between their streams) write the same buffer and corrupt
+ * each other's results.  Calls ordered on one stream are safe. */
+dgrad_status_t dgrad_pointwise_splitk_noalloc(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
+                                              const void* dY, const void* W, void* dX, void* stream);
+
 /* Depthwise dgrad (groups = C; requires K == C, else DGRAD_ERR_UNSUPPORTED).
  * Rotated-filter mode requires stride 1, KH and KW <= 64 and
  * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1 (the rotated padding KH-1-pad_h and
