@@ -250,12 +250,15 @@ KERNEL_SOURCE = {"pointwise": {"bf16": "convolution_backward_b200/csrc/pointwise
                  "rotated": "convolution_backward_b200/csrc/dw_rotated.cu",
                  "rowstream": "convolution_backward_b200/csrc/dw_rowstream.cu",
                  "rowstream_fast": "convolution_backward_b200/csrc/dw_rowstream_fast.cu",
-                 "tile": "convolution_backward_b200/csrc/dw_tile.cu"}
+                 "tile": "convolution_backward_b200/csrc/dw_tile.cu",
+                 "toeplitz": "convolution_backward_b200/csrc/dw_toeplitz.cu"}
 
 
 def kernel_of(p):
     if p.variant == "splitk":
         return "pw_tc_splitk_kernel", KERNEL_SOURCE["pointwise"]["bf16"]
+    if p.variant == "tc":
+        return "dw_toeplitz_kernel", KERNEL_SOURCE["toeplitz"]
     if p.kind == "pointwise":
         return ("pw_tc_pair_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
     if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
@@ -296,11 +299,17 @@ def run_ours(args, world, rank, local):
         if p.variant == "splitk":
             nb, _ = cb.splitk_workspace_bytes(p.N, p.H, p.W, p.K, p.C, 0)
             workspaces[p.name] = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        if p.variant == "tc":
+            nb = cb.depthwise_tc_workspace_bytes(p.N, p.H, p.W, p.C, p.KH, p.KW, p.pad_h, p.pad_w)
+            workspaces[p.name] = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def call(p, dy, w, out):
         if p.variant == "splitk":
             cb.pointwise_splitk(dy, w, splits=0, workspace=workspaces[p.name], out=out)
+        elif p.variant == "tc":
+            cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=workspaces[p.name],
+                            out=out)
         elif p.kind == "pointwise":
             cb.pointwise(dy, w, out=out)
         else:

@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwise_tc", "depthwise_tc_workspace_bytes", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +99,10 @@ def lib():
             L.dgrad_pointwise_splitk_workspace.restype = ctypes.c_int
             L.dgrad_pointwise_splitk_noalloc.argtypes = [P(Problem), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
             L.dgrad_pointwise_splitk_noalloc.restype = ctypes.c_int
+            L.dgrad_depthwise_tc.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp, ctypes.c_size_t, vp]
+            L.dgrad_depthwise_tc.restype = ctypes.c_int
+            L.dgrad_depthwise_tc_workspace.argtypes = [P(Problem), P(ctypes.c_size_t)]
+            L.dgrad_depthwise_tc_workspace.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -251,6 +255,52 @@ def depthwise(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, mode="auto",
             raise ValueError("out has the wrong shape or dtype")
     _check(lib().dgrad_depthwise(ctypes.byref(prob), _dtype_code(dY), DW_MODES[mode], dY.data_ptr(),
                                  W.data_ptr(), out.data_ptr(), _stream_ptr(stream)), "dgrad_depthwise")
+    return out
+
+
+def depthwise_tc_workspace_bytes(N, H, W, C, KH, KW, pad_h=0, pad_w=-1) -> int:
+    """Workspace bytes dgrad_depthwise_tc needs (host only); raises DgradError when unsupported."""
+    prob = Problem(N, H, W, C, C, KH, KW, 1, pad_h, pad_w)
+    nb = ctypes.c_size_t()
+    _check(lib().dgrad_depthwise_tc_workspace(ctypes.byref(prob), ctypes.byref(nb)), "dgrad_depthwise_tc_workspace")
+    return nb.value
+
+
+def depthwise_tc(dY, W, *, H, W_out=None, pad_h=0, pad_w=-1, workspace=None, out=None, stream=None, **kw):
+    """Stride-1 depthwise dgrad on the tensor cores (bf16; dgrad_depthwise_tc).
+
+    Same arguments and result as depthwise() at stride 1.  workspace: a CUDA
+    tensor of at least depthwise_tc_workspace_bytes(...) bytes, allocated here
+    with torch when None."""
+    import torch
+    if W_out is None:
+        W_out = kw.pop("Wd")
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 3 or W.shape[2] != dY.shape[3]:
+        raise ValueError("expected dY (N,Ho,Wo,C) and W (KH,KW,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
+    N, Ho, Wo, C = dY.shape
+    KH, KW = W.shape[0], W.shape[1]
+    eho, ewo = out_dims(H, W_out, KH, KW, 1, pad_h, pad_w)
+    if (eho, ewo) != (Ho, Wo):
+        raise ValueError(f"dY spatial extent {(Ho, Wo)} does not match the geometry ({eho}, {ewo})")
+    prob = Problem(N, H, W_out, C, C, KH, KW, 1, pad_h, pad_w)
+    nbytes = depthwise_tc_workspace_bytes(N, H, W_out, C, KH, KW, pad_h, pad_w)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dY.device)
+    if out is None:
+        out = torch.empty((N, H, W_out, C), dtype=dY.dtype, device=dY.device)
+    else:
+        _need_cuda(out)
+        if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
+            raise ValueError("out has the wrong shape or dtype")
+    _check(lib().dgrad_depthwise_tc(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
+                                    out.data_ptr(), workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "dgrad_depthwise_tc")
     return out
 
 

@@ -109,6 +109,23 @@ bool encode_nhwc_bf16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H
     return r == CUDA_SUCCESS;
 }
 
+// 4-D bf16 planar tensor [C][Y][N][Xs] seen as dims (X, N, Y, C) inner first,
+// box (8, 8, nr, 1), no swizzle, zero fill outside the tensor.
+bool encode_planar_bf16(CUtensorMap* map, const void* base, uint64_t X, uint64_t N, uint64_t Y, uint64_t C,
+                        uint64_t Xs, unsigned nr)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {X, N, Y, C};
+    const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
+    const cuuint32_t b[4] = {8, 8, nr, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int env_int(const char* name, int dflt)
@@ -276,6 +293,76 @@ dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t
         return cuda_fail(cudaErrorInvalidValue);
     cudaError_t e = dgrad::launch_pointwise_tc_splitk(a, map_a, map_b, splits, static_cast<float*>(workspace),
                                                        st->sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+// Shared checks for the tensor-core depthwise entry points: stride-1 depthwise,
+// bf16, extents within the kernels' 32-bit indexing and grid limits, and a tile
+// plan that fits one SM.
+static dgrad_status_t toeplitz_prepare(const dgrad_problem_t* prob, dgrad_dtype_t dtype, dgrad::DwArgs* a,
+                                       dgrad::ToepPlan* plan)
+{
+    int64_t Ho = 0, Wo = 0;
+    int pw = 0;
+    dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
+    if (s != DGRAD_OK) return s;
+    if (dtype != DGRAD_BF16 || prob->stride != 1 || prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;
+    if ((prob->C * 2) % 16) return DGRAD_ERR_ALIGNMENT;
+    if (prob->N > 65535 || prob->H > 65535 || prob->W > 65535 || prob->C > (1 << 24)) return DGRAD_ERR_UNSUPPORTED;
+    *a = dgrad::DwArgs{};
+    a->N = static_cast<int>(prob->N);
+    a->H = static_cast<int>(prob->H);
+    a->W = static_cast<int>(prob->W);
+    a->C = static_cast<int>(prob->C);
+    a->Ho = static_cast<int>(Ho);
+    a->Wo = static_cast<int>(Wo);
+    a->KH = prob->KH;
+    a->KW = prob->KW;
+    a->S = 1;
+    a->ph = prob->pad_h;
+    a->pw = pw;
+    a->bf16 = true;
+    if (!dgrad::plan_dw_toeplitz(*a, plan)) return DGRAD_ERR_UNSUPPORTED;
+    return DGRAD_OK;
+}
+
+dgrad_status_t dgrad_depthwise_tc_workspace(const dgrad_problem_t* prob, size_t* bytes)
+{
+    if (!bytes) return DGRAD_ERR_INVALID;
+    dgrad::DwArgs a{};
+    dgrad::ToepPlan plan{};
+    dgrad_status_t s = toeplitz_prepare(prob, DGRAD_BF16, &a, &plan);
+    if (s != DGRAD_OK) return s;
+    *bytes = prob->N == 0 ? 0 : plan.ws_in + plan.ws_out;
+    return DGRAD_OK;
+}
+
+dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W,
+                                  void* dX, void* workspace, size_t workspace_bytes, void* stream)
+{
+    dgrad::DwArgs a{};
+    dgrad::ToepPlan plan{};
+    dgrad_status_t s = toeplitz_prepare(prob, dtype, &a, &plan);
+    if (s != DGRAD_OK) return s;
+    if (prob->N == 0) return DGRAD_OK;
+    if (!dY || !W || !dX || !workspace) return DGRAD_ERR_INVALID;
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || !aligned16(workspace)) return DGRAD_ERR_ALIGNMENT;
+    if (workspace_bytes < plan.ws_in + plan.ws_out) return DGRAD_ERR_INVALID;
+    DeviceState* st = nullptr;
+    s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    a.dY = dY;
+    a.filt = W;
+    a.dX = dX;
+    a.status = st->status;
+    CUtensorMap map_b;
+    if (!encode_planar_bf16(&map_b, workspace, static_cast<uint64_t>(plan.Xi), static_cast<uint64_t>(a.N),
+                            static_cast<uint64_t>(plan.Yi), static_cast<uint64_t>(a.C),
+                            static_cast<uint64_t>(plan.Xsi), static_cast<unsigned>(plan.NR)))
+        return cuda_fail(cudaErrorInvalidValue);
+    cudaError_t e = dgrad::launch_dw_toeplitz(a, plan, map_b, workspace, st->sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 

@@ -44,7 +44,7 @@ class Problem:
     dy_var: float = 1.0
     w_dist: str = "normal"
     w_var: float = 1.0
-    variant: str = ""    # "splitk": run through the split-K pointwise entry point
+    variant: str = ""    # "splitk": split-K pointwise entry point; "tc": tensor-core depthwise entry point
 
     @property
     def Ho(self) -> int:
@@ -120,6 +120,10 @@ EXTRA_WORKLOADS: dict[str, list[Problem]] = {
                                       K=2048, seed=5, w_var=1.0 / 2048, variant="splitk")],
     "pw_bf16_smallm": [Problem("pw_bf16_smallm", "pointwise", "bf16", N=2, H=14, W=14, C=512, K=2048,
                                seed=5, w_var=1.0 / 2048)],
+    # the large stride-1 depthwise problems through the tensor-core entry point
+    "dw_large_tc": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_tc", variant="tc"),
+                    WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_tc", variant="tc"),
+                    WORKLOADS["dw_nonsquare_strided_bf16"][1].replace(name="dw5x51_bf16_tc", variant="tc")],
 }
 
 

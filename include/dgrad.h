@@ -155,6 +155,30 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
                                dgrad_dw_mode_t mode,
                                const void* dY, const void* W, void* dX, void* stream);
 
+/* Stride-1 depthwise dgrad on the tensor cores, for large filters.  Each
+ * channel's plane is a sum of GEMMs, one per filter line along the shorter
+ * filter side, whose other operand is the banded (Toeplitz) matrix of that
+ * filter line along the longer side: the implicit-GEMM formulation of the
+ * rotated-filter correlation ("channel-packed and large-filter depthwise
+ * dgrad", Technical Details: rotated-filter dgrad; the pages sent large filters
+ * through an implicit-GEMM path before the FP32 rotated-filter kernel).  The
+ * MMAs run in bf16 with fp32 accumulation (tcgen05), so results equal those of
+ * dgrad_depthwise up to fp32 summation order.
+ * Requirements: DGRAD_BF16, stride 1, K == C, KH and KW <= 64,
+ * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1, N, H, W <= 65535; else
+ * DGRAD_ERR_UNSUPPORTED (also when the filter is too large for the tile plan).
+ * workspace: caller-owned device memory, 16-byte aligned, at least the size
+ * dgrad_depthwise_tc_workspace reports; it holds dY and dX as per-channel planes
+ * (channel-outermost copies of both); its contents on entry do not matter.
+ * Three kernels run in order on `stream`: dY to planes, the tensor-core kernel,
+ * planes to dX. */
+dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W,
+                                  void* dX, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes dgrad_depthwise_tc needs (0 for an empty batch); returns the
+ * same refusals as dgrad_depthwise_tc for the problem (host only). */
+dgrad_status_t dgrad_depthwise_tc_workspace(const dgrad_problem_t* prob, size_t* bytes);
+
 /* Output extents of the forward convolution the problem describes (host only,
  * no CUDA call).  Returns DGRAD_ERR_INVALID for an invalid problem. */
 dgrad_status_t dgrad_out_dims(const dgrad_problem_t* prob, int64_t* Ho, int64_t* Wo);

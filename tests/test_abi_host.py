@@ -175,3 +175,30 @@ def test_splitk_workspace_empty_batch():
     p = _prob(N=0, H=14, W=14, C=64, K=256, KH=1, KW=1, ph=0, pw=0)
     assert L.dgrad_pointwise_splitk_workspace(ctypes.byref(p), 3, ctypes.byref(nb), None) == OK
     assert nb.value == 0
+
+
+def test_depthwise_tc_validation_and_workspace_size():
+    L = cb.lib()
+    nb = ctypes.c_size_t()
+    p31 = cb.Problem(16, 64, 64, 384, 384, 31, 31, 1, 15, 15)
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p31), ctypes.byref(nb)) == OK
+    assert nb.value == 2 * 384 * 64 * 16 * 64 * 2                # planar dY + planar dX
+    p51 = cb.Problem(8, 64, 64, 768, 768, 51, 5, 1, 25, 2)
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), ctypes.byref(nb)) == OK
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), None) == INVALID
+    empty = cb.Problem(0, 64, 64, 384, 384, 31, 31, 1, 15, 15)
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(empty), ctypes.byref(nb)) == OK and nb.value == 0
+    refused = [cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 32, 32),   # 64x64 does not fit the tile plan
+               cb.Problem(1, 64, 64, 32, 32, 7, 7, 2, 3, 3),       # stride 2
+               cb.Problem(1, 64, 64, 32, 64, 7, 7, 1, 3, 3),       # depth multiplier 2
+               cb.Problem(1, 64, 64, 32, 32, 7, 7, 1, 7, 3)]       # pad beyond KH-1
+    for q in refused:
+        assert L.dgrad_depthwise_tc_workspace(ctypes.byref(q), ctypes.byref(nb)) == UNSUPPORTED
+    call = lambda prob, dtype=BF16, ws=FAKE, ws_bytes=1 << 40: L.dgrad_depthwise_tc(
+        ctypes.byref(prob), dtype, FAKE, FAKE, FAKE, ws, ws_bytes, None)
+    assert call(p31, dtype=F32) == UNSUPPORTED
+    assert call(p31, ws=0) == INVALID
+    assert call(p31, ws=FAKE + 8) == ALIGNMENT
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p31), ctypes.byref(nb)) == OK
+    assert call(p31, ws_bytes=nb.value - 256) == INVALID
+    assert L.dgrad_depthwise_tc(ctypes.byref(empty), BF16, 0, 0, 0, 0, 0, None) == OK

@@ -177,6 +177,44 @@ def test_pointwise_splitk(p, splits):
     cb.check_status()
 
 
+TC_SMALL = [
+    P("tc3x3", "depthwise", "bf16", 1, 10, 9, 8, 8, 3, 3, 1, 1, 1, seed=141),
+    P("tc5x11_ragged_images", "depthwise", "bf16", 9, 7, 70, 8, 8, 5, 11, 1, 2, 5, seed=142),
+    P("tc11x4_long_h", "depthwise", "bf16", 2, 70, 12, 8, 8, 11, 4, 1, 0, 3, seed=143),
+    P("tc31x31", "depthwise", "bf16", 3, 20, 20, 16, 16, 31, 31, 1, 15, 15, seed=144),
+    P("tc13x5", "depthwise", "bf16", 2, 16, 16, 8, 8, 13, 5, 1, 6, 2, seed=145),
+    P("tc5x13", "depthwise", "bf16", 2, 16, 16, 8, 8, 5, 13, 1, 2, 6, seed=146),
+    P("tc3x3_two_by_two_tiles", "depthwise", "bf16", 1, 70, 70, 8, 8, 3, 3, 1, 1, 1, seed=147),
+    P("tc41x41", "depthwise", "bf16", 1, 12, 12, 8, 8, 41, 41, 1, 20, 20, seed=148),
+    P("tc51x51_half_tile", "depthwise", "bf16", 1, 64, 64, 8, 8, 51, 51, 1, 25, 25, seed=149),
+    P("tc31x31_c40", "depthwise", "bf16", 1, 37, 45, 40, 40, 31, 31, 1, 15, 15, seed=150),
+    P("tc7x7_nonsame", "depthwise", "bf16", 2, 17, 18, 16, 16, 7, 7, 1, 1, 5, seed=151),
+    P("tc1x1", "depthwise", "bf16", 2, 5, 6, 16, 16, 1, 1, 1, 0, 0, seed=152),
+    P("tc51x5", "depthwise", "bf16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=153),
+    P("tc5x51", "depthwise", "bf16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=154),
+]
+
+
+@pytest.mark.parametrize("p", TC_SMALL, ids=[p.name for p in TC_SMALL])
+def test_depthwise_tensor_core(p):
+    """Stride-1 depthwise on tcgen05 (banded-Toeplitz GEMMs, §8 NEXT-2) against the oracle; the
+    workspace starts as NaN (its contents must not matter) and a second call gives identical bits."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    nb = cb.depthwise_tc_workspace_bytes(p.N, p.H, p.W, p.C, p.KH, p.KW, p.pad_h, p.pad_w)
+    ws = torch.full((nb // 2 + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=ws)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/tc")
+    again = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=ws)
+    assert torch.equal(out, again)
+    cb.check_status()
+
+
 RS_FAST = [
     P("rs7x7s2_p3", "depthwise", "bf16", 2, 29, 27, 40, 40, 7, 7, 2, 3, 3, seed=71),
     P("rs7x7s2_p0", "depthwise", "bf16", 1, 30, 31, 32, 32, 7, 7, 2, 0, 0, seed=72),
@@ -254,6 +292,30 @@ def test_full_size_workloads(p):
     err = (out.float() - tref).abs().max().item()
     assert err / (tref.abs().max().item() + 1e-6) <= 1e-2
     import convolution_backward_b200 as cb
+    cb.check_status()
+
+
+TC_FULL = synthetic.EXTRA_WORKLOADS["dw_large_tc"]
+
+
+@pytest.mark.parametrize("p", TC_FULL, ids=[p.name for p in TC_FULL])
+def test_full_size_tensor_core_depthwise(p):
+    """The large stride-1 workloads through dgrad_depthwise_tc, as the benchmark's tensor-core
+    variant runs them: sampled oracle points, and every element against cuDNN fp32."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    torch.cuda.synchronize()
+    pts = h.sample_points(p, 3000)
+    got = out.float()[pts[:, 0], pts[:, 1], pts[:, 2], pts[:, 3]].cpu().numpy().astype(np.float64)
+    ref = h.oracle_points(p, inp.dy, inp.w, pts)
+    absref = h.oracle_points(p, np.abs(inp.dy), np.abs(inp.w), pts)
+    h.check(p, got, ref, absref, what=f"{p.name} sampled")
+    tref = _torch_fp32_reference(p, dy, w)
+    err = (out.float() - tref).abs().max().item()
+    assert err / (tref.abs().max().item() + 1e-6) <= 1e-2
     cb.check_status()
 
 
