@@ -381,7 +381,10 @@ def run_ours(args, world, rank, local):
     clocks = sampler.stop()
     barrier(world)
     cb.check_status()
-    n_launches = args.steps * len(problems) + sum(kern_iters * reps[j] for j in range(len(problems)))
+    # kernels one call launches: the tensor-core depthwise call runs pack, filter pack, MMA and
+    # unpack kernels; split-K runs the GEMM and the reduction; every other call is one kernel
+    per_call = [4 if p.variant == "tc" else 2 if p.variant == "splitk" else 1 for p in problems]
+    n_launches = sum((args.steps + kern_iters * reps[j]) * per_call[j] for j in range(len(problems)))
 
     step_ms_max = max_over_ranks(world, step_ms, dev)
     flops_step = sum(p.nominal_flops() for p in problems)
@@ -401,7 +404,9 @@ def run_ours(args, world, rank, local):
         tf = fl / (ms * 1e-3) / 1e12
         gbs = by / (ms * 1e-3) / 1e9
         t_bytes = by / (hbm * 1e9)
-        if p.kind == "pointwise" and p.dtype == "bf16":
+        if (p.kind == "pointwise" and p.dtype == "bf16") or p.variant == "tc":
+            # tensor-core paths: nominal FLOPs against the bf16 tensor peak (the banded-Toeplitz
+            # depthwise issues about 3x its nominal FLOPs as MMAs; the fraction stays nominal)
             t_flop = fl / (bf16_peak * 1e12)
             bound = "tensor"
         else:
@@ -420,11 +425,12 @@ def run_ours(args, world, rank, local):
             "floor_us": round(max(t_bytes, t_flop) * 1e6, 3),
             "frac_of_tensor_peak": round(tf / bf16_peak, 4) if bound == "tensor" else None,
             "frac_of_hbm": round(gbs / hbm, 4),
+            "fp32_floor_us": round(fl / (fp32_peak * 1e12) * 1e6, 3) if p.kind == "depthwise" else None,
             "dram_bytes_per_launch": tr})
     dom = max(range(len(problems)), key=lambda j: kern_ms[j])
     dp = problems[dom]
     dk = per_kernel[dom]
-    if dp.kind == "pointwise" and dp.dtype == "bf16":
+    if (dp.kind == "pointwise" and dp.dtype == "bf16") or dp.variant == "tc":
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": bf16_peak, "unit": "TFLOP/s",
                 "frac": round(dk["tflops"] / bf16_peak, 4), "traffic": dk["dram_bytes_per_launch"]}
     elif dk["binding"] == "hbm":

@@ -110,7 +110,7 @@ bool encode_nhwc_bf16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H
 }
 
 // 4-D bf16 planar tensor [C][Y][N][Xs] seen as dims (X, N, Y, C) inner first,
-// box (8, 8, nr, 1), no swizzle, zero fill outside the tensor.
+// box (64, 8, nr, 1), 128-byte swizzle, zero fill outside the tensor.
 bool encode_planar_bf16(CUtensorMap* map, const void* base, uint64_t X, uint64_t N, uint64_t Y, uint64_t C,
                         uint64_t Xs, unsigned nr)
 {
@@ -118,10 +118,10 @@ bool encode_planar_bf16(CUtensorMap* map, const void* base, uint64_t X, uint64_t
     if (!enc) return false;
     const cuuint64_t dims[4] = {X, N, Y, C};
     const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
-    const cuuint32_t b[4] = {8, 8, nr, 1};
+    const cuuint32_t b[4] = {64, 8, nr, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -335,7 +335,7 @@ dgrad_status_t dgrad_depthwise_tc_workspace(const dgrad_problem_t* prob, size_t*
     dgrad::ToepPlan plan{};
     dgrad_status_t s = toeplitz_prepare(prob, DGRAD_BF16, &a, &plan);
     if (s != DGRAD_OK) return s;
-    *bytes = prob->N == 0 ? 0 : plan.ws_in + plan.ws_out;
+    *bytes = prob->N == 0 ? 0 : plan.ws_in + plan.ws_out + plan.ws_f;
     return DGRAD_OK;
 }
 
@@ -349,7 +349,7 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
     if (prob->N == 0) return DGRAD_OK;
     if (!dY || !W || !dX || !workspace) return DGRAD_ERR_INVALID;
     if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || !aligned16(workspace)) return DGRAD_ERR_ALIGNMENT;
-    if (workspace_bytes < plan.ws_in + plan.ws_out) return DGRAD_ERR_INVALID;
+    if (workspace_bytes < plan.ws_in + plan.ws_out + plan.ws_f) return DGRAD_ERR_INVALID;
     DeviceState* st = nullptr;
     s = device_state(&st);
     if (s != DGRAD_OK) return s;

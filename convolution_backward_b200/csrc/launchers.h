@@ -76,14 +76,15 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 // Stride-1 depthwise on the tcgen05 tensor cores (bf16): each channel plane as
 // a sum of banded-Toeplitz GEMMs, one per filter line.  plan_dw_toeplitz picks
 // the plane orientation and tile and returns false when the problem does not
-// fit; the launch needs a workspace of ws_in + ws_out bytes (planar dY, then
-// planar dX) and map_b, a 4-D bf16 map of the planar dY [C][Yi][N][Xsi] with
-// dims (Xi, N, Yi, C), box (8, 8, NR, 1), no swizzle, zero fill.
+// fit; the launch needs a workspace of ws_in + ws_out + ws_f bytes (planar dY,
+// planar dX, packed filter lines) and map_b, a 4-D bf16 map of the planar dY
+// [C][Yi][N][Xsi] with dims (Xi, N, Yi, C), box (64, 8, NR, 1), 128-byte
+// swizzle, zero fill.
 struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
-    int NH, K, NR, NI, L, a_cols;
-    uint32_t b_bytes, f_off, bar_off;
-    size_t smem, ws_in, ws_out;
+    int NH, K, NR, NI, half_l, f_words, a_col0, a_cols, na;
+    uint32_t panel_bytes, b_bytes, f_off, bar_off;
+    size_t smem, ws_in, ws_out, ws_f;
 };
 bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* p);
 cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtensorMap& map_b, void* ws,

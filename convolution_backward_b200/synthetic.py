@@ -91,6 +91,9 @@ class Problem:
 
 # The five workloads.  Sizes, seeds and distributions are the ones the
 # benchmark is quoted on; the fifth holds three problems drawn from seed 4.
+# `variant` names the entry point the benchmark step calls: the three large
+# stride-1 depthwise problems run through dgrad_depthwise_tc (tensor cores).
+# Parity tests run every problem through dgrad_depthwise as well.
 WORKLOADS: dict[str, list[Problem]] = {
     "pw_f32_small": [Problem("pw_f32_small", "pointwise", "f32", N=2, H=14, W=14, C=64, K=64,
                              seed=0, dy_dist="uniform", w_dist="uniform")],
@@ -99,12 +102,12 @@ WORKLOADS: dict[str, list[Problem]] = {
     "pw_bf16": [Problem("pw_bf16", "pointwise", "bf16", N=32, H=28, W=28, C=256, K=512,
                         seed=2, w_var=1.0 / 512)],
     "dw31x31_bf16": [Problem("dw31x31_bf16", "depthwise", "bf16", N=16, H=64, W=64, C=384, K=384,
-                             KH=31, KW=31, pad_h=15, pad_w=15, seed=3, w_var=1.0 / 961)],
+                             KH=31, KW=31, pad_h=15, pad_w=15, seed=3, w_var=1.0 / 961, variant="tc")],
     "dw_nonsquare_strided_bf16": [
         Problem("dw51x5_bf16", "depthwise", "bf16", N=8, H=64, W=64, C=768, K=768,
-                KH=51, KW=5, pad_h=25, pad_w=2, seed=4, w_var=1.0 / 255),
+                KH=51, KW=5, pad_h=25, pad_w=2, seed=4, w_var=1.0 / 255, variant="tc"),
         Problem("dw5x51_bf16", "depthwise", "bf16", N=8, H=64, W=64, C=768, K=768,
-                KH=5, KW=51, pad_h=2, pad_w=25, seed=4, w_var=1.0 / 255),
+                KH=5, KW=51, pad_h=2, pad_w=25, seed=4, w_var=1.0 / 255, variant="tc"),
         Problem("dw7x7s2_bf16", "depthwise", "bf16", N=32, H=112, W=112, C=96, K=96,
                 KH=7, KW=7, stride=2, pad_h=3, pad_w=3, seed=4, w_var=1.0 / 49),
     ],
@@ -120,10 +123,10 @@ EXTRA_WORKLOADS: dict[str, list[Problem]] = {
                                       K=2048, seed=5, w_var=1.0 / 2048, variant="splitk")],
     "pw_bf16_smallm": [Problem("pw_bf16_smallm", "pointwise", "bf16", N=2, H=14, W=14, C=512, K=2048,
                                seed=5, w_var=1.0 / 2048)],
-    # the large stride-1 depthwise problems through the tensor-core entry point
-    "dw_large_tc": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_tc", variant="tc"),
-                    WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_tc", variant="tc"),
-                    WORKLOADS["dw_nonsquare_strided_bf16"][1].replace(name="dw5x51_bf16_tc", variant="tc")],
+    # the large stride-1 depthwise problems through the FP32 rotated-filter kernel (dgrad_depthwise)
+    "dw_large_fp32": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_fp32", variant=""),
+                      WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_fp32", variant=""),
+                      WORKLOADS["dw_nonsquare_strided_bf16"][1].replace(name="dw5x51_bf16_fp32", variant="")],
 }
 
 

@@ -182,13 +182,16 @@ def test_depthwise_tc_validation_and_workspace_size():
     nb = ctypes.c_size_t()
     p31 = cb.Problem(16, 64, 64, 384, 384, 31, 31, 1, 15, 15)
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p31), ctypes.byref(nb)) == OK
-    assert nb.value == 2 * 384 * 64 * 16 * 64 * 2                # planar dY + planar dX
+    # planar dY + planar dX + packed filter lines (31 lines of (96 + 80) / 2 words per channel)
+    assert nb.value == 2 * 384 * 64 * 16 * 64 * 2 + 384 * 31 * 88 * 4
     p51 = cb.Problem(8, 64, 64, 768, 768, 51, 5, 1, 25, 2)
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), ctypes.byref(nb)) == OK
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), None) == INVALID
     empty = cb.Problem(0, 64, 64, 384, 384, 31, 31, 1, 15, 15)
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(empty), ctypes.byref(nb)) == OK and nb.value == 0
-    refused = [cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 32, 32),   # 64x64 does not fit the tile plan
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 32, 32)),
+                                          ctypes.byref(nb)) == OK
+    refused = [cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 6, 6),     # 64x64 at pad 6: K = 144, too large a tile
                cb.Problem(1, 64, 64, 32, 32, 7, 7, 2, 3, 3),       # stride 2
                cb.Problem(1, 64, 64, 32, 64, 7, 7, 1, 3, 3),       # depth multiplier 2
                cb.Problem(1, 64, 64, 32, 32, 7, 7, 1, 7, 3)]       # pad beyond KH-1

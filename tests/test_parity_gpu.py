@@ -191,6 +191,8 @@ TC_SMALL = [
     P("tc7x7_nonsame", "depthwise", "bf16", 2, 17, 18, 16, 16, 7, 7, 1, 1, 5, seed=151),
     P("tc1x1", "depthwise", "bf16", 2, 5, 6, 16, 16, 1, 1, 1, 0, 0, seed=152),
     P("tc51x5", "depthwise", "bf16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=153),
+    P("tc64x64", "depthwise", "bf16", 1, 70, 66, 8, 8, 64, 64, 1, 32, 31, seed=155),
+    P("tc17x17_nonsame", "depthwise", "bf16", 10, 40, 33, 16, 16, 17, 17, 1, 3, 11, seed=156),
     P("tc5x51", "depthwise", "bf16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=154),
 ]
 
@@ -295,7 +297,7 @@ def test_full_size_workloads(p):
     cb.check_status()
 
 
-TC_FULL = synthetic.EXTRA_WORKLOADS["dw_large_tc"]
+TC_FULL = [p for p in synthetic.all_problems() if p.variant == "tc"]
 
 
 @pytest.mark.parametrize("p", TC_FULL, ids=[p.name for p in TC_FULL])
