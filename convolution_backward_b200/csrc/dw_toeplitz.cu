@@ -38,9 +38,9 @@
 // brings them in with one bulk copy whenever the channel changes.
 //
 // Three helper kernels run around the MMA kernel, all through the caller's
-// workspace: dw_pack_kernel writes NHWC dY as planes [C][Yi][N][Xs] (channels
+// workspace: dw_transpose_kernel writes NHWC dY as planes [C][Yi][N][Xs] (channels
 // outermost, images between rows and columns), dw_filter_pack_kernel writes the
-// padded filter lines of every channel, and dw_unpack_kernel writes the planar
+// padded filter lines of every channel, and dw_transpose_kernel writes the planar
 // output of the MMA epilogue back to NHWC dX.
 //
 // Roles (448 threads, one CTA per SM, a contiguous range of tiles per CTA so
@@ -52,6 +52,10 @@
 //               into registers, release it, then round to bf16 and store planes
 // Every wait is bounded; a timeout is recorded in the status word, raises the
 // CTA's abort flag, lets issued copies and MMAs finish and frees TMEM.
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "launchers.h"
@@ -59,13 +63,12 @@
 namespace dgrad {
 namespace {
 
-constexpr int kTW = 64;          // output columns per tile
-constexpr int kP = 2;            // output-row phases stacked in M
 constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epilogue
-constexpr int kOff = kTW + 8;    // offset of filter tap 0 in a padded filter line
+constexpr int kOff = 72;         // offset of filter tap 0 in a padded filter line (>= 64 + 8)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxA = 4;         // A buffers in tensor memory
-constexpr int kNumBars = 2 + 2 * kMaxA + 5;
+constexpr int kMaxB = 2;         // B blocks in shared memory
+constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 5;
 
 __host__ __device__ inline int floor8(int v) { return v >= 0 ? (v & ~7) : -((-v + 7) & ~7); }
 
@@ -75,10 +78,10 @@ struct ToepArgs {
     int* status;
     int N, C, Yo, Xo, Xso;
     int KY, py, px;
-    int NH, K, NR, NI, half_l;
+    int P, TW, XT, NH, Ks, NR, NI, half_l, NB;
     int num_xt, num_yt, num_g, num_units;
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
-    uint32_t panel_bytes, b_bytes, f_bytes, f_words, f_off, bar_off;
+    uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
 };
 
 struct Unit {
@@ -94,8 +97,8 @@ __device__ __forceinline__ Unit decode_unit(const ToepArgs& a, int u)
     r /= a.num_yt;
     t.g = r % a.num_g;
     t.c = r / a.num_g;
-    t.Y0 = yt * kP * a.NH;
-    t.x0 = xt * kTW;
+    t.Y0 = yt * a.P * a.NH;
+    t.x0 = xt * a.XT * a.TW;
     t.xb = floor8(t.x0 - a.px);
     return t;
 }
@@ -121,6 +124,9 @@ __device__ __forceinline__ void store_a_row(uint32_t taddr, const uint32_t* src,
 __device__ __forceinline__ void store_a(int kq, uint32_t taddr, const uint32_t* src, bool odd, bool nonzero)
 {
     switch (kq) {
+    case 1: store_a_row<1>(taddr, src, odd, nonzero); break;
+    case 2: store_a_row<2>(taddr, src, odd, nonzero); break;
+    case 3: store_a_row<3>(taddr, src, odd, nonzero); break;
     case 4: store_a_row<4>(taddr, src, odd, nonzero); break;
     case 5: store_a_row<5>(taddr, src, odd, nonzero); break;
     case 6: store_a_row<6>(taddr, src, odd, nonzero); break;
@@ -130,8 +136,107 @@ __device__ __forceinline__ void store_a(int kq, uint32_t taddr, const uint32_t* 
     }
 }
 
-// Units [u_begin, u_end) of this CTA: a contiguous range, so that the image
-// groups of one channel follow each other and share one filter load.
+// The MMAs of one shift step: for each 16-deep step q and sub-tile sx (sub-tiles
+// innermost, so consecutive MMAs go to different accumulators), D_sx += A[:, 16q..]
+// * B columns sx*TW + 16q ... (TW = 64 / XT).  The B descriptor of the step is
+// precomputed; each MMA only adds a constant to it (start address field, units of
+// 16 bytes: one 64-column panel is pb16, 16 columns are 2).
+template <int KQ, int XT>
+__device__ __forceinline__ void issue_step(const uint32_t (&d_tmem)[4], uint32_t a_tmem, uint64_t desc_i,
+                                           uint32_t pb16, uint32_t idesc, bool first)
+{
+    constexpr int TW = 64 / XT;
+#pragma unroll
+    for (int q = 0; q < KQ; ++q) {
+#pragma unroll
+        for (int sx = 0; sx < XT; ++sx) {
+            const int col = sx * TW + 16 * q;
+            const uint64_t bd = desc_i + static_cast<uint64_t>((col >> 6) * pb16 + ((col & 63) >> 4) * 2);
+            umma_f16_ts(d_tmem[sx], a_tmem + 8u * q, bd, idesc, (first && q == 0) ? 0u : 1u);
+        }
+    }
+}
+
+// Shared-memory barriers and addresses the MMA issuer works with.
+struct MmaCtx {
+    uint64_t* b_full;
+    uint64_t* b_empty;
+    uint64_t* a_full;
+    uint64_t* a_empty;
+    uint64_t* d_full;
+    uint64_t* d_empty;
+    const volatile int* abort_flag;
+    uint32_t tmem_base;
+    uint32_t bblk_addr;
+};
+
+// The MMA issuer's loop over its units, compiled per (16-deep steps per tile,
+// sub-tiles) so that each shift step is a short straight run of MMAs: buffer
+// indices and phases advance incrementally and the B descriptor moves by one
+// swizzle atom per step.  Returns false when a wait gave up.
+template <int KQ, int XT>
+__device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
+{
+    const int ncol_sub = 8 * a.NH;
+    const uint32_t idesc = idesc_bf16_f32(128, ncol_sub, /*b_mn_major=*/false);
+    const uint32_t sbo = static_cast<uint32_t>(a.P) * 1024u;
+    const uint32_t pb16 = a.panel_bytes >> 4;
+    uint32_t d_tmem[4];
+#pragma unroll
+    for (int sx = 0; sx < 4; ++sx) d_tmem[sx] = c.tmem_base + static_cast<uint32_t>(sx * ncol_sub);
+    const uint32_t a_first = c.tmem_base + static_cast<uint32_t>(a.a_col0);
+    const uint32_t a_last = a_first + static_cast<uint32_t>((a.na - 1) * a.a_cols);
+    uint32_t bb = 0, bph = 0, ab = 0, aph = 0, dph = 0;
+    uint32_t a_tmem = a_first;
+    for (int u = u_begin; u < u_end; ++u) {
+        if (!mbar_wait(&c.b_full[bb], bph, c.abort_flag) || !mbar_wait(c.d_empty, dph ^ 1u, c.abort_flag))
+            return false;
+        tc_fence_after();
+        uint64_t desc = sw128_desc(c.bblk_addr + bb * a.b_bytes, 16, sbo);
+        for (int i = 0; i < a.NI; ++i) {
+            if (!mbar_wait(&c.a_full[ab], aph, c.abort_flag)) return false;
+            tc_fence_after();
+            issue_step<KQ, XT>(d_tmem, a_tmem, desc, pb16, idesc, i == 0);
+            umma_commit(&c.a_empty[ab]);   // A buffer free once these MMAs have read it
+            desc += 64;                     // next shift step: one 1024-byte atom
+            if (a_tmem == a_last) {
+                a_tmem = a_first;
+                ab = 0;
+                aph ^= 1u;
+            } else {
+                a_tmem += static_cast<uint32_t>(a.a_cols);
+                ++ab;
+            }
+        }
+        umma_commit(c.d_full);
+        umma_commit(&c.b_empty[bb]);
+        if (++bb == static_cast<uint32_t>(a.NB)) {
+            bb = 0;
+            bph ^= 1u;
+        }
+        dph ^= 1u;
+    }
+    return true;
+}
+
+template <int XT>
+__device__ __forceinline__ bool mma_role_x(int kq, const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
+{
+    switch (kq) {
+    case 1: return mma_role<1, XT>(a, c, u_begin, u_end);
+    case 2: return mma_role<2, XT>(a, c, u_begin, u_end);
+    case 3: return mma_role<3, XT>(a, c, u_begin, u_end);
+    case 4: return mma_role<4, XT>(a, c, u_begin, u_end);
+    case 5: return mma_role<5, XT>(a, c, u_begin, u_end);
+    case 6: return mma_role<6, XT>(a, c, u_begin, u_end);
+    case 7: return mma_role<7, XT>(a, c, u_begin, u_end);
+    case 8: return mma_role<8, XT>(a, c, u_begin, u_end);
+    default: return mma_role<9, XT>(a, c, u_begin, u_end);
+    }
+}
+
+// Units [u_begin, u_end) of this CTA: a contiguous range, so that the tiles of
+// one channel follow each other and share one filter load.
 __device__ __forceinline__ void unit_range(const ToepArgs& a, int* u_begin, int* u_end)
 {
     *u_begin = static_cast<int>((static_cast<long long>(blockIdx.x) * a.num_units) / gridDim.x);
@@ -145,14 +250,14 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
 
-    uint8_t* bblk = smem;                                               // B panels (128-byte swizzle)
+    uint8_t* bblk = smem;                                               // NB blocks of B panels (128-byte swizzle)
     uint32_t* fwords = reinterpret_cast<uint32_t*>(smem + a.f_off);     // padded filter lines
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
-    uint64_t* b_full = bars + 0;
-    uint64_t* b_empty = bars + 1;
-    uint64_t* a_full = bars + 2;              // [kMaxA]
-    uint64_t* a_empty = bars + 2 + kMaxA;     // [kMaxA]
-    uint64_t* d_full = bars + 2 + 2 * kMaxA;
+    uint64_t* b_full = bars;                          // [kMaxB]
+    uint64_t* b_empty = bars + kMaxB;                 // [kMaxB]
+    uint64_t* a_full = bars + 2 * kMaxB;              // [kMaxA]
+    uint64_t* a_empty = a_full + kMaxA;               // [kMaxA]
+    uint64_t* d_full = a_empty + kMaxA;
     uint64_t* d_empty = d_full + 1;
     uint64_t* f_full = d_full + 2;
     uint64_t* f_empty = d_full + 3;
@@ -163,12 +268,16 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t na = static_cast<uint32_t>(a.na);
+    const uint32_t nb = static_cast<uint32_t>(a.NB);
+    const int ncol_sub = 8 * a.NH;                    // accumulator columns per sub-tile
     int u_begin, u_end;
     unit_range(a, &u_begin, &u_end);
 
     if (threadIdx.x == 0) {
-        mbar_init(b_full, 1);
-        mbar_init(b_empty, 1);
+        for (int b = 0; b < kMaxB; ++b) {
+            mbar_init(&b_full[b], 1);
+            mbar_init(&b_empty[b], 1);
+        }
         for (int b = 0; b < kMaxA; ++b) {
             mbar_init(&a_full[b], 128);
             mbar_init(&a_empty[b], 1);
@@ -194,7 +303,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         // Per unit: the filter lines when the channel changes (one bulk copy),
-        // then the B panels (one TMA box per 64 columns).
+        // then the B panels (one TMA box per 64 columns) into the next B block.
         if (lane == 0) {
             uint32_t ub = 0, fe = 0;
             int prev_c = -1;
@@ -211,13 +320,16 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                     ++fe;
                     prev_c = t.c;
                 }
-                if (!mbar_wait(b_empty, (ub & 1u) ^ 1u, abort_flag)) {
+                const uint32_t bb = ub % nb;
+                if (!mbar_wait(&b_empty[bb], ((ub / nb) & 1u) ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(b_full, a.b_bytes);
-                for (int pn = 0; pn * 64 < a.K; ++pn)
-                    tma_load_4d(bblk + pn * a.panel_bytes, &map_b, b_full, t.xb + 64 * pn, 8 * t.g, t.Y0 - a.py, t.c);
+                mbar_arrive_expect_tx(&b_full[bb], a.b_bytes);
+                uint8_t* blk = bblk + bb * a.b_bytes;
+                for (uint32_t pn = 0; pn < a.npanels; ++pn)
+                    tma_load_4d(blk + pn * a.panel_bytes, &map_b, &b_full[bb], t.xb + 64 * static_cast<int>(pn),
+                                8 * t.g, t.Y0 - a.py, t.c);
                 ++ub;
             }
             if (!ok) {
@@ -225,10 +337,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 *abort_flag = 1;
             }
             // the last copies have landed before the CTA may exit
-            if (ub > 0 && !mbar_wait(b_full, (ub - 1u) & 1u)) {
-                report_timeout(a.status);
-                *abort_flag = 1;
-            }
+            for (uint32_t k = (ub > nb ? ub - nb : 0); k < ub; ++k)
+                if (!mbar_wait(&b_full[k % nb], (k / nb) & 1u)) {
+                    report_timeout(a.status);
+                    *abort_flag = 1;
+                }
             if (fe > 0 && !mbar_wait(f_full, (fe - 1u) & 1u)) {
                 report_timeout(a.status);
                 *abort_flag = 1;
@@ -237,41 +350,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, 8 * a.NH, /*b_mn_major=*/false);
-            const uint32_t b_addr = smem_u32(bblk);
-            uint32_t ub = 0, step = 0;
-            bool ok = true;
-            for (int u = u_begin; u < u_end && ok; ++u) {
-                if (!mbar_wait(b_full, ub & 1u, abort_flag) || !mbar_wait(d_empty, (ub & 1u) ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                for (int i = 0; i < a.NI; ++i) {
-                    const uint32_t b = step % na;
-                    if (!mbar_wait(&a_full[b], (step / na) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a_tmem =
-                        tmem_base + static_cast<uint32_t>(a.a_col0) + b * static_cast<uint32_t>(a.a_cols);
-                    // B_i: rows (h', img) are panel rows (2h' + i, img); one shift step is one
-                    // 1024-byte swizzle atom, the row-group stride two atoms.
-                    for (int q = 0; q < (a.K >> 4); ++q) {
-                        const uint32_t start = b_addr + static_cast<uint32_t>(q >> 2) * a.panel_bytes +
-                                               static_cast<uint32_t>(i) * 1024u + static_cast<uint32_t>(q & 3) * 32u;
-                        const uint64_t bdesc = sw128_desc(start, 16, kP * 1024u);
-                        umma_f16_ts(tmem_base, a_tmem + 8u * q, bdesc, idesc, (i | q) != 0 ? 1u : 0u);
-                    }
-                    umma_commit(&a_empty[b]);   // A buffer free once these MMAs have read it
-                    ++step;
-                }
-                if (!ok) break;
-                umma_commit(d_full);
-                umma_commit(b_empty);
-                ++ub;
-            }
+            MmaCtx ctx{b_full, b_empty, a_full, a_empty, d_full, d_empty, abort_flag, tmem_base, smem_u32(bblk)};
+            const int kq = a.Ks >> 4;
+            const bool ok = a.XT == 1   ? mma_role_x<1>(kq, a, ctx, u_begin, u_end)
+                            : a.XT == 2 ? mma_role_x<2>(kq, a, ctx, u_begin, u_end)
+                                        : mma_role_x<4>(kq, a, ctx, u_begin, u_end);
             if (!ok) {
                 report_timeout(a.status);
                 *abort_flag = 1;
@@ -286,10 +369,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         // ----------------------------------------------------------- A builders
         const int quarter = warp & 3;
         const int m = quarter * 32 + lane;
-        const int p = m / kTW;
-        const int xl = m % kTW;
+        const int p = m / a.TW;
+        const int xl = m % a.TW;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t step = 0, fe = 0;
+        uint32_t ab = 0, aph = 0, fe = 0;
         int prev_c = -1;
         bool ok = true;
         for (int u = u_begin; u < u_end && ok; ++u) {
@@ -302,13 +385,14 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 ++fe;
                 prev_c = t.c;
             }
-            // A_i[m][j] = F[i-p][j + e], e = xb - x0 + px - xl; padded tap index t0 = e + kOff >= 0.
+            // A_i[m][j] = F[i-p][j + e], e = xb - x0 + px - xl (the same for every sub-tile);
+            // padded tap index t0 = e + kOff >= 0.
             const int t0 = t.xb - t.x0 + a.px - xl + kOff;
             const uint32_t* rowbase = fwords + (t0 >> 1);
             const bool odd = (t0 & 1) != 0;
             for (int i = 0; i < a.NI; ++i) {
-                const uint32_t b = step % na;
-                if (!mbar_wait(&a_empty[b], ((step / na) & 1u) ^ 1u, abort_flag)) {
+                const uint32_t b = ab;
+                if (!mbar_wait(&a_empty[b], aph ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -317,11 +401,14 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 const uint32_t taddr =
                     tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0) + b * static_cast<uint32_t>(a.a_cols);
                 const bool nonzero = ry >= 0 && ry < a.KY;
-                store_a(a.K >> 4, taddr, rowbase + (nonzero ? ry : 0) * a.half_l, odd, nonzero);
+                store_a(a.Ks >> 4, taddr, rowbase + (nonzero ? ry : 0) * a.half_l, odd, nonzero);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&a_full[b]);
-                ++step;
+                if (++ab == na) {
+                    ab = 0;
+                    aph ^= 1u;
+                }
             }
             // Done with this channel's filter lines: let the producer replace them.
             const bool last = u + 1 >= u_end || decode_unit(a, u + 1).c != t.c;
@@ -333,18 +420,18 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         }
     } else {
         // ------------------------------------------------------------- epilogue
-        // Two warps per TMEM lane quarter, each draining half of the columns into
-        // registers (as bf16 pairs) before releasing the accumulator.
+        // Two warps per TMEM lane quarter, each draining half of the accumulator
+        // columns into registers (as bf16 pairs) before releasing the accumulator.
         const int quarter = warp & 3;
         const int half = (warp - 6) >> 2;
         const int m = quarter * 32 + lane;
-        const int p = m / kTW;
-        const int xl = m % kTW;
+        const int p = m / a.TW;
+        const int xl = m % a.TW;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        const int ncol = 4 * a.NH;          // columns per half: 128 or 64
-        const int nch = ncol >> 5;          // 32-column chunks per half: 4 or 2
+        const int hcols = (a.XT * ncol_sub) >> 1;   // columns per half: at most 128
+        const int nch = hcols >> 5;                  // 32-column chunks per half: 1 .. 4
         const int64_t img_stride = a.Xso;
-        const int64_t hrow_stride = static_cast<int64_t>(kP) * a.N * a.Xso;
+        const int64_t hrow_stride = static_cast<int64_t>(a.P) * a.N * a.Xso;
         uint32_t ub = 0;
         bool ok = true;
         for (int u = u_begin; u < u_end; ++u) {
@@ -359,7 +446,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             for (int cc = 0; cc < 4; ++cc) {
                 if (cc < nch) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(half * ncol + cc * 32), v);
+                    tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(half * hcols + cc * 32), v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
@@ -368,27 +455,30 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             }
             tc_fence_before();
             mbar_arrive(d_empty);   // the accumulator may be overwritten now
-            const int x = t.x0 + xl;
-            if (x < a.Xo) {
-                // column n = half*ncol + k: h' = n >> 3, image 8g + (n & 7), row Y0 + 2h' + p
-                const int hp0 = (half * ncol) >> 3;
-                uint16_t* base = reinterpret_cast<uint16_t*>(a.dXp) +
-                                 ((static_cast<int64_t>(t.c) * a.Yo + t.Y0 + kP * hp0 + p) * a.N + 8 * t.g) * a.Xso + x;
-                const bool full = t.Y0 + kP * a.NH <= a.Yo && 8 * t.g + 8 <= a.N;
+            const bool full = t.Y0 + a.P * a.NH <= a.Yo && 8 * t.g + 8 <= a.N;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    if (cc < nch) {
+            for (int cc = 0; cc < 4; ++cc) {
+                if (cc < nch) {
+                    // a 32-column chunk lies inside one sub-tile (ncol_sub is a multiple of 32)
+                    const int col0 = half * hcols + cc * 32;
+                    const int sx = col0 / ncol_sub;
+                    const int n0 = col0 - sx * ncol_sub;          // column within the sub-tile
+                    const int x = t.x0 + sx * a.TW + xl;
+                    if (x < a.Xo) {
+                        const int hp0 = n0 >> 3;
+                        uint16_t* base = reinterpret_cast<uint16_t*>(a.dXp) +
+                                         ((static_cast<int64_t>(t.c) * a.Yo + t.Y0 + a.P * hp0 + p) * a.N + 8 * t.g) *
+                                             a.Xso + x;
 #pragma unroll
                         for (int k = 0; k < 16; ++k) {
-                            const int kk = cc * 32 + 2 * k;        // column within the half (even)
-                            const int hp = kk >> 3;
-                            const int img = kk & 7;
+                            const int hp = (2 * k) >> 3;              // h' offset inside the chunk
+                            const int img = (2 * k) & 7;
                             uint16_t* dst = base + hp * hrow_stride + img * img_stride;
                             const uint32_t v = pk[cc * 16 + k];
                             if (full) {
                                 dst[0] = static_cast<uint16_t>(v & 0xFFFFu);
                                 dst[img_stride] = static_cast<uint16_t>(v >> 16);
-                            } else if (t.Y0 + kP * (hp0 + hp) + p < a.Yo) {
+                            } else if (t.Y0 + a.P * (hp0 + hp) + p < a.Yo) {
                                 if (8 * t.g + img < a.N) dst[0] = static_cast<uint16_t>(v & 0xFFFFu);
                                 if (8 * t.g + img + 1 < a.N) dst[img_stride] = static_cast<uint16_t>(v >> 16);
                             }
@@ -416,118 +506,126 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 // Padded filter lines of every channel, in the plane orientation: line ry of
 // channel c is F[ry][rx] = W[KH-1-ry][KW-1-rx] (orientation 0) or
 // W[KH-1-rx][KW-1-ry] (orientation 1) at tap index rx + kOff, zero elsewhere;
-// word w of a line holds taps (2w - kOff, 2w + 1 - kOff).  f_words words per channel.
-__global__ void __launch_bounds__(128)
+// word w of a line holds taps (2w - kOff, 2w + 1 - kOff).  f_words words per
+// channel.  One CTA handles one line ry of 32 channels: the taps are read
+// channel-contiguous (coalesced) into shared memory, then each warp writes whole
+// lines.
+__global__ void __launch_bounds__(256)
     dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
                           int KY, int KX, int orient, int half_l, int f_words)
 {
-    const int c = blockIdx.x;
+    __shared__ uint16_t taps[64][34];   // [rx][channel]
+    const int ry = blockIdx.y;
+    const int c0 = blockIdx.x * 32;
     const unsigned short* w16 = reinterpret_cast<const unsigned short*>(filt);
-    for (int idx = threadIdx.x; idx < f_words; idx += blockDim.x) {
-        uint32_t packed = 0;
-        const int ry = idx / half_l;
-        const int w = idx - ry * half_l;
-        if (ry < KY) {
+    for (int idx = threadIdx.x; idx < KX * 32; idx += blockDim.x) {
+        const int rx = idx >> 5;
+        const int cl = idx & 31;
+        const int r = orient ? (KH - 1 - rx) : (KH - 1 - ry);
+        const int s = orient ? (KW - 1 - ry) : (KW - 1 - rx);
+        taps[rx][cl] = c0 + cl < C ? w16[(static_cast<int64_t>(r) * KW + s) * C + c0 + cl] : 0;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    for (int cl = warp; cl < 32; cl += blockDim.x >> 5) {
+        const int c = c0 + cl;
+        if (c >= C) break;
+        uint32_t* line = dst + static_cast<int64_t>(c) * f_words + static_cast<int64_t>(ry) * half_l;
+        for (int w = lane; w < half_l; w += 32) {
+            const int rx0 = 2 * w - kOff;
+            const uint32_t lo = (rx0 >= 0 && rx0 < KX) ? taps[rx0][cl] : 0u;
+            const uint32_t hi = (rx0 + 1 >= 0 && rx0 + 1 < KX) ? taps[rx0 + 1][cl] : 0u;
+            line[w] = lo | (hi << 16);
+        }
+        if (ry == KY - 1)   // zero the words that round the channel's block up to f_words
+            for (int w = KY * half_l + lane; w < f_words; w += 32) dst[static_cast<int64_t>(c) * f_words + w] = 0u;
+    }
+}
+
+// NHWC <-> planar [C][Y][N][Xs] for bf16.  The NHWC side addresses element
+// (n, y, x, c) at n*sN + y*sY + x*sX + c; the planar side at ((c*Y + y)*N + n)*Xs
+// + x.  A tile is 64 x-positions by 64 channels of one (n, y), moved as 16-byte
+// chunks through a shared-memory transpose.  Each CTA takes kRowsPerCta
+// consecutive y of one (n, x block, channel block): it loads all of their tiles
+// into registers first (eight 16-byte loads per thread in flight), then
+// transposes and stores them one after the other.
+constexpr int kRowsPerCta = 4;
+
+template <bool TO_PLANAR>
+__global__ void __launch_bounds__(256)
+    dw_transpose_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int N, int Y, int X,
+                        int Xs, int C, int64_t sN, int64_t sY, int64_t sX)
+{
+    __shared__ uint32_t tile[64][33];   // [row][pair]: rows are x (to planar) or c (from planar)
+    const int nct = (C + 63) >> 6;
+    const int ct = blockIdx.x % nct;
+    const int x0 = (blockIdx.x / nct) * 64;
+    const int c0 = ct * 64;
+    const int y0 = blockIdx.y * kRowsPerCta;
+    const int n = blockIdx.z;
+    uint4 v[kRowsPerCta][2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int rx = 2 * w + h - kOff;
-                if (rx >= 0 && rx < KX) {
-                    const int r = orient ? (KH - 1 - rx) : (KH - 1 - ry);
-                    const int s = orient ? (KW - 1 - ry) : (KW - 1 - rx);
-                    packed |= static_cast<uint32_t>(w16[(static_cast<int64_t>(r) * KW + s) * C + c]) << (16 * h);
+    for (int r = 0; r < kRowsPerCta; ++r) {
+        const int y = y0 + r;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int idx = threadIdx.x + 256 * k;
+            const int row = idx >> 3;          // x (to planar) or c (from planar)
+            const int col = (idx & 7) * 8;     // c chunk (to planar) or x chunk (from planar)
+            v[r][k] = make_uint4(0, 0, 0, 0);
+            if (y < Y) {
+                if (TO_PLANAR) {
+                    if (x0 + row < X && c0 + col < C)
+                        v[r][k] = *reinterpret_cast<const uint4*>(src + n * sN + y * sY +
+                                                                  static_cast<int64_t>(x0 + row) * sX + c0 + col);
+                } else {
+                    if (c0 + row < C && x0 + col < X)
+                        v[r][k] = *reinterpret_cast<const uint4*>(
+                            src + ((static_cast<int64_t>(c0 + row) * Y + y) * N + n) * Xs + x0 + col);
                 }
             }
         }
-        dst[static_cast<int64_t>(c) * f_words + idx] = packed;
     }
-}
-
-// NHWC -> planar [C][Y][N][Xs]: element (n, y, x, c) of the source sits at
-// n*sN + y*sY + x*sX + c.  One CTA moves a 64 (x) x 64 (c) tile of one (n, y).
-__global__ void __launch_bounds__(256)
-    dw_pack_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int N, int Y, int X,
-                   int Xs, int C, int64_t sN, int64_t sY, int64_t sX)
-{
-    __shared__ uint32_t tile[64][33];   // [x][c pair]
-    const int nct = (C + 63) >> 6;
-    const int ct = blockIdx.x % nct;
-    const int xt = blockIdx.x / nct;
-    const int y = blockIdx.y;
-    const int n = blockIdx.z;
-    const int c0 = ct * 64;
-    const int x0 = xt * 64;
-    for (int idx = threadIdx.x; idx < 512; idx += 256) {
-        const int xr = idx >> 3;
-        const int cc = (idx & 7) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (x0 + xr < X && c0 + cc < C)
-            v = *reinterpret_cast<const uint4*>(src + n * sN + y * sY + static_cast<int64_t>(x0 + xr) * sX + c0 + cc);
-        tile[xr][cc / 2 + 0] = v.x;
-        tile[xr][cc / 2 + 1] = v.y;
-        tile[xr][cc / 2 + 2] = v.z;
-        tile[xr][cc / 2 + 3] = v.w;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < 512; idx += 256) {
-        const int cr = idx >> 3;
-        const int xc = (idx & 7) * 8;
-        const int c = c0 + cr;
-        const int x = x0 + xc;
-        if (c >= C || x >= X) continue;
-        const int sh = (cr & 1) * 16;
-        uint32_t w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t lo = (tile[xc + 2 * k][cr >> 1] >> sh) & 0xFFFFu;
-            const uint32_t hi = (tile[xc + 2 * k + 1][cr >> 1] >> sh) & 0xFFFFu;
-            w[k] = lo | (hi << 16);
-        }
-        *reinterpret_cast<uint4*>(dst + ((static_cast<int64_t>(c) * Y + y) * N + n) * Xs + x) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-// planar [C][Y][N][Xs] -> NHWC (inverse of dw_pack_kernel).
-__global__ void __launch_bounds__(256)
-    dw_unpack_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int N, int Y, int X,
-                     int Xs, int C, int64_t sN, int64_t sY, int64_t sX)
-{
-    __shared__ uint32_t tile[64][33];   // [c][x pair]
-    const int nct = (C + 63) >> 6;
-    const int ct = blockIdx.x % nct;
-    const int xt = blockIdx.x / nct;
-    const int y = blockIdx.y;
-    const int n = blockIdx.z;
-    const int c0 = ct * 64;
-    const int x0 = xt * 64;
-    for (int idx = threadIdx.x; idx < 512; idx += 256) {
-        const int cr = idx >> 3;
-        const int xc = (idx & 7) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (c0 + cr < C && x0 + xc < X)
-            v = *reinterpret_cast<const uint4*>(src + ((static_cast<int64_t>(c0 + cr) * Y + y) * N + n) * Xs + x0 + xc);
-        tile[cr][xc / 2 + 0] = v.x;
-        tile[cr][xc / 2 + 1] = v.y;
-        tile[cr][xc / 2 + 2] = v.z;
-        tile[cr][xc / 2 + 3] = v.w;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < 512; idx += 256) {
-        const int xr = idx >> 3;
-        const int cc = (idx & 7) * 8;
-        const int x = x0 + xr;
-        const int c = c0 + cc;
-        if (x >= X || c >= C) continue;
-        const int sh = (xr & 1) * 16;
-        uint32_t w[4];
+    for (int r = 0; r < kRowsPerCta; ++r) {
+        const int y = y0 + r;
+        if (y >= Y) break;   // uniform across the CTA
+        if (r > 0) __syncthreads();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t lo = (tile[cc + 2 * k][xr >> 1] >> sh) & 0xFFFFu;
-            const uint32_t hi = (tile[cc + 2 * k + 1][xr >> 1] >> sh) & 0xFFFFu;
-            w[k] = lo | (hi << 16);
+        for (int k = 0; k < 2; ++k) {
+            const int idx = threadIdx.x + 256 * k;
+            const int row = idx >> 3;
+            const int col = (idx & 7) * 8;
+            tile[row][col / 2 + 0] = v[r][k].x;
+            tile[row][col / 2 + 1] = v[r][k].y;
+            tile[row][col / 2 + 2] = v[r][k].z;
+            tile[row][col / 2 + 3] = v[r][k].w;
         }
-        *reinterpret_cast<uint4*>(dst + n * sN + y * sY + static_cast<int64_t>(x) * sX + c) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int idx = threadIdx.x + 256 * k;
+            const int orow = idx >> 3;         // c (to planar) or x (from planar)
+            const int ocol = (idx & 7) * 8;    // x chunk (to planar) or c chunk (from planar)
+            const int sh = (orow & 1) * 16;
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t lo = (tile[ocol + 2 * j][orow >> 1] >> sh) & 0xFFFFu;
+                const uint32_t hi = (tile[ocol + 2 * j + 1][orow >> 1] >> sh) & 0xFFFFu;
+                w[j] = lo | (hi << 16);
+            }
+            if (TO_PLANAR) {
+                if (c0 + orow < C && x0 + ocol < X)
+                    *reinterpret_cast<uint4*>(dst + ((static_cast<int64_t>(c0 + orow) * Y + y) * N + n) * Xs + x0 +
+                                              ocol) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else {
+                if (x0 + orow < X && c0 + ocol < C)
+                    *reinterpret_cast<uint4*>(dst + n * sN + y * sY + static_cast<int64_t>(x0 + orow) * sX + c0 +
+                                              ocol) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
     }
 }
 
@@ -538,60 +636,84 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
 {
     if (!a.bf16 || a.S != 1) return false;
+    // Tile shapes (P row phases, NH row groups, XT sub-tiles of 128/P columns), in the
+    // order measured fastest on B200: N = 256 tiles (two row phases) first.  Smaller
+    // tiles issue more MMAs per output at a lower rate per MMA, so they serve only
+    // filters whose B block would not fit otherwise.  Among the two orientations the
+    // first fitting shape with fewer MMAs (rounds of tiles x shift steps x depth)
+    // wins.  The plan does not depend on the device, so the workspace size can be
+    // queried on the host.
+    constexpr int kPlanSms = 148;
+    static const int cand[][3] = {{2, 32, 1}, {2, 16, 1}, {4, 16, 2}, {4, 8, 2}, {8, 8, 4}, {8, 4, 4}};
+    // DGRAD_TC_TILE="orient,P,NH,XT" restricts the plan to that shape (testing and tuning).
+    int force[4] = {-1, -1, -1, -1};
+    if (const char* ft = getenv("DGRAD_TC_TILE"))
+        if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
     ToepPlan best{};
-    long long best_cost = 0;
+    double best_cost = 0;
     for (int orient = 0; orient < 2; ++orient) {
-        ToepPlan p{};
-        p.orient = orient;
-        p.KY = orient ? a.KW : a.KH;
-        p.KX = orient ? a.KH : a.KW;
-        p.py = orient ? (a.KW - 1 - a.pw) : (a.KH - 1 - a.ph);
-        p.px = orient ? (a.KH - 1 - a.ph) : (a.KW - 1 - a.pw);
-        p.Yi = orient ? a.Wo : a.Ho;
-        p.Xi = orient ? a.Ho : a.Wo;
-        p.Yo = orient ? a.W : a.H;
-        p.Xo = orient ? a.H : a.W;
-        p.Xsi = (p.Xi + 7) & ~7;
-        p.Xso = (p.Xo + 7) & ~7;
-        const int mis = (-p.px) - floor8(-p.px);
-        p.K = (kTW + p.KX - 1 + mis + 15) & ~15;
-        if (p.K > 144) continue;
-        p.NI = p.KY + kP - 1;
-        p.half_l = (p.K + kOff + 8) / 2;     // words per padded filter line
-        p.f_words = static_cast<int>(round_up(static_cast<size_t>(p.KY) * p.half_l, 4));
-        p.a_cols = ((p.K / 2) + 31) & ~31;
-        const int panels = (p.K + 63) / 64;
-        bool fits = false;
-        for (int nh : {32, 16}) {
-            p.NH = nh;
-            p.NR = kP * nh - 1 + p.KY;
+        ToepPlan g{};
+        g.orient = orient;
+        g.KY = orient ? a.KW : a.KH;
+        g.KX = orient ? a.KH : a.KW;
+        g.py = orient ? (a.KW - 1 - a.pw) : (a.KH - 1 - a.ph);
+        g.px = orient ? (a.KH - 1 - a.ph) : (a.KW - 1 - a.pw);
+        g.Yi = orient ? a.Wo : a.Ho;
+        g.Xi = orient ? a.Ho : a.Wo;
+        g.Yo = orient ? a.W : a.H;
+        g.Xo = orient ? a.H : a.W;
+        g.Xsi = (g.Xi + 7) & ~7;
+        g.Xso = (g.Xo + 7) & ~7;
+        const int mis = (-g.px) - floor8(-g.px);   // the same for every tile (x0 is a multiple of 8)
+        for (const auto& cd : cand) {
+            if (force[0] >= 0 && (force[0] != orient || force[1] != cd[0] || force[2] != cd[1] || force[3] != cd[2]))
+                continue;
+            ToepPlan p = g;
+            p.P = cd[0];
+            p.NH = cd[1];
+            p.XT = cd[2];
+            p.TW = 128 / p.P;
+            p.Ks = (p.TW + p.KX - 1 + mis + 15) & ~15;
+            if (p.Ks > 144) continue;
+            const int span = (p.XT - 1) * p.TW + p.Ks;
+            p.npanels = (span + 63) / 64;
+            p.NR = p.P * p.NH + p.KY - 1;
             if (p.NR > 256) continue;
-            p.a_col0 = 8 * nh;                               // the accumulator takes columns [0, 8*NH)
+            p.NI = p.KY + p.P - 1;
+            p.half_l = (p.Ks + kOff + 8) / 2;
+            p.f_words = static_cast<int>(round_up(static_cast<size_t>(p.KY) * p.half_l, 4));
+            p.a_cols = ((p.Ks / 2) + 31) & ~31;
+            const int ncols_d = p.XT * 8 * p.NH;
+            if (ncols_d > 256 || (ncols_d / 2) % 32 != 0) continue;
+            p.a_col0 = ncols_d;
             p.na = (static_cast<int>(kTmemCols) - p.a_col0) / p.a_cols;
             if (p.na < 2) continue;
             if (p.na > kMaxA) p.na = kMaxA;
             p.panel_bytes = static_cast<uint32_t>(p.NR) * 1024u;
-            p.b_bytes = static_cast<uint32_t>(panels) * p.panel_bytes;
-            p.f_off = p.b_bytes;
-            p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.f_words, 16));
-            // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
-            p.smem = p.bar_off + kNumBars * 8 + 16 + 1024;
-            if (p.smem < 120 * 1024) p.smem = 120 * 1024;
-            if (p.smem <= 227 * 1024) {
-                fits = true;
-                break;
+            p.b_bytes = static_cast<uint32_t>(p.npanels) * p.panel_bytes;
+            bool fits = false;
+            for (int nbuf = kMaxB; nbuf >= 1 && !fits; --nbuf) {
+                p.NB = nbuf;
+                p.f_off = static_cast<uint32_t>(nbuf) * p.b_bytes;
+                p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.f_words, 16));
+                // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
+                p.smem = p.bar_off + kNumBars * 8 + 16 + 1024;
+                if (p.smem < 120 * 1024) p.smem = 120 * 1024;
+                fits = p.smem <= 227 * 1024;
             }
-        }
-        if (!fits) continue;
-        const int num_yt = (p.Yo + kP * p.NH - 1) / (kP * p.NH);
-        const int num_xt = (p.Xo + kTW - 1) / kTW;
-        // MMA work per channel-image: tiles x shift steps x K x N
-        const long long cost = static_cast<long long>(num_yt) * num_xt * p.NI * p.K * p.NH;
-        if (!have || cost < best_cost) {
-            best = p;
-            best_cost = cost;
-            have = true;
+            if (!fits) continue;
+            const long long num_yt = (p.Yo + p.P * p.NH - 1) / (p.P * p.NH);
+            const long long num_xt = (p.Xo + p.XT * p.TW - 1) / (p.XT * p.TW);
+            const long long units = num_xt * num_yt * ((a.N + 7) / 8) * a.C;
+            const double rounds = static_cast<double>((units + kPlanSms - 1) / kPlanSms);
+            const double cost = rounds * p.NI * p.XT * (p.Ks / 16) * (8.0 * p.NH);
+            if (!have || cost < best_cost) {
+                best = p;
+                best_cost = cost;
+                have = true;
+            }
+            break;   // first fitting shape of this orientation
         }
     }
     if (!have) return false;
@@ -616,14 +738,15 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         const int64_t sN = static_cast<int64_t>(a.Ho) * a.Wo * C;
         const int64_t sY = p.orient ? C : static_cast<int64_t>(a.Wo) * C;
         const int64_t sX = p.orient ? static_cast<int64_t>(a.Wo) * C : C;
-        dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct), static_cast<unsigned>(p.Yi),
-                  static_cast<unsigned>(a.N));
-        dw_pack_kernel<<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N, p.Yi, p.Xi,
-                                                 p.Xsi, a.C, sN, sY, sX);
+        dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct),
+                  static_cast<unsigned>((p.Yi + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
+        dw_transpose_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N, p.Yi,
+                                                            p.Xi, p.Xsi, a.C, sN, sY, sX);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        dw_filter_pack_kernel<<<a.C, 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
-                                                       a.KW, p.KY, p.KX, p.orient, p.half_l, p.f_words);
+        dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
+        dw_filter_pack_kernel<<<fgrid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
+                                                         a.KW, p.KY, p.KX, p.orient, p.half_l, p.f_words);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -640,13 +763,17 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         t.KY = p.KY;
         t.py = p.py;
         t.px = p.px;
+        t.P = p.P;
+        t.TW = p.TW;
+        t.XT = p.XT;
         t.NH = p.NH;
-        t.K = p.K;
+        t.Ks = p.Ks;
         t.NR = p.NR;
         t.NI = p.NI;
         t.half_l = p.half_l;
-        t.num_xt = (p.Xo + kTW - 1) / kTW;
-        t.num_yt = (p.Yo + kP * p.NH - 1) / (kP * p.NH);
+        t.NB = p.NB;
+        t.num_xt = (p.Xo + p.XT * p.TW - 1) / (p.XT * p.TW);
+        t.num_yt = (p.Yo + p.P * p.NH - 1) / (p.P * p.NH);
         t.num_g = (a.N + 7) / 8;
         const long long units = static_cast<long long>(t.num_xt) * t.num_yt * t.num_g * a.C;
         if (units > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
@@ -656,6 +783,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         t.na = p.na;
         t.panel_bytes = p.panel_bytes;
         t.b_bytes = p.b_bytes;
+        t.npanels = static_cast<uint32_t>(p.npanels);
         t.f_words = static_cast<uint32_t>(p.f_words);
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;
         t.f_off = p.f_off;
@@ -672,10 +800,10 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         const int64_t sN = static_cast<int64_t>(a.H) * a.W * C;
         const int64_t sY = p.orient ? C : static_cast<int64_t>(a.W) * C;
         const int64_t sX = p.orient ? static_cast<int64_t>(a.W) * C : C;
-        dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct), static_cast<unsigned>(p.Yo),
-                  static_cast<unsigned>(a.N));
-        dw_unpack_kernel<<<grid, 256, 0, stream>>>(dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo, p.Xo, p.Xso,
-                                                   a.C, sN, sY, sX);
+        dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct),
+                  static_cast<unsigned>((p.Yo + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
+        dw_transpose_kernel<false><<<grid, 256, 0, stream>>>(dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo, p.Xo,
+                                                             p.Xso, a.C, sN, sY, sX);
     }
     return cudaGetLastError();
 }

@@ -82,7 +82,7 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 // swizzle, zero fill.
 struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
-    int NH, K, NR, NI, half_l, f_words, a_col0, a_cols, na;
+    int P, TW, XT, NH, Ks, NR, NI, NB, npanels, half_l, f_words, a_col0, a_cols, na;
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     size_t smem, ws_in, ws_out, ws_f;
 };

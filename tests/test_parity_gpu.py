@@ -297,6 +297,27 @@ def test_full_size_workloads(p):
     cb.check_status()
 
 
+TC_TILES = ["0,2,32,1", "0,2,16,1", "0,4,16,2", "0,4,8,2", "0,8,8,4", "0,8,4,4", "1,4,16,2", "1,8,8,4"]
+
+
+@pytest.mark.parametrize("tile", TC_TILES)
+def test_depthwise_tensor_core_tile_shapes(tile, monkeypatch):
+    """Every tile shape of the tensor-core depthwise kernel (orientation, row phases P, row groups NH,
+    sub-tiles XT), forced through DGRAD_TC_TILE, on a ragged problem (N = 9, odd extents)."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_TILE", tile)
+    p = P("tc_tile", "depthwise", "bf16", 9, 37, 41, 24, 24, 9, 7, 1, 4, 3, seed=160)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"tile {tile}")
+    cb.check_status()
+
+
 TC_FULL = [p for p in synthetic.all_problems() if p.variant == "tc"]
 
 
