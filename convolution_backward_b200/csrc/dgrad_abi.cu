@@ -126,6 +126,36 @@ bool encode_planar_bf16(CUtensorMap* map, const void* base, uint64_t X, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+// Maps of the depthwise transposes (128-byte swizzle, box rows of 64 elements):
+// NHWC (dims C, W, H, N) with a box of 64 channels by 64 positions along W
+// (orientation 0) or H (orientation 1), and planar [C][Y][N][Xs] (dims X, N, Y, C)
+// with a box of 64 x by 64 c.
+bool encode_nhwc_tr(CUtensorMap* map, const void* base, uint64_t N, uint64_t H, uint64_t W, uint64_t C, int orient)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {C, W, H, N};
+    const cuuint64_t strides[3] = {C * 2, W * C * 2, H * W * C * 2};
+    const cuuint32_t b[4] = {64, orient ? 1u : 64u, orient ? 64u : 1u, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_planar_tr(CUtensorMap* map, const void* base, uint64_t X, uint64_t N, uint64_t Y, uint64_t C, uint64_t Xs)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {X, N, Y, C};
+    const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
+    const cuuint32_t b[4] = {64, 1, 1, 64};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int env_int(const char* name, int dflt)
@@ -357,12 +387,25 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
     a.filt = W;
     a.dX = dX;
     a.status = st->status;
-    CUtensorMap map_b;
-    if (!encode_planar_bf16(&map_b, workspace, static_cast<uint64_t>(plan.Xi), static_cast<uint64_t>(a.N),
+    dgrad::ToepMaps maps{};
+    if (!encode_planar_bf16(&maps.b, workspace, static_cast<uint64_t>(plan.Xi), static_cast<uint64_t>(a.N),
                             static_cast<uint64_t>(plan.Yi), static_cast<uint64_t>(a.C),
                             static_cast<uint64_t>(plan.Xsi), static_cast<unsigned>(plan.NR)))
         return cuda_fail(cudaErrorInvalidValue);
-    cudaError_t e = dgrad::launch_dw_toeplitz(a, plan, map_b, workspace, st->sms, static_cast<cudaStream_t>(stream));
+    // TMA transposes when every map encodes (DGRAD_TC_TRANSPOSE=cuda selects the CUDA-core ones)
+    const void* dXp = static_cast<const uint8_t*>(workspace) + plan.ws_in;
+    const char* trm = getenv("DGRAD_TC_TRANSPOSE");
+    maps.tma_transpose =
+        !(trm && strcmp(trm, "cuda") == 0) &&
+        encode_nhwc_tr(&maps.pack_src, dY, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.Ho),
+                       static_cast<uint64_t>(a.Wo), static_cast<uint64_t>(a.C), plan.orient) &&
+        encode_planar_tr(&maps.pack_dst, workspace, static_cast<uint64_t>(plan.Xi), static_cast<uint64_t>(a.N),
+                         static_cast<uint64_t>(plan.Yi), static_cast<uint64_t>(a.C), static_cast<uint64_t>(plan.Xsi)) &&
+        encode_planar_tr(&maps.unpack_src, dXp, static_cast<uint64_t>(plan.Xo), static_cast<uint64_t>(a.N),
+                         static_cast<uint64_t>(plan.Yo), static_cast<uint64_t>(a.C), static_cast<uint64_t>(plan.Xso)) &&
+        encode_nhwc_tr(&maps.unpack_dst, dX, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.H),
+                       static_cast<uint64_t>(a.W), static_cast<uint64_t>(a.C), plan.orient);
+    cudaError_t e = dgrad::launch_dw_toeplitz(a, plan, maps, workspace, st->sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 

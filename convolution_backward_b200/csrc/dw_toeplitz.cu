@@ -629,6 +629,125 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// The same NHWC <-> planar move with TMA on both sides: a persistent kernel
+// walks 64 x 64 tiles with a four-deep ring of loaded tiles (128-byte swizzle,
+// rows of 64 elements), transposes each in-warp with ldmatrix.trans and
+// stmatrix (conflict-free on swizzled rows), and writes it back with a TMA
+// store, which clips the ragged edges.  Tile t = ((n*Y + y)*nxb + xb)*ncb + cb.
+// src_map and dst_map are the NHWC map (dims C, W, H, N; box 64 channels by 64
+// positions along x) and the planar map (dims X, N, Y, C; box 64 x by 64 c), in
+// the order of the move.
+constexpr int kTrStages = 4;
+
+struct TrArgs {
+    int to_planar, orient, N, Y, nxb, ncb, ntiles;
+    int* status;
+};
+
+__device__ __forceinline__ void tr_coords(const TrArgs& a, int t, bool nhwc_side, int (&c)[4])
+{
+    const int cb = t % a.ncb;
+    int q = t / a.ncb;
+    const int xb = q % a.nxb;
+    q /= a.nxb;
+    const int y = q % a.Y;
+    const int n = q / a.Y;
+    if (nhwc_side) {   // (C, W, H, N): x is W in orientation 0, H in orientation 1
+        c[0] = cb * 64;
+        c[1] = a.orient ? y : xb * 64;
+        c[2] = a.orient ? xb * 64 : y;
+        c[3] = n;
+    } else {           // (X, N, Y, C)
+        c[0] = xb * 64;
+        c[1] = n;
+        c[2] = y;
+        c[3] = cb * 64;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    dw_transpose_tma_kernel(const __grid_constant__ CUtensorMap src_map, const __grid_constant__ CUtensorMap dst_map,
+                            const __grid_constant__ TrArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* in_t = smem;                                  // kTrStages tiles of 8 KB
+    uint8_t* out_t = smem + kTrStages * 8192;              // 2 tiles of 8 KB
+    uint64_t* full = reinterpret_cast<uint64_t*>(out_t + 2 * 8192);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const bool src_nhwc = a.to_planar != 0;
+    if (tid == 0) {
+        for (int s = 0; s < kTrStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    int issued[kTrStages] = {0, 0, 0, 0};   // loads thread 0 has issued into each stage
+    if (tid == 0) {
+        tma_prefetch_desc(&src_map);
+        tma_prefetch_desc(&dst_map);
+        for (int s = 0; s < kTrStages; ++s) {
+            const int t = blockIdx.x + s * gridDim.x;
+            if (t >= a.ntiles) break;
+            int c[4];
+            tr_coords(a, t, src_nhwc, c);
+            mbar_arrive_expect_tx(&full[s], 8192);
+            tma_load_4d(in_t + s * 8192, &src_map, &full[s], c[0], c[1], c[2], c[3]);
+            ++issued[s];
+        }
+    }
+    bool aborted = false;
+    int k = 0;
+    for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++k) {
+        const int s = k % kTrStages;
+        const int o = k & 1;
+        const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((k / kTrStages) & 1));
+        if (tid == 0 && k >= 2) bulk_wait_group_read<1>();   // the store of tile k-2 has read out[o]
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) report_timeout(a.status);
+            aborted = true;
+            break;
+        }
+        // warp w transposes the eight 8x8 blocks of rows 8w .. 8w+7: block (w, j) of the
+        // input becomes block (j, w) of the output
+        const uint32_t in_base = smem_u32(in_t + s * 8192);
+        const uint32_t out_base = smem_u32(out_t + o * 8192);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int m = lane >> 3;                 // matrix of this lane's address
+            const int j = 4 * h + m;                 // input chunk (column block)
+            const int rin = 8 * warp + (lane & 7);   // input row
+            uint32_t r[4];
+            ldmatrix_x4_trans(in_base + rin * 128 + ((j ^ (rin & 7)) << 4), r);
+            const int rout = 8 * j + (lane & 7);     // output row
+            stmatrix_x4(out_base + rout * 128 + ((warp ^ (rout & 7)) << 4), r);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            int c[4];
+            tr_coords(a, t, !src_nhwc, c);
+            tma_store_4d(&dst_map, out_t + o * 8192, c[0], c[1], c[2], c[3]);
+            bulk_commit_group();
+            const int tn = t + kTrStages * gridDim.x;
+            if (tn < a.ntiles) {
+                tr_coords(a, tn, src_nhwc, c);
+                mbar_arrive_expect_tx(&full[s], 8192);
+                tma_load_4d(in_t + s * 8192, &src_map, &full[s], c[0], c[1], c[2], c[3]);
+                ++issued[s];
+            }
+        }
+    }
+    if (tid == 0) {
+        if (aborted)   // let the loads still in flight land (bounded) before the CTA exits
+            for (int s = 0; s < kTrStages; ++s)
+                if (issued[s] > 0) mbar_wait(&full[s], static_cast<uint32_t>((issued[s] - 1) & 1));
+        bulk_wait_group<0>();   // every store has completed before the CTA exits
+    }
+}
+
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
@@ -724,9 +843,29 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
     return true;
 }
 
-cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtensorMap& map_b, void* ws,
-                               int num_sms, cudaStream_t stream)
+cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMaps& maps, void* ws, int num_sms,
+                               cudaStream_t stream)
 {
+    const CUtensorMap& map_b = maps.b;
+    const int tr_smem = (kTrStages + 2) * 8192 + kTrStages * 8 + 1024;
+    if (maps.tma_transpose) {
+        cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_transpose_tma_kernel), tr_smem);
+        if (e != cudaSuccess) return e;
+    }
+    auto tma_transpose = [&](const CUtensorMap& src, const CUtensorMap& dst, bool to_planar, int Y, int X) {
+        TrArgs t{};
+        t.to_planar = to_planar ? 1 : 0;
+        t.orient = p.orient;
+        t.N = a.N;
+        t.Y = Y;
+        t.nxb = (X + 63) / 64;
+        t.ncb = (a.C + 63) / 64;
+        t.ntiles = a.N * Y * t.nxb * t.ncb;
+        t.status = a.status;
+        const int grid = t.ntiles < 4 * num_sms ? t.ntiles : 4 * num_sms;   // four CTAs per SM
+        dw_transpose_tma_kernel<<<grid, 256, tr_smem, stream>>>(src, dst, t);
+        return cudaGetLastError();
+    };
     if (a.N <= 0) return cudaSuccess;
     auto* dYp = static_cast<__nv_bfloat16*>(ws);
     auto* dXp = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + p.ws_in);
@@ -738,11 +877,16 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         const int64_t sN = static_cast<int64_t>(a.Ho) * a.Wo * C;
         const int64_t sY = p.orient ? C : static_cast<int64_t>(a.Wo) * C;
         const int64_t sX = p.orient ? static_cast<int64_t>(a.Wo) * C : C;
-        dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct),
-                  static_cast<unsigned>((p.Yi + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
-        dw_transpose_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N, p.Yi,
-                                                            p.Xi, p.Xsi, a.C, sN, sY, sX);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e;
+        if (maps.tma_transpose) {
+            e = tma_transpose(maps.pack_src, maps.pack_dst, true, p.Yi, p.Xi);
+        } else {
+            dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct),
+                      static_cast<unsigned>((p.Yi + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
+            dw_transpose_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N,
+                                                                p.Yi, p.Xi, p.Xsi, a.C, sN, sY, sX);
+            e = cudaGetLastError();
+        }
         if (e != cudaSuccess) return e;
         dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
         dw_filter_pack_kernel<<<fgrid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
@@ -800,10 +944,15 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtenso
         const int64_t sN = static_cast<int64_t>(a.H) * a.W * C;
         const int64_t sY = p.orient ? C : static_cast<int64_t>(a.W) * C;
         const int64_t sX = p.orient ? static_cast<int64_t>(a.W) * C : C;
-        dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct),
-                  static_cast<unsigned>((p.Yo + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
-        dw_transpose_kernel<false><<<grid, 256, 0, stream>>>(dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo, p.Xo,
-                                                             p.Xso, a.C, sN, sY, sX);
+        if (maps.tma_transpose) {
+            cudaError_t e = tma_transpose(maps.unpack_src, maps.unpack_dst, false, p.Yo, p.Xo);
+            if (e != cudaSuccess) return e;
+        } else {
+            dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct),
+                      static_cast<unsigned>((p.Yo + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
+            dw_transpose_kernel<false><<<grid, 256, 0, stream>>>(dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo,
+                                                                 p.Xo, p.Xso, a.C, sN, sY, sX);
+        }
     }
     return cudaGetLastError();
 }

@@ -86,9 +86,19 @@ struct ToepPlan {
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     size_t smem, ws_in, ws_out, ws_f;
 };
+// Tensor maps of one call: b as above; for the transposes (when tma_transpose),
+// the NHWC maps of dY and dX (dims C, W, H, N; box 64 channels by 64 positions
+// along the plane's x axis: W in orientation 0, H in orientation 1) and the
+// planar maps of the workspace planes (dims X, N, Y, C; box 64 x by 64 c), all
+// with the 128-byte swizzle.  Without them the transposes run on CUDA cores.
+struct ToepMaps {
+    CUtensorMap b;
+    CUtensorMap pack_src, pack_dst, unpack_src, unpack_dst;
+    bool tma_transpose;
+};
 bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* p);
-cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const CUtensorMap& map_b, void* ws,
-                               int num_sms, cudaStream_t stream);
+cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMaps& maps, void* ws, int num_sms,
+                               cudaStream_t stream);
 
 // Row-streaming kernel with a circular shared-memory accumulator ring (any S <= 8).
 cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);

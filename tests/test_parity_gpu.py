@@ -193,6 +193,9 @@ TC_SMALL = [
     P("tc51x5", "depthwise", "bf16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=153),
     P("tc64x64", "depthwise", "bf16", 1, 70, 66, 8, 8, 64, 64, 1, 32, 31, seed=155),
     P("tc17x17_nonsame", "depthwise", "bf16", 10, 40, 33, 16, 16, 17, 17, 1, 3, 11, seed=156),
+    P("tc11x9_c136_ragged_x", "depthwise", "bf16", 3, 37, 70, 136, 136, 11, 9, 1, 5, 4, seed=157),
+    P("tc9x21_c64_long_w", "depthwise", "bf16", 9, 66, 45, 64, 64, 9, 21, 1, 4, 10, seed=158),
+    P("tc21x9_c192_long_h", "depthwise", "bf16", 2, 45, 67, 192, 192, 21, 9, 1, 10, 4, seed=159),
     P("tc5x51", "depthwise", "bf16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=154),
 ]
 
@@ -294,6 +297,22 @@ def test_full_size_workloads(p):
     err = (out.float() - tref).abs().max().item()
     assert err / (tref.abs().max().item() + 1e-6) <= 1e-2
     import convolution_backward_b200 as cb
+    cb.check_status()
+
+
+@pytest.mark.parametrize("p", [q for q in TC_SMALL if q.C >= 64], ids=[q.name for q in TC_SMALL if q.C >= 64])
+def test_depthwise_tensor_core_cuda_transposes(p, monkeypatch):
+    """The tensor-core path with its transposes on CUDA cores (DGRAD_TC_TRANSPOSE=cuda) instead of TMA."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_TRANSPOSE", "cuda")
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/cuda transposes")
     cb.check_status()
 
 
