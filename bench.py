@@ -161,8 +161,16 @@ def _sample_call(p, inp, n, c):
     """Oracle arguments for a bounded sample of problem p and the nominal FLOPs it covers.
 
     Depthwise: the first n images and first c channels (channels of a depthwise
-    dgrad are independent).  Pointwise: the first n*c rows of dY[M, K] as n
-    pseudo-images of c rows (rows of a pointwise dgrad are independent)."""
+    dgrad are independent).  Dense: the first n images and the first c dX
+    channels (each dX channel reads only its own filter slice).  Pointwise: the
+    first n*c rows of dY[M, K] as n pseudo-images of c rows (rows of a pointwise
+    dgrad are independent)."""
+    if p.kind == "dense":
+        dy = inp.dy[:n]
+        w = np.ascontiguousarray(inp.w[:, :, :, :c].transpose(2, 0, 1, 3))   # (K, KH, KW, c): grouped layout
+        kw = dict(kind="grouped", groups=1, C=c, H=p.H, W=p.W, KH=p.KH, KW=p.KW, S=p.stride, ph=p.pad_h,
+                  pw=p.pad_w)
+        return dy, w, kw, p.nominal_flops() * n * c // (p.N * p.C)
     if p.kind == "pointwise":
         rows = n * c
         dy = inp.dy.reshape(-1, p.K)[:rows].reshape(n, 1, c, p.K)
@@ -184,15 +192,16 @@ def oracle_sample_plan(problems, inputs, budget_s: float):
     plan = []
     for p in problems:
         inp = inputs[p.name]
-        n = min(p.N, threads) if p.kind == "depthwise" else threads
-        full_c = p.C if p.kind == "depthwise" else (p.N * p.H * p.W) // n
-        c = min(full_c, 8 if p.kind == "depthwise" else 64)
+        per_image = p.kind in ("depthwise", "dense")
+        n = min(p.N, threads) if per_image else threads
+        full_c = p.C if per_image else (p.N * p.H * p.W) // n
+        c = min(full_c, 8 if per_image else 64)
         dy, w, kw, _ = _sample_call(p, inp, n, c)
         t0 = time.perf_counter()
         oracle.dgrad(dy, w, **kw)
         dt = max(time.perf_counter() - t0, 1e-4)
         c = int(max(1, min(full_c, c * per / dt)))
-        if p.kind == "depthwise" and c >= 8:
+        if per_image and c >= 8:
             c -= c % 8
         plan.append((p, n, c))
     return plan, threads
@@ -251,7 +260,8 @@ KERNEL_SOURCE = {"pointwise": {"bf16": "convolution_backward_b200/csrc/pointwise
                  "rowstream": "convolution_backward_b200/csrc/dw_rowstream.cu",
                  "rowstream_fast": "convolution_backward_b200/csrc/dw_rowstream_fast.cu",
                  "tile": "convolution_backward_b200/csrc/dw_tile.cu",
-                 "toeplitz": "convolution_backward_b200/csrc/dw_toeplitz.cu"}
+                 "toeplitz": "convolution_backward_b200/csrc/dw_toeplitz.cu",
+                 "dense": "convolution_backward_b200/csrc/dense_tc.cu"}
 
 
 def kernel_of(p):
@@ -259,6 +269,8 @@ def kernel_of(p):
         return "pw_tc_splitk_kernel", KERNEL_SOURCE["pointwise"]["bf16"]
     if p.variant == "tc":
         return "dw_toeplitz_kernel", KERNEL_SOURCE["toeplitz"]
+    if p.kind == "dense":
+        return "dense_tc_kernel", KERNEL_SOURCE["dense"]
     if p.kind == "pointwise":
         return ("pw_tc_pair_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
     if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
@@ -312,6 +324,8 @@ def run_ours(args, world, rank, local):
                             out=out)
         elif p.kind == "pointwise":
             cb.pointwise(dy, w, out=out)
+        elif p.kind == "dense":
+            cb.dense(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
         else:
             cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
 
@@ -404,7 +418,7 @@ def run_ours(args, world, rank, local):
         tf = fl / (ms * 1e-3) / 1e12
         gbs = by / (ms * 1e-3) / 1e9
         t_bytes = by / (hbm * 1e9)
-        if (p.kind == "pointwise" and p.dtype == "bf16") or p.variant == "tc":
+        if (p.kind in ("pointwise", "dense") and p.dtype == "bf16") or p.variant == "tc":
             # tensor-core paths: nominal FLOPs against the bf16 tensor peak (the banded-Toeplitz
             # depthwise issues about 3x its nominal FLOPs as MMAs; the fraction stays nominal)
             t_flop = fl / (bf16_peak * 1e12)
@@ -430,7 +444,7 @@ def run_ours(args, world, rank, local):
     dom = max(range(len(problems)), key=lambda j: kern_ms[j])
     dp = problems[dom]
     dk = per_kernel[dom]
-    if (dp.kind == "pointwise" and dp.dtype == "bf16") or dp.variant == "tc":
+    if (dp.kind in ("pointwise", "dense") and dp.dtype == "bf16") or dp.variant == "tc":
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": bf16_peak, "unit": "TFLOP/s",
                 "frac": round(dk["tflops"] / bf16_peak, 4), "traffic": dk["dram_bytes_per_launch"]}
     elif dk["binding"] == "hbm":

@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwise_tc", "depthwise_tc_workspace_bytes", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwise_tc", "depthwise_tc_workspace_bytes", "dense", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -99,6 +99,8 @@ def lib():
             L.dgrad_pointwise_splitk_workspace.restype = ctypes.c_int
             L.dgrad_pointwise_splitk_noalloc.argtypes = [P(Problem), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
             L.dgrad_pointwise_splitk_noalloc.restype = ctypes.c_int
+            L.dgrad_dense.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp]
+            L.dgrad_dense.restype = ctypes.c_int
             L.dgrad_depthwise_tc.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp, ctypes.c_size_t, vp]
             L.dgrad_depthwise_tc.restype = ctypes.c_int
             L.dgrad_depthwise_tc_workspace.argtypes = [P(Problem), P(ctypes.c_size_t)]
@@ -255,6 +257,36 @@ def depthwise(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, mode="auto",
             raise ValueError("out has the wrong shape or dtype")
     _check(lib().dgrad_depthwise(ctypes.byref(prob), _dtype_code(dY), DW_MODES[mode], dY.data_ptr(),
                                  W.data_ptr(), out.data_ptr(), _stream_ptr(stream)), "dgrad_depthwise")
+    return out
+
+
+def dense(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=None, stream=None, **kw):
+    """Dense (ungrouped) dgrad on the tensor cores (bf16; dgrad_dense): dY (N,Ho,Wo,K),
+    W (KH,KW,K,C) -> dX (N,H,W,C).  H and W_out (alias ``Wd``) are dX's spatial extents."""
+    import torch
+    if W_out is None:
+        W_out = kw.pop("Wd")
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 4 or W.shape[2] != dY.shape[3]:
+        raise ValueError("expected dY (N,Ho,Wo,K) and W (KH,KW,K,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
+    N, Ho, Wo, K = dY.shape
+    KH, KW, _, C = W.shape
+    eho, ewo = out_dims(H, W_out, KH, KW, stride, pad_h, pad_w)
+    if (eho, ewo) != (Ho, Wo):
+        raise ValueError(f"dY spatial extent {(Ho, Wo)} does not match the geometry ({eho}, {ewo})")
+    if out is None:
+        out = torch.empty((N, H, W_out, C), dtype=dY.dtype, device=dY.device)
+    else:
+        _need_cuda(out)
+        if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
+            raise ValueError("out has the wrong shape or dtype")
+    prob = Problem(N, H, W_out, C, K, KH, KW, stride, pad_h, pad_w)
+    _check(lib().dgrad_dense(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(), out.data_ptr(),
+                             _stream_ptr(stream)), "dgrad_dense")
     return out
 
 

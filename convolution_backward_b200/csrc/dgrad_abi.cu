@@ -326,6 +326,70 @@ dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 
+dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W, void* dX,
+                           void* stream)
+{
+    int64_t Ho = 0, Wo = 0;
+    int pw = 0;
+    dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
+    if (s != DGRAD_OK) return s;
+    if (dtype != DGRAD_BF16) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->KH > 64 || prob->KW > 64 || prob->stride > 64) return DGRAD_ERR_UNSUPPORTED;
+    if (prob->K > 65536 || prob->C > 65536 || prob->H > (1 << 24) || prob->W > (1 << 24) || prob->N > (1 << 24))
+        return DGRAD_ERR_UNSUPPORTED;
+    if (prob->N == 0) return DGRAD_OK;
+    if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (prob->K * 2) % 16 || (prob->C * 2) % 16)
+        return DGRAD_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    s = device_state(&st);
+    if (s != DGRAD_OK) return s;
+    dgrad::DenseArgs d{};
+    d.dX = static_cast<__nv_bfloat16*>(dX);
+    d.status = st->status;
+    d.N = static_cast<int>(prob->N);
+    d.H = static_cast<int>(prob->H);
+    d.W = static_cast<int>(prob->W);
+    d.C = static_cast<int>(prob->C);
+    d.K = static_cast<int>(prob->K);
+    d.Ho = static_cast<int>(Ho);
+    d.Wo = static_cast<int>(Wo);
+    d.KH = prob->KH;
+    d.KW = prob->KW;
+    d.S = prob->stride;
+    d.ph = prob->pad_h;
+    d.pw = pw;
+    dgrad::plan_dense(&d);
+    auto enc = tensor_map_encoder();
+    if (!enc) return cuda_fail(cudaErrorInvalidValue);
+    CUtensorMap map_a, map_b;
+    {
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(prob->K), static_cast<cuuint64_t>(Wo),
+                                    static_cast<cuuint64_t>(Ho), static_cast<cuuint64_t>(prob->N)};
+        const cuuint64_t strides[3] = {dims[0] * 2, dims[1] * dims[0] * 2, dims[2] * dims[1] * dims[0] * 2};
+        const cuuint32_t box[4] = {64, 16, 8, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (enc(&map_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(dY), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cuda_fail(cudaErrorInvalidValue);
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(prob->C), static_cast<cuuint64_t>(prob->K),
+                                    static_cast<cuuint64_t>(prob->KH) * static_cast<cuuint64_t>(prob->KW)};
+        const cuuint64_t strides[2] = {dims[0] * 2, dims[1] * dims[0] * 2};
+        const cuuint32_t box[3] = {64, 64, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&map_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cuda_fail(cudaErrorInvalidValue);
+    }
+    const int bn = env_int("DGRAD_DENSE_BN", prob->C <= 64 ? 64 : 128);
+    cudaError_t e = dgrad::launch_dense_tc(d, map_a, map_b, bn, st->sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
 // Shared checks for the tensor-core depthwise entry points: stride-1 depthwise,
 // bf16, extents within the kernels' 32-bit indexing and grid limits, and a tile
 // plan that fits one SM.

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -49,6 +50,22 @@ int pointwise_splitk_auto(const PwArgs& a, int num_sms);
 size_t pointwise_splitk_workspace_bytes(const PwArgs& a, int splits);
 cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                        int splits, float* ws, int num_sms, cudaStream_t stream);
+
+// Dense (ungrouped) KH x KW dgrad on tcgen05, by output phase (S*S sub-GEMMs),
+// bf16.  W is [KH][KW][K][C].  map_a covers dY as a 4-D bf16 tensor (K, Wo, Ho,
+// N) with a 64 x 16 x 8 x 1 box and the 128-byte swizzle; map_b covers W as a
+// 3-D bf16 tensor (C, K, KH*KW) with a 64 x 64 x 1 box and the 128-byte swizzle.
+// plan_dense fills the phase-grid fields (hq_min, wq_min, nth, ntw) from the
+// geometry; bn is the channel tile (64, 128 or 256).
+struct DenseArgs {
+    __nv_bfloat16* dX;
+    int* status;
+    int N, H, W, C, K, Ho, Wo, KH, KW, S, ph, pw;
+    int hq_min, wq_min, nth, ntw, nc, num_tiles;
+};
+void plan_dense(DenseArgs* d);
+cudaError_t launch_dense_tc(const DenseArgs& d, const CUtensorMap& map_a, const CUtensorMap& map_b, int bn,
+                            int num_sms, cudaStream_t stream);
 
 // Keep a CUDA error code for dgrad_last_cuda_error (entry points defined
 // outside the ABI file report their failures through this).

@@ -9,7 +9,8 @@ textbook one, Ho = floor((H + 2*pad_h - KH)/stride) + 1, with Wo from pad_w.
 Recipe (one per workload, in this order):
   1. rng = numpy.random.default_rng(seed)
   2. dY: draw in float64 in logical NHWC order and shape (N, Ho, Wo, K)
-  3. W : draw in float64 in its storage layout ((K, C) pointwise, (KH, KW, C) depthwise)
+  3. W : draw in float64 in its storage layout ((K, C) pointwise, (KH, KW, C) depthwise,
+     (KH, KW, K, C) dense)
   4. cast to float32; for bf16 workloads round to bf16 with round-to-nearest-even.
 Distributions: "normal" is N(0, var) with ``var`` the variance (std = sqrt(var));
 "uniform" is U[-1, 1].  A workload with several problems (the non-square and
@@ -27,7 +28,7 @@ import numpy as np
 @dataclass(frozen=True)
 class Problem:
     name: str
-    kind: str            # "pointwise" | "depthwise"
+    kind: str            # "pointwise" | "depthwise" | "dense"
     dtype: str           # "f32" | "bf16"
     N: int
     H: int
@@ -56,7 +57,7 @@ class Problem:
 
     @property
     def groups(self) -> int:
-        return 1 if self.kind == "pointwise" else self.C
+        return self.C if self.kind == "depthwise" else 1
 
     @property
     def dy_shape(self):
@@ -64,7 +65,11 @@ class Problem:
 
     @property
     def w_shape(self):
-        return (self.K, self.C) if self.kind == "pointwise" else (self.KH, self.KW, self.C)
+        if self.kind == "pointwise":
+            return (self.K, self.C)
+        if self.kind == "dense":
+            return (self.KH, self.KW, self.K, self.C)
+        return (self.KH, self.KW, self.C)
 
     @property
     def dx_shape(self):
@@ -123,6 +128,11 @@ EXTRA_WORKLOADS: dict[str, list[Problem]] = {
                                       K=2048, seed=5, w_var=1.0 / 2048, variant="splitk")],
     "pw_bf16_smallm": [Problem("pw_bf16_smallm", "pointwise", "bf16", N=2, H=14, W=14, C=512, K=2048,
                                seed=5, w_var=1.0 / 2048)],
+    # dense (ungrouped) 3x3 dgrad through dgrad_dense, stride 1 and stride 2
+    "dense3x3_bf16": [Problem("dense3x3_bf16", "dense", "bf16", N=32, H=28, W=28, C=256, K=256, KH=3, KW=3,
+                              pad_h=1, pad_w=1, seed=6, w_var=1.0 / 2304)],
+    "dense3x3s2_bf16": [Problem("dense3x3s2_bf16", "dense", "bf16", N=32, H=56, W=56, C=128, K=256, KH=3, KW=3,
+                                stride=2, pad_h=1, pad_w=1, seed=7, w_var=1.0 / 2304)],
     # the large stride-1 depthwise problems through the FP32 rotated-filter kernel (dgrad_depthwise)
     "dw_large_fp32": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_fp32", variant=""),
                       WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_fp32", variant=""),

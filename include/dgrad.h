@@ -146,6 +146,18 @@ dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int
 dgrad_status_t dgrad_pointwise_splitk_noalloc(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
                                               const void* dY, const void* W, void* dX, void* stream);
 
+/* Dense (ungrouped, groups = 1) dgrad with a KH x KW filter and any stride, on
+ * the tcgen05 tensor cores; W is [KH][KW][K][C] (tap-major: each tap is a
+ * pointwise [K][C] matrix).  The pages' main dgrad engine decomposes a strided
+ * dgrad by output phase into stride*stride sub-GEMMs ("add the pointwise fast
+ * path dgrad was missing", Technical Details); here each phase's GEMM sums, over
+ * the phase's taps, products of a shifted window of dY (K deep) with that tap's
+ * [K][C] matrix, so no im2col buffer is built.  DGRAD_BF16 only (else
+ * DGRAD_ERR_UNSUPPORTED); KH, KW, stride <= 64; K and C multiples of 8; padding
+ * any value >= 0 that leaves Ho, Wo >= 1. */
+dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W, void* dX,
+                           void* stream);
+
 /* Depthwise dgrad (groups = C; requires K == C, else DGRAD_ERR_UNSUPPORTED).
  * Rotated-filter mode requires stride 1, KH and KW <= 64 and
  * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1 (the rotated padding KH-1-pad_h and

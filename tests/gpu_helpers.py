@@ -41,22 +41,37 @@ def run_gpu(p: synthetic.Problem, dy, w, mode="auto", out=None):
     import convolution_backward_b200 as cb
     if p.kind == "pointwise":
         return cb.pointwise(dy, w, out=out)
+    if p.kind == "dense":
+        return cb.dense(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
     return cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, mode=mode,
                         out=out)
 
 
+def _oracle_kind(p: synthetic.Problem, w: np.ndarray):
+    """The oracle's kind and filter for p: a dense W [KH][KW][K][C] goes in as the grouped layout
+    (K, KH, KW, C) with one group (the same values, reordered)."""
+    if p.kind == "dense":
+        return dict(kind="grouped", groups=1, C=p.C), np.ascontiguousarray(np.asarray(w).transpose(2, 0, 1, 3))
+    return dict(kind=p.kind), w
+
+
 def oracle_full(p: synthetic.Problem, dy: np.ndarray, w: np.ndarray) -> np.ndarray:
-    return oracle.dgrad(dy, w, kind=p.kind, H=p.H, W=p.W, KH=p.KH, KW=p.KW, S=p.stride, ph=p.pad_h,
-                        pw=p.pad_w)
+    kw, w = _oracle_kind(p, w)
+    return oracle.dgrad(dy, w, H=p.H, W=p.W, KH=p.KH, KW=p.KW, S=p.stride, ph=p.pad_h, pw=p.pad_w, **kw)
 
 
 def oracle_points(p: synthetic.Problem, dy: np.ndarray, w: np.ndarray, pts) -> np.ndarray:
-    return oracle.dgrad_points(dy, w, pts, kind=p.kind, H=p.H, W=p.W, KH=p.KH, KW=p.KW, S=p.stride,
-                               ph=p.pad_h, pw=p.pad_w)
+    kw, w = _oracle_kind(p, w)
+    return oracle.dgrad_points(dy, w, pts, H=p.H, W=p.W, KH=p.KH, KW=p.KW, S=p.stride, ph=p.pad_h,
+                               pw=p.pad_w, **kw)
 
 
 def terms_per_output(p: synthetic.Problem) -> int:
-    return p.K if p.kind == "pointwise" else p.KH * p.KW
+    if p.kind == "pointwise":
+        return p.K
+    if p.kind == "dense":
+        return p.K * p.KH * p.KW
+    return p.KH * p.KW
 
 
 def check(p: synthetic.Problem, got: np.ndarray, ref: np.ndarray, absref: np.ndarray, what: str = ""):

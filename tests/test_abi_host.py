@@ -207,3 +207,16 @@ def test_depthwise_tc_validation_and_workspace_size():
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p31), ctypes.byref(nb)) == OK
     assert call(p31, ws_bytes=nb.value - 256) == INVALID
     assert L.dgrad_depthwise_tc(ctypes.byref(empty), BF16, 0, 0, 0, 0, 0, None) == OK
+
+
+def test_dense_validation():
+    L = cb.lib()
+    p = cb.Problem(1, 8, 8, 16, 16, 3, 3, 1, 1, 1)
+    call = lambda prob, dtype=BF16, ptrs=(FAKE, FAKE, FAKE): L.dgrad_dense(ctypes.byref(prob), dtype, *ptrs, None)
+    assert call(p, dtype=F32) == UNSUPPORTED
+    assert call(p, dtype=7) == INVALID
+    assert call(cb.Problem(1, 8, 8, 16, 20, 3, 3, 1, 1, 1)) == ALIGNMENT      # K*2 = 40 bytes
+    assert call(p, ptrs=(FAKE, FAKE + 4, FAKE)) == ALIGNMENT
+    assert call(p, ptrs=(0, FAKE, FAKE)) == INVALID
+    assert call(cb.Problem(1, 80, 80, 16, 16, 65, 3, 1, 1, 1)) == UNSUPPORTED   # filter over 64
+    assert call(cb.Problem(0, 8, 8, 16, 16, 3, 3, 1, 1, 1), ptrs=(0, 0, 0)) == OK

@@ -316,6 +316,66 @@ def test_depthwise_tensor_core_cuda_transposes(p, monkeypatch):
     cb.check_status()
 
 
+DENSE = [
+    P("dense3x3_s1", "dense", "bf16", 2, 13, 21, 72, 40, 3, 3, 1, 1, 1, seed=171),
+    P("dense1x1_s1", "dense", "bf16", 1, 9, 11, 64, 128, 1, 1, 1, 0, 0, seed=172),
+    P("dense5x3_s1_nonsame", "dense", "bf16", 3, 17, 10, 136, 24, 5, 3, 1, 1, 2, seed=173),
+    P("dense7x7_s1", "dense", "bf16", 1, 20, 19, 64, 64, 7, 7, 1, 3, 3, seed=174),
+    P("dense3x3_s2", "dense", "bf16", 2, 15, 17, 48, 80, 3, 3, 2, 1, 1, seed=175),
+    P("dense4x4_s2_even", "dense", "bf16", 1, 16, 18, 32, 16, 4, 4, 2, 1, 1, seed=176),
+    P("dense1x1_s2", "dense", "bf16", 2, 14, 15, 40, 56, 1, 1, 2, 0, 0, seed=177),
+    P("dense7x7_s2", "dense", "bf16", 1, 23, 22, 24, 32, 7, 7, 2, 3, 3, seed=178),
+    P("dense5x5_s3", "dense", "bf16", 2, 19, 20, 16, 24, 5, 5, 3, 2, 2, seed=179),
+    P("dense2x3_s2_gaps", "dense", "bf16", 1, 13, 14, 8, 8, 2, 3, 3, 0, 1, seed=180),
+    P("dense3x3_k200_c264", "dense", "bf16", 1, 9, 9, 264, 200, 3, 3, 1, 1, 1, seed=181),
+]
+
+
+@pytest.mark.parametrize("bn", ["64", "128", "256"])
+@pytest.mark.parametrize("p", DENSE, ids=[p.name for p in DENSE])
+def test_dense_tensor_core(p, bn, monkeypatch):
+    """Dense (ungrouped) KxK dgrad on tcgen05 by output phase (§8 NEXT-1), every channel tile width,
+    against the oracle on whole outputs: strides 1-3, odd and even filters, padding that is not
+    'same', ragged K, C, extents and tile edges."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_DENSE_BN", bn)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/bn={bn}")
+    cb.check_status()
+
+
+DENSE_LARGE = [P("dense3x3_s1_large", "dense", "bf16", 8, 28, 28, 256, 256, 3, 3, 1, 1, 1, seed=182),
+               P("dense3x3_s2_large", "dense", "bf16", 8, 56, 56, 128, 256, 3, 3, 2, 1, 1, seed=183)]
+
+
+@pytest.mark.parametrize("p", DENSE_LARGE, ids=[p.name for p in DENSE_LARGE])
+def test_dense_tensor_core_sampled(p):
+    """Larger dense problems (many tiles and k-blocks): sampled oracle points and every element against
+    cuDNN in fp32."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = h.run_gpu(p, dy, w)
+    torch.cuda.synchronize()
+    pts = h.sample_points(p, 2000)
+    got = out.float()[pts[:, 0], pts[:, 1], pts[:, 2], pts[:, 3]].cpu().numpy().astype(np.float64)
+    ref = h.oracle_points(p, inp.dy, inp.w, pts)
+    absref = h.oracle_points(p, np.abs(inp.dy), np.abs(inp.w), pts)
+    h.check(p, got, ref, absref, what=f"{p.name} sampled")
+    wt = w.float().permute(2, 3, 0, 1).contiguous()      # (K, C, KH, KW): the forward weight
+    tref = torch.nn.grad.conv2d_input((p.N, p.C, p.H, p.W), wt, dy.float().permute(0, 3, 1, 2).contiguous(),
+                                      stride=p.stride, padding=(p.pad_h, p.pad_w)).permute(0, 2, 3, 1)
+    err = (out.float() - tref).abs().max().item()
+    assert err / (tref.abs().max().item() + 1e-6) <= 1e-2
+    cb.check_status()
+
+
 TC_TILES = ["0,2,32,1", "0,2,16,1", "0,4,16,2", "0,4,8,2", "0,8,8,4", "0,8,4,4", "1,4,16,2", "1,8,8,4"]
 
 
