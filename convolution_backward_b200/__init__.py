@@ -19,7 +19,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwise_tc", "depthwise_tc_workspace_bytes", "dense", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
+__all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwise_tc", "depthwise_tc_workspace_bytes", "dense", "grouped", "splitk_workspace_bytes", "depthwise", "out_dims", "check_status", "DgradError", "DgradUnavailable",
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -30,7 +30,7 @@ _lib = None
 STATUS = {0: "DGRAD_OK", 1: "DGRAD_ERR_INVALID", 2: "DGRAD_ERR_UNSUPPORTED", 3: "DGRAD_ERR_ALIGNMENT",
           4: "DGRAD_ERR_CUDA", 5: "DGRAD_ERR_TIMEOUT"}
 DW_MODES = {"auto": 0, "rotated": 1, "rowstream": 2}
-DTYPES = {"f32": 0, "bf16": 1}
+DTYPES = {"f32": 0, "bf16": 1, "f16": 2}
 SPLITK_SCRATCH_BYTES = 8 << 20   # DGRAD_SPLITK_SCRATCH_BYTES: the fixed per-device split-K buffer
 
 
@@ -101,6 +101,8 @@ def lib():
             L.dgrad_pointwise_splitk_noalloc.restype = ctypes.c_int
             L.dgrad_dense.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp]
             L.dgrad_dense.restype = ctypes.c_int
+            L.dgrad_grouped.argtypes = [P(Problem), ctypes.c_int64, ctypes.c_int, vp, vp, vp, vp]
+            L.dgrad_grouped.restype = ctypes.c_int
             L.dgrad_depthwise_tc.argtypes = [P(Problem), ctypes.c_int, vp, vp, vp, vp, ctypes.c_size_t, vp]
             L.dgrad_depthwise_tc.restype = ctypes.c_int
             L.dgrad_depthwise_tc_workspace.argtypes = [P(Problem), P(ctypes.c_size_t)]
@@ -127,7 +129,9 @@ def _dtype_code(t) -> int:
         return 0
     if t.dtype == torch.bfloat16:
         return 1
-    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    if t.dtype == torch.float16:
+        return 2
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32, bfloat16 or float16")
 
 
 def _need_cuda(*ts):
@@ -287,6 +291,37 @@ def dense(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=None, stream
     prob = Problem(N, H, W_out, C, K, KH, KW, stride, pad_h, pad_w)
     _check(lib().dgrad_dense(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(), out.data_ptr(),
                              _stream_ptr(stream)), "dgrad_dense")
+    return out
+
+
+def grouped(dY, W, groups, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=None, stream=None, **kw):
+    """Grouped dgrad on the tensor cores (bf16 or f16; dgrad_grouped): dY (N,Ho,Wo,K),
+    W (KH,KW,K,C/groups) -> dX (N,H,W,C).  A 1x1 filter is grouped pointwise dgrad."""
+    import torch
+    if W_out is None:
+        W_out = kw.pop("Wd")
+    if kw:
+        raise TypeError(f"unexpected arguments {sorted(kw)}")
+    _need_cuda(dY, W)
+    if dY.dim() != 4 or W.dim() != 4 or W.shape[2] != dY.shape[3]:
+        raise ValueError("expected dY (N,Ho,Wo,K) and W (KH,KW,K,C/groups)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
+    N, Ho, Wo, K = dY.shape
+    KH, KW, _, Cg = W.shape
+    C = Cg * int(groups)
+    eho, ewo = out_dims(H, W_out, KH, KW, stride, pad_h, pad_w)
+    if (eho, ewo) != (Ho, Wo):
+        raise ValueError(f"dY spatial extent {(Ho, Wo)} does not match the geometry ({eho}, {ewo})")
+    if out is None:
+        out = torch.empty((N, H, W_out, C), dtype=dY.dtype, device=dY.device)
+    else:
+        _need_cuda(out)
+        if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
+            raise ValueError("out has the wrong shape or dtype")
+    prob = Problem(N, H, W_out, C, K, KH, KW, stride, pad_h, pad_w)
+    _check(lib().dgrad_grouped(ctypes.byref(prob), int(groups), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
+                               out.data_ptr(), _stream_ptr(stream)), "dgrad_grouped")
     return out
 
 

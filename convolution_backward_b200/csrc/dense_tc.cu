@@ -1,7 +1,11 @@
-// dense_tc.cu -- dense (ungrouped) KH x KW dgrad on the Blackwell tensor cores.
+// dense_tc.cu -- dense and grouped KH x KW dgrad on the Blackwell tensor cores.
 //
 // dX[n,h,w,c] = sum over (ho,wo,k,r,s) with h = ho*S - pad_h + r, w = wo*S -
-// pad_w + s of dY[n,ho,wo,k] * W[r][s][k][c].  Split by output phase (the
+// pad_w + s and k in c's group of dY[n,ho,wo,k] * W[r][s][k][c - group base]
+// (G groups of Kg dY and Cg dX channels; W is [KH][KW][K][Cg], G = 1 dense).
+// Each group is its own GEMM: dY is seen as a 5-D tensor (Kg, G, Wo, Ho, N) and
+// W as (Cg, Kg, G, KH*KW), so the zero fill of the TMA boxes stops every k-block
+// and channel tile at its group's edge.  Split by output phase (the
 // pages' sub-pixel decomposition of strided dgrad into S*S sub-GEMMs, "add the
 // pointwise fast path dgrad was missing", Technical Details): for a = (h +
 // pad_h) mod S and b = (w + pad_w) mod S, the rows h = S*hq + a - pad_h and
@@ -13,7 +17,9 @@
 // the single phase (0, 0).  No im2col buffer, no gather.
 //
 // Tile: 128 positions = 8 rows hq x 16 columns wq of one phase of one image
-// (M), BN channels c (N); K-loop over the phase's taps x 64-deep k-blocks.
+// (M), BN channels of one group (N); K-loop over the phase's taps x 64-deep
+// k-blocks of the group.  bf16 or f16 operands (same type for A and B), fp32
+// accumulation, output in the input type.
 // Kernel structure as the streaming pointwise kernel (persistent, one CTA per
 // SM, 192 threads): warp 0 TMA producer (A box 64 k x 16 wq x 8 hq, W box BN c x
 // 64 k, 128-byte swizzle), warp 1 TMEM allocation and MMA issue (M = 128, N =
@@ -45,9 +51,9 @@ struct DenseLayout {
     static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
-// One tile: image n, phase (a, b), first hq / wq, first channel.
+// One tile: image n, phase (a, b), first hq / wq, group g, first channel of the group.
 struct DTile {
-    int n, a, b, hq0, wq0, c0, nt, nu;
+    int n, a, b, hq0, wq0, g, c0, nt, nu;
 };
 
 __device__ __forceinline__ DTile decode_tile(const DenseArgs& d, int t, int bn)
@@ -55,6 +61,8 @@ __device__ __forceinline__ DTile decode_tile(const DenseArgs& d, int t, int bn)
     DTile r;
     const int ct = t % d.nc;
     int q = t / d.nc;
+    r.g = q % d.G;
+    q /= d.G;
     const int wt = q % d.ntw;
     q /= d.ntw;
     const int ht = q % d.nth;
@@ -71,7 +79,7 @@ __device__ __forceinline__ DTile decode_tile(const DenseArgs& d, int t, int bn)
     return r;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     dense_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ DenseArgs d)
@@ -92,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_kb = (d.K + kBK - 1) / kBK;
+    const int num_kb = (d.Kg + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -140,12 +148,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
                             uint8_t* a_tile = smem + stage * L::kStageBytes;
                             uint8_t* b_tile = a_tile + L::kABytes;
-                            // A: dY[n, hq0 - t .. +8, wq0 - u .. +16, kb*64 .. +64] (zero outside)
-                            tma_load_4d(a_tile, &map_a, &full[stage], kb * kBK, tl.wq0 - ui, tl.hq0 - ti, tl.n);
-                            // B: W[tap][kb*64 .. +64][c0 .. c0 + BN] (zero outside)
+                            // A: dY[n, hq0 - t .. +8, wq0 - u .. +16, group g, kb*64 .. +64] (zero outside)
+                            tma_load_5d(a_tile, &map_a, &full[stage], kb * kBK, tl.g, tl.wq0 - ui, tl.hq0 - ti,
+                                        tl.n);
+                            // B: W[tap][group g][kb*64 .. +64][c0 .. c0 + BN] (zero outside)
 #pragma unroll
                             for (int j = 0; j < BN / 64; ++j)
-                                tma_load_3d(b_tile + j * 8192, &map_b, &full[stage], tl.c0 + j * 64, kb * kBK, tap);
+                                tma_load_4d(b_tile + j * 8192, &map_b, &full[stage], tl.c0 + j * 64, kb * kBK, tl.g,
+                                            tap);
                             ++issued;
                             if (++stage == STAGES) {
                                 stage = 0;
@@ -171,7 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // --------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+            constexpr uint32_t idesc =
+                F16 ? idesc_f16_f32(kBM, BN, /*b_mn_major=*/true) : idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -239,8 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h = d.S * (tl.hq0 + row / kTW) + tl.a - d.ph;
             const int w = d.S * (tl.wq0 + row % kTW) + tl.b - d.pw;
             const bool pos_ok = h >= 0 && h < d.H && w >= 0 && w < d.W;
-            __nv_bfloat16* out_row =
-                d.dX + ((static_cast<int64_t>(tl.n) * d.H + (pos_ok ? h : 0)) * d.W + (pos_ok ? w : 0)) * d.C;
+            uint16_t* out_row = reinterpret_cast<uint16_t*>(d.dX) +
+                                ((static_cast<int64_t>(tl.n) * d.H + (pos_ok ? h : 0)) * d.W + (pos_ok ? w : 0)) * d.C +
+                                static_cast<int64_t>(tl.g) * d.Cg;
             // A phase with no taps (filter extent below the stride) receives nothing: its
             // positions are written as zeros and the accumulator is not read.
             const bool no_taps = tl.nt == 0 || tl.nu == 0;
@@ -259,12 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         const int col = col0 + g * 8;
-                        if (col < d.C) {
+                        if (col < d.Cg) {
+                            auto cvt = [](uint32_t lo, uint32_t hi) {
+                                return F16 ? float2_to_f16x2(__uint_as_float(lo), __uint_as_float(hi))
+                                           : float2_to_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
+                            };
                             uint4 o;
-                            o.x = float2_to_bf16x2(__uint_as_float(v[g * 8 + 0]), __uint_as_float(v[g * 8 + 1]));
-                            o.y = float2_to_bf16x2(__uint_as_float(v[g * 8 + 2]), __uint_as_float(v[g * 8 + 3]));
-                            o.z = float2_to_bf16x2(__uint_as_float(v[g * 8 + 4]), __uint_as_float(v[g * 8 + 5]));
-                            o.w = float2_to_bf16x2(__uint_as_float(v[g * 8 + 6]), __uint_as_float(v[g * 8 + 7]));
+                            o.x = cvt(v[g * 8 + 0], v[g * 8 + 1]);
+                            o.y = cvt(v[g * 8 + 2], v[g * 8 + 3]);
+                            o.z = cvt(v[g * 8 + 4], v[g * 8 + 5]);
+                            o.w = cvt(v[g * 8 + 6], v[g * 8 + 7]);
                             *reinterpret_cast<uint4*>(out_row + col) = o;
                         }
                     }
@@ -295,11 +311,11 @@ cudaError_t launch_dense_bn(DenseArgs d, const CUtensorMap& map_a, const CUtenso
                             cudaStream_t stream)
 {
     using L = DenseLayout<BN, STAGES>;
-    auto kern = dense_tc_kernel<BN, STAGES>;
+    auto kern = d.f16 ? dense_tc_kernel<BN, STAGES, true> : dense_tc_kernel<BN, STAGES, false>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::kAlloc);
     if (e != cudaSuccess) return e;
-    d.nc = (d.C + BN - 1) / BN;
-    const long long tiles = static_cast<long long>(d.N) * d.S * d.S * d.nth * d.ntw * d.nc;
+    d.nc = (d.Cg + BN - 1) / BN;
+    const long long tiles = static_cast<long long>(d.N) * d.S * d.S * d.nth * d.ntw * d.G * d.nc;
     if (tiles > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     d.num_tiles = static_cast<int>(tiles);
     if (d.num_tiles == 0) return cudaSuccess;

@@ -169,7 +169,7 @@ dgrad_status_t validate_common(const dgrad_problem_t* p, dgrad_dtype_t dtype, in
                                int* pad_w)
 {
     if (!p) return DGRAD_ERR_INVALID;
-    if (dtype != DGRAD_F32 && dtype != DGRAD_BF16) return DGRAD_ERR_INVALID;
+    if (dtype != DGRAD_F32 && dtype != DGRAD_BF16 && dtype != DGRAD_F16) return DGRAD_ERR_INVALID;
     if (p->N < 0 || p->H < 1 || p->W < 1 || p->C < 1 || p->K < 1) return DGRAD_ERR_INVALID;
     if (p->KH < 1 || p->KW < 1 || p->stride < 1) return DGRAD_ERR_INVALID;
     if (p->pad_h < 0 || p->pad_w < -1) return DGRAD_ERR_INVALID;
@@ -211,6 +211,7 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     if (s != DGRAD_OK) return s;
     if (prob->KH != 1 || prob->KW != 1 || prob->stride != 1 || prob->pad_h != 0 || pw != 0)
         return DGRAD_ERR_UNSUPPORTED;
+    if (dtype == DGRAD_F16) return dgrad_grouped(prob, 1, dtype, dY, W, dX, stream);   // 1x1 through the tap kernel
     const int64_t M = prob->N * prob->H * prob->W;
     if (M == 0) return DGRAD_OK;
     if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
@@ -326,26 +327,29 @@ dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 
-dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W, void* dX,
-                           void* stream)
+dgrad_status_t dgrad_grouped(const dgrad_problem_t* prob, int64_t groups, dgrad_dtype_t dtype, const void* dY,
+                             const void* W, void* dX, void* stream)
 {
     int64_t Ho = 0, Wo = 0;
     int pw = 0;
     dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
     if (s != DGRAD_OK) return s;
-    if (dtype != DGRAD_BF16) return DGRAD_ERR_UNSUPPORTED;
+    if (groups < 1 || prob->K % groups || prob->C % groups) return DGRAD_ERR_INVALID;
+    if (dtype == DGRAD_F32) return DGRAD_ERR_UNSUPPORTED;
     if (prob->KH > 64 || prob->KW > 64 || prob->stride > 64) return DGRAD_ERR_UNSUPPORTED;
     if (prob->K > 65536 || prob->C > 65536 || prob->H > (1 << 24) || prob->W > (1 << 24) || prob->N > (1 << 24))
         return DGRAD_ERR_UNSUPPORTED;
+    const int64_t Kg = prob->K / groups;
+    const int64_t Cg = prob->C / groups;
     if (prob->N == 0) return DGRAD_OK;
     if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
-    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (prob->K * 2) % 16 || (prob->C * 2) % 16)
+    if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (Kg * 2) % 16 || (Cg * 2) % 16)
         return DGRAD_ERR_ALIGNMENT;
     DeviceState* st = nullptr;
     s = device_state(&st);
     if (s != DGRAD_OK) return s;
     dgrad::DenseArgs d{};
-    d.dX = static_cast<__nv_bfloat16*>(dX);
+    d.dX = dX;
     d.status = st->status;
     d.N = static_cast<int>(prob->N);
     d.H = static_cast<int>(prob->H);
@@ -359,35 +363,51 @@ dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, con
     d.S = prob->stride;
     d.ph = prob->pad_h;
     d.pw = pw;
+    d.G = static_cast<int>(groups);
+    d.Kg = static_cast<int>(Kg);
+    d.Cg = static_cast<int>(Cg);
+    d.f16 = dtype == DGRAD_F16;
     dgrad::plan_dense(&d);
     auto enc = tensor_map_encoder();
     if (!enc) return cuda_fail(cudaErrorInvalidValue);
+    const CUtensorMapDataType ty = d.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap map_a, map_b;
     {
-        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(prob->K), static_cast<cuuint64_t>(Wo),
-                                    static_cast<cuuint64_t>(Ho), static_cast<cuuint64_t>(prob->N)};
-        const cuuint64_t strides[3] = {dims[0] * 2, dims[1] * dims[0] * 2, dims[2] * dims[1] * dims[0] * 2};
-        const cuuint32_t box[4] = {64, 16, 8, 1};
-        const cuuint32_t estr[4] = {1, 1, 1, 1};
-        if (enc(&map_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(dY), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        // dY as (Kg, G, Wo, Ho, N)
+        const cuuint64_t dims[5] = {static_cast<cuuint64_t>(Kg), static_cast<cuuint64_t>(groups),
+                                    static_cast<cuuint64_t>(Wo), static_cast<cuuint64_t>(Ho),
+                                    static_cast<cuuint64_t>(prob->N)};
+        const cuuint64_t kb = static_cast<cuuint64_t>(prob->K) * 2;
+        const cuuint64_t strides[4] = {static_cast<cuuint64_t>(Kg) * 2, kb, kb * dims[2], kb * dims[2] * dims[3]};
+        const cuuint32_t box[5] = {64, 1, 16, 8, 1};
+        const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+        if (enc(&map_a, ty, 5, const_cast<void*>(dY), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cuda_fail(cudaErrorInvalidValue);
     }
     {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(prob->C), static_cast<cuuint64_t>(prob->K),
+        // W [KH][KW][K][Cg] as (Cg, Kg, G, KH*KW)
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(Cg), static_cast<cuuint64_t>(Kg),
+                                    static_cast<cuuint64_t>(groups),
                                     static_cast<cuuint64_t>(prob->KH) * static_cast<cuuint64_t>(prob->KW)};
-        const cuuint64_t strides[2] = {dims[0] * 2, dims[1] * dims[0] * 2};
-        const cuuint32_t box[3] = {64, 64, 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (enc(&map_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(W), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        const cuuint64_t strides[3] = {dims[0] * 2, dims[0] * dims[1] * 2, dims[0] * dims[1] * dims[2] * 2};
+        const cuuint32_t box[4] = {64, 64, 1, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (enc(&map_b, ty, 4, const_cast<void*>(W), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cuda_fail(cudaErrorInvalidValue);
     }
-    const int bn = env_int("DGRAD_DENSE_BN", prob->C <= 64 ? 64 : 128);
+    const int bn = env_int("DGRAD_DENSE_BN", Cg <= 64 ? 64 : 128);
     cudaError_t e = dgrad::launch_dense_tc(d, map_a, map_b, bn, st->sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+}
+
+dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W, void* dX,
+                           void* stream)
+{
+    return dgrad_grouped(prob, 1, dtype, dY, W, dX, stream);
 }
 
 // Shared checks for the tensor-core depthwise entry points: stride-1 depthwise,
@@ -481,6 +501,7 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
     if (s != DGRAD_OK) return s;
     if (mode != DGRAD_DW_AUTO && mode != DGRAD_DW_ROTATED && mode != DGRAD_DW_ROWSTREAM) return DGRAD_ERR_INVALID;
+    if (dtype == DGRAD_F16) return DGRAD_ERR_UNSUPPORTED;
     if (prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
     if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
     if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;

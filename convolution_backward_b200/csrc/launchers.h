@@ -51,16 +51,19 @@ size_t pointwise_splitk_workspace_bytes(const PwArgs& a, int splits);
 cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a, const CUtensorMap& map_b,
                                        int splits, float* ws, int num_sms, cudaStream_t stream);
 
-// Dense (ungrouped) KH x KW dgrad on tcgen05, by output phase (S*S sub-GEMMs),
-// bf16.  W is [KH][KW][K][C].  map_a covers dY as a 4-D bf16 tensor (K, Wo, Ho,
-// N) with a 64 x 16 x 8 x 1 box and the 128-byte swizzle; map_b covers W as a
-// 3-D bf16 tensor (C, K, KH*KW) with a 64 x 64 x 1 box and the 128-byte swizzle.
+// Dense or grouped KH x KW dgrad on tcgen05, by output phase (S*S sub-GEMMs),
+// bf16 or f16 (f16 = true).  G groups of Kg dY and Cg dX channels; W is
+// [KH][KW][K][Cg].  map_a covers dY as a 5-D tensor (Kg, G, Wo, Ho, N) with a
+// 64 x 1 x 16 x 8 x 1 box and the 128-byte swizzle; map_b covers W as a 4-D
+// tensor (Cg, Kg, G, KH*KW) with a 64 x 64 x 1 x 1 box and the 128-byte swizzle.
 // plan_dense fills the phase-grid fields (hq_min, wq_min, nth, ntw) from the
 // geometry; bn is the channel tile (64, 128 or 256).
 struct DenseArgs {
-    __nv_bfloat16* dX;
+    void* dX;
     int* status;
     int N, H, W, C, K, Ho, Wo, KH, KW, S, ph, pw;
+    int G, Kg, Cg;
+    bool f16;
     int hq_min, wq_min, nth, ntw, nc, num_tiles;
 };
 void plan_dense(DenseArgs* d);

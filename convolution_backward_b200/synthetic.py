@@ -11,7 +11,8 @@ Recipe (one per workload, in this order):
   2. dY: draw in float64 in logical NHWC order and shape (N, Ho, Wo, K)
   3. W : draw in float64 in its storage layout ((K, C) pointwise, (KH, KW, C) depthwise,
      (KH, KW, K, C) dense)
-  4. cast to float32; for bf16 workloads round to bf16 with round-to-nearest-even.
+  4. cast to float32; for bf16 workloads round to bf16, for f16 ones to IEEE half,
+     both with round-to-nearest-even.
 Distributions: "normal" is N(0, var) with ``var`` the variance (std = sqrt(var));
 "uniform" is U[-1, 1].  A workload with several problems (the non-square and
 strided depthwise set) draws each problem from a fresh generator with the same
@@ -28,8 +29,8 @@ import numpy as np
 @dataclass(frozen=True)
 class Problem:
     name: str
-    kind: str            # "pointwise" | "depthwise" | "dense"
-    dtype: str           # "f32" | "bf16"
+    kind: str            # "pointwise" | "depthwise" | "dense" | "grouped"
+    dtype: str           # "f32" | "bf16" | "f16"
     N: int
     H: int
     W: int
@@ -46,6 +47,7 @@ class Problem:
     w_dist: str = "normal"
     w_var: float = 1.0
     variant: str = ""    # "splitk": split-K pointwise entry point; "tc": tensor-core depthwise entry point
+    ngroups: int = 1     # groups of a "grouped" problem (K and C multiples of it)
 
     @property
     def Ho(self) -> int:
@@ -57,7 +59,9 @@ class Problem:
 
     @property
     def groups(self) -> int:
-        return self.C if self.kind == "depthwise" else 1
+        if self.kind == "depthwise":
+            return self.C
+        return self.ngroups if self.kind == "grouped" else 1
 
     @property
     def dy_shape(self):
@@ -69,6 +73,8 @@ class Problem:
             return (self.K, self.C)
         if self.kind == "dense":
             return (self.KH, self.KW, self.K, self.C)
+        if self.kind == "grouped":
+            return (self.KH, self.KW, self.K, self.C // self.ngroups)
         return (self.KH, self.KW, self.C)
 
     @property
@@ -179,8 +185,9 @@ def _draw(rng: np.random.Generator, shape, dist: str, var: float) -> np.ndarray:
 @dataclass
 class Inputs:
     """One problem's inputs.  ``dy``/``w`` are float32 arrays holding exactly the
-    values the kernels see (bf16-representable for bf16 problems); ``dy_bits`` /
-    ``w_bits`` are the bf16 bit patterns (uint16) for bf16 problems, else None."""
+    values the kernels see (bf16- or f16-representable for 16-bit problems);
+    ``dy_bits`` / ``w_bits`` are the 16-bit patterns (uint16) for 16-bit
+    problems, else None."""
     problem: Problem
     dy: np.ndarray
     w: np.ndarray
@@ -198,6 +205,10 @@ def make_inputs(p: Problem, seed: int | None = None) -> Inputs:
     w32 = w64.astype(np.float32)
     if p.dtype == "f32":
         return Inputs(p, dy32, w32)
+    if p.dtype == "f16":
+        dyh = dy32.astype(np.float16)
+        wh = w32.astype(np.float16)
+        return Inputs(p, dyh.astype(np.float32), wh.astype(np.float32), dyh.view(np.uint16), wh.view(np.uint16))
     dyb = f32_to_bf16_bits(dy32)
     wb = f32_to_bf16_bits(w32)
     return Inputs(p, bf16_bits_to_f32(dyb), bf16_bits_to_f32(wb), dyb, wb)

@@ -64,7 +64,10 @@ typedef struct {
     int32_t pad_h, pad_w;
 } dgrad_problem_t;
 
-typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1 } dgrad_dtype_t;
+/* Element type of dY, W and dX (one type for all three).  DGRAD_F16 is served by
+ * dgrad_pointwise, dgrad_dense and dgrad_grouped (tcgen05 f16 operands, fp32
+ * accumulation); other entry points return DGRAD_ERR_UNSUPPORTED for it. */
+typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1, DGRAD_F16 = 2 } dgrad_dtype_t;
 
 /* Depthwise kernel choice.  AUTO: rotated-filter for stride 1, row-streaming
  * otherwise.  ROTATED requires stride 1.  ROWSTREAM serves any stride (at
@@ -84,6 +87,7 @@ typedef enum {
  * Requires KH = KW = 1, stride 1, pad_h = pad_w = 0 (else DGRAD_ERR_UNSUPPORTED;
  * the pointwise page's shape class).  DGRAD_BF16 runs on the tcgen05 tensor
  * cores (TMA-fed shared-memory tiles, fp32 accumulators in tensor memory);
+ * DGRAD_F16 runs on them through the tap kernel of dgrad_grouped (one 1x1 tap);
  * DGRAD_F32 runs as an fp32 FMA kernel (no reduced-precision inputs). */
 dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
                                const void* dY, const void* W, void* dX, void* stream);
@@ -146,13 +150,25 @@ dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int
 dgrad_status_t dgrad_pointwise_splitk_noalloc(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
                                               const void* dY, const void* W, void* dX, void* stream);
 
+/* Grouped dgrad: `groups` groups, each of K/groups dY and C/groups dX channels,
+ * any KH x KW filter and stride, on the tcgen05 tensor cores; W is
+ * [KH][KW][K][C/groups] (tap-major; each tap holds, for every dY channel k, the
+ * C/groups filter values of k's group).  A 1x1 filter is the pages' grouped
+ * pointwise dgrad (per-group output channel base and a C/groups W stride; "add
+ * the pointwise fast path dgrad was missing", Technical Details).  Each group
+ * runs as its own set of phase GEMMs, as in dgrad_dense.  groups must divide K
+ * and C (else DGRAD_ERR_INVALID); K/groups and C/groups multiples of 8 (else
+ * DGRAD_ERR_ALIGNMENT); DGRAD_BF16 or DGRAD_F16; other limits as dgrad_dense. */
+dgrad_status_t dgrad_grouped(const dgrad_problem_t* prob, int64_t groups, dgrad_dtype_t dtype, const void* dY,
+                             const void* W, void* dX, void* stream);
+
 /* Dense (ungrouped, groups = 1) dgrad with a KH x KW filter and any stride, on
  * the tcgen05 tensor cores; W is [KH][KW][K][C] (tap-major: each tap is a
  * pointwise [K][C] matrix).  The pages' main dgrad engine decomposes a strided
  * dgrad by output phase into stride*stride sub-GEMMs ("add the pointwise fast
  * path dgrad was missing", Technical Details); here each phase's GEMM sums, over
  * the phase's taps, products of a shifted window of dY (K deep) with that tap's
- * [K][C] matrix, so no im2col buffer is built.  DGRAD_BF16 only (else
+ * [K][C] matrix, so no im2col buffer is built.  DGRAD_BF16 or DGRAD_F16 (else
  * DGRAD_ERR_UNSUPPORTED); KH, KW, stride <= 64; K and C multiples of 8; padding
  * any value >= 0 that leaves Ho, Wo >= 1. */
 dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, const void* dY, const void* W, void* dX,

@@ -3,13 +3,14 @@ oracle references and the comparison rules.
 
 Tolerances (written out here, used by every parity test):
   normwise, the acceptance bar:
-    bf16 I/O : max|gpu - ref| / (max|ref| + 1e-6) <= 1e-2
+    bf16, f16 I/O : max|gpu - ref| / (max|ref| + 1e-6) <= 1e-2
     f32 I/O  : max|gpu - ref| / max|ref|          <= 1e-5
   elementwise, derived from the arithmetic (fp32 accumulation of n terms in any
   order, then one rounding of the output):
     |gpu - ref| <= u_out*|ref| + (1 + u_out) * n * 2^-24 * sum|terms| + tiny
   with u_out = 2^-8 for a bf16 output (8 significant bits, round to nearest
-  even: half an ulp is 2^-8 relative) and 2^-24 for f32 (24 significant bits),
+  even: half an ulp is 2^-8 relative), 2^-11 for f16 (11 significant bits) and
+  2^-24 for f32 (24 significant bits),
   n the number of products per output and sum|terms| the same dgrad
   evaluated on |dY| and |W| (by the oracle).
 """
@@ -22,15 +23,17 @@ import oracle
 from convolution_backward_b200 import synthetic
 
 U_BF16 = 2.0 ** -8
+U_F16 = 2.0 ** -11
 U_F32 = 2.0 ** -24
 
 
 def to_dev(inp: synthetic.Inputs):
     """Device tensors (dY, W) holding exactly the values in inp."""
     p = inp.problem
-    if p.dtype == "bf16":
-        dy = torch.from_numpy(inp.dy_bits.view(np.int16)).view(torch.bfloat16).cuda()
-        w = torch.from_numpy(inp.w_bits.view(np.int16)).view(torch.bfloat16).cuda()
+    if p.dtype in ("bf16", "f16"):
+        tt = torch.bfloat16 if p.dtype == "bf16" else torch.float16
+        dy = torch.from_numpy(inp.dy_bits.view(np.int16)).view(tt).cuda()
+        w = torch.from_numpy(inp.w_bits.view(np.int16)).view(tt).cuda()
     else:
         dy = torch.from_numpy(inp.dy).cuda()
         w = torch.from_numpy(inp.w).cuda()
@@ -43,6 +46,9 @@ def run_gpu(p: synthetic.Problem, dy, w, mode="auto", out=None):
         return cb.pointwise(dy, w, out=out)
     if p.kind == "dense":
         return cb.dense(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
+    if p.kind == "grouped":
+        return cb.grouped(dy, w, p.ngroups, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w,
+                          out=out)
     return cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, mode=mode,
                         out=out)
 
@@ -50,8 +56,9 @@ def run_gpu(p: synthetic.Problem, dy, w, mode="auto", out=None):
 def _oracle_kind(p: synthetic.Problem, w: np.ndarray):
     """The oracle's kind and filter for p: a dense W [KH][KW][K][C] goes in as the grouped layout
     (K, KH, KW, C) with one group (the same values, reordered)."""
-    if p.kind == "dense":
-        return dict(kind="grouped", groups=1, C=p.C), np.ascontiguousarray(np.asarray(w).transpose(2, 0, 1, 3))
+    if p.kind in ("dense", "grouped"):
+        return (dict(kind="grouped", groups=p.groups, C=p.C),
+                np.ascontiguousarray(np.asarray(w).transpose(2, 0, 1, 3)))
     return dict(kind=p.kind), w
 
 
@@ -69,8 +76,8 @@ def oracle_points(p: synthetic.Problem, dy: np.ndarray, w: np.ndarray, pts) -> n
 def terms_per_output(p: synthetic.Problem) -> int:
     if p.kind == "pointwise":
         return p.K
-    if p.kind == "dense":
-        return p.K * p.KH * p.KW
+    if p.kind in ("dense", "grouped"):
+        return (p.K // p.groups) * p.KH * p.KW
     return p.KH * p.KW
 
 
@@ -80,10 +87,10 @@ def check(p: synthetic.Problem, got: np.ndarray, ref: np.ndarray, absref: np.nda
     err = np.abs(got - ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     mx = float(np.max(np.abs(ref))) if ref.size else 0.0
-    if p.dtype == "bf16":
+    if p.dtype in ("bf16", "f16"):
         norm = float(err.max(initial=0.0)) / (mx + 1e-6)
         assert norm <= 1e-2, f"{what}: normwise error {norm:.3e} > 1e-2"
-        u = U_BF16
+        u = U_BF16 if p.dtype == "bf16" else U_F16
     else:
         norm = float(err.max(initial=0.0)) / mx if mx > 0 else float(err.max(initial=0.0))
         assert norm <= 1e-5, f"{what}: normwise error {norm:.3e} > 1e-5"

@@ -220,3 +220,20 @@ def test_dense_validation():
     assert call(p, ptrs=(0, FAKE, FAKE)) == INVALID
     assert call(cb.Problem(1, 80, 80, 16, 16, 65, 3, 1, 1, 1)) == UNSUPPORTED   # filter over 64
     assert call(cb.Problem(0, 8, 8, 16, 16, 3, 3, 1, 1, 1), ptrs=(0, 0, 0)) == OK
+
+
+def test_grouped_validation():
+    L = cb.lib()
+    call = lambda prob, groups, dtype=BF16, ptrs=(FAKE, FAKE, FAKE): L.dgrad_grouped(
+        ctypes.byref(prob), groups, dtype, *ptrs, None)
+    p = cb.Problem(1, 8, 8, 64, 128, 1, 1, 1, 0, 0)
+    assert call(p, 3) == INVALID            # 3 divides neither K nor C
+    assert call(p, 0) == INVALID
+    assert call(p, 4, dtype=F32) == UNSUPPORTED
+    assert call(p, 16) == ALIGNMENT         # C/groups = 4 channels: 8-byte rows
+    assert call(cb.Problem(0, 8, 8, 64, 128, 3, 3, 1, 1, 1), 4, ptrs=(0, 0, 0)) == OK
+    F16 = 2
+    dw = cb.Problem(1, 8, 8, 16, 16, 3, 3, 1, 1, 1)
+    assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE, FAKE, FAKE, None) == UNSUPPORTED
+    pw = cb.Problem(1, 8, 8, 16, 16, 1, 1, 1, 0, 0)
+    assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F16, 0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == UNSUPPORTED

@@ -349,6 +349,52 @@ def test_dense_tensor_core(p, bn, monkeypatch):
     cb.check_status()
 
 
+GROUPED = [
+    # grouped pointwise (1x1): per-group dY columns, W [K][C/groups]
+    P("grouped1x1_g4", "grouped", "bf16", 2, 13, 17, 64, 128, seed=191).replace(ngroups=4),
+    P("grouped1x1_g2_ragged", "grouped", "bf16", 1, 9, 23, 272, 144, seed=192).replace(ngroups=2),
+    P("grouped1x1_g16_small", "grouped", "bf16", 1, 7, 9, 128, 256, seed=193).replace(ngroups=16),
+    P("grouped3x3_g2", "grouped", "bf16", 2, 11, 14, 48, 80, 3, 3, 1, 1, 1, seed=194).replace(ngroups=2),
+    P("grouped3x3_s2_g4", "grouped", "bf16", 1, 15, 16, 64, 32, 3, 3, 2, 1, 1, seed=195).replace(ngroups=4),
+    P("grouped5x5_g8_k8", "grouped", "bf16", 1, 12, 13, 64, 64, 5, 5, 1, 2, 2, seed=196).replace(ngroups=8),
+    # fp16 I/O
+    P("dense3x3_f16", "dense", "f16", 2, 13, 21, 72, 40, 3, 3, 1, 1, 1, seed=197),
+    P("grouped1x1_f16_g4", "grouped", "f16", 1, 11, 13, 128, 64, seed=198).replace(ngroups=4),
+    P("dense3x3_s2_f16", "dense", "f16", 1, 15, 17, 48, 80, 3, 3, 2, 1, 1, seed=199),
+]
+
+
+@pytest.mark.parametrize("p", GROUPED, ids=[p.name for p in GROUPED])
+def test_grouped_and_f16_tensor_core(p):
+    """Grouped dgrad (1x1 = the grouped pointwise fast path) and fp16 I/O through the tap kernel (§8 NEXT-3),
+    against the oracle on whole outputs."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=p.name)
+    cb.check_status()
+
+
+@pytest.mark.parametrize("shape", [(2, 13, 23, 264, 200), (1, 9, 11, 64, 512), (3, 7, 5, 8, 8)])
+def test_pointwise_f16(shape):
+    """dgrad_pointwise with fp16 I/O (routed to the tap kernel with one 1x1 tap)."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    N, H, W, C, K = shape
+    p = P("pw_f16", "pointwise", "f16", N, H, W, C, K, seed=61)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(cb.pointwise(dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"pointwise f16 {shape}")
+    cb.check_status()
+
+
 DENSE_LARGE = [P("dense3x3_s1_large", "dense", "bf16", 8, 28, 28, 256, 256, 3, 3, 1, 1, 1, seed=182),
                P("dense3x3_s2_large", "dense", "bf16", 8, 56, 56, 128, 256, 3, 3, 2, 1, 1, seed=183)]
 
