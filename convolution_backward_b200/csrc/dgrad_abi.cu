@@ -420,7 +420,8 @@ static dgrad_status_t toeplitz_prepare(const dgrad_problem_t* prob, dgrad_dtype_
     int pw = 0;
     dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
     if (s != DGRAD_OK) return s;
-    if (dtype != DGRAD_BF16 || prob->stride != 1 || prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
+    if ((dtype != DGRAD_BF16 && dtype != DGRAD_F16) || prob->stride != 1 || prob->K != prob->C)
+        return DGRAD_ERR_UNSUPPORTED;
     if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
     if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;
     if ((prob->C * 2) % 16) return DGRAD_ERR_ALIGNMENT;
@@ -437,7 +438,8 @@ static dgrad_status_t toeplitz_prepare(const dgrad_problem_t* prob, dgrad_dtype_
     a->S = 1;
     a->ph = prob->pad_h;
     a->pw = pw;
-    a->bf16 = true;
+    a->bf16 = dtype == DGRAD_BF16;
+    a->f16 = dtype == DGRAD_F16;
     if (!dgrad::plan_dw_toeplitz(*a, plan)) return DGRAD_ERR_UNSUPPORTED;
     return DGRAD_OK;
 }

@@ -33,7 +33,9 @@
 // row-group stride is two atoms: one TMA load of the planar input per 64
 // columns serves every shift.  A_i is a 128 x K bf16 tile written by four warps
 // straight into tensor memory (up to four buffers), so the MMA reads only B
-// from shared memory.  The A builders read the channel's filter lines, padded
+// from shared memory.  bf16 or f16 operands: the transposes, the filter packing
+// and the TMA copies move 16-bit patterns, only the MMA's operand format and the
+// output rounding depend on the type.  The A builders read the channel's filter lines, padded
 // with zeros and packed two taps per word, from shared memory; the producer
 // brings them in with one bulk copy whenever the channel changes.
 //
@@ -81,6 +83,7 @@ struct ToepArgs {
     int P, TW, XT, NH, Ks, NR, NI, half_l, NB;
     int num_xt, num_yt, num_g, num_units;
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
+    int f16;                     // operands and output are f16 (else bf16)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
 };
 
@@ -178,7 +181,8 @@ template <int KQ, int XT>
 __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
 {
     const int ncol_sub = 8 * a.NH;
-    const uint32_t idesc = idesc_bf16_f32(128, ncol_sub, /*b_mn_major=*/false);
+    const uint32_t idesc =
+        a.f16 ? idesc_f16_f32(128, ncol_sub, /*b_mn_major=*/false) : idesc_bf16_f32(128, ncol_sub, false);
     const uint32_t sbo = static_cast<uint32_t>(a.P) * 1024u;
     const uint32_t pb16 = a.panel_bytes >> 4;
     uint32_t d_tmem[4];
@@ -450,7 +454,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
-                        pk[cc * 16 + k] = float2_to_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                        pk[cc * 16 + k] = a.f16 ? float2_to_f16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]))
+                                                : float2_to_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
                 }
             }
             tc_fence_before();
@@ -754,7 +759,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
 {
-    if (!a.bf16 || a.S != 1) return false;
+    if (!(a.bf16 || a.f16) || a.S != 1) return false;
     // Tile shapes (P row phases, NH row groups, XT sub-tiles of 128/P columns), in the
     // order measured fastest on B200: N = 256 tiles (two row phases) first.  Smaller
     // tiles issue more MMAs per output at a lower rate per MMA, so they serve only
@@ -925,6 +930,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.a_col0 = p.a_col0;
         t.a_cols = p.a_cols;
         t.na = p.na;
+        t.f16 = a.f16 ? 1 : 0;
         t.panel_bytes = p.panel_bytes;
         t.b_bytes = p.b_bytes;
         t.npanels = static_cast<uint32_t>(p.npanels);

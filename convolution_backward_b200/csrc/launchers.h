@@ -78,6 +78,7 @@ void record_cuda_error(cudaError_t e);
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;
     bool bf16;  // element type of dY, W and dX: bf16 (true) or f32 (false)
+    bool f16;   // f16 instead (tensor-core depthwise only)
     const void* dY;
     const void* filt;  // W[KH][KW][C]
     void* dX;

@@ -65,8 +65,9 @@ typedef struct {
 } dgrad_problem_t;
 
 /* Element type of dY, W and dX (one type for all three).  DGRAD_F16 is served by
- * dgrad_pointwise, dgrad_dense and dgrad_grouped (tcgen05 f16 operands, fp32
- * accumulation); other entry points return DGRAD_ERR_UNSUPPORTED for it. */
+ * dgrad_pointwise, dgrad_dense, dgrad_grouped and dgrad_depthwise_tc (tcgen05
+ * f16 operands, fp32 accumulation); other entry points return
+ * DGRAD_ERR_UNSUPPORTED for it. */
 typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1, DGRAD_F16 = 2 } dgrad_dtype_t;
 
 /* Depthwise kernel choice.  AUTO: rotated-filter for stride 1, row-streaming
@@ -190,9 +191,9 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
  * rotated-filter correlation ("channel-packed and large-filter depthwise
  * dgrad", Technical Details: rotated-filter dgrad; the pages sent large filters
  * through an implicit-GEMM path before the FP32 rotated-filter kernel).  The
- * MMAs run in bf16 with fp32 accumulation (tcgen05), so results equal those of
- * dgrad_depthwise up to fp32 summation order.
- * Requirements: DGRAD_BF16, stride 1, K == C, KH and KW <= 64,
+ * MMAs run in bf16 (or f16) with fp32 accumulation (tcgen05), so results equal
+ * those of dgrad_depthwise up to fp32 summation order.
+ * Requirements: DGRAD_BF16 or DGRAD_F16, stride 1, K == C, KH and KW <= 64,
  * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1, N, H, W <= 65535; else
  * DGRAD_ERR_UNSUPPORTED (also when the filter is too large for the tile plan).
  * workspace: caller-owned device memory, 16-byte aligned, at least the size

@@ -195,6 +195,8 @@ TC_SMALL = [
     P("tc17x17_nonsame", "depthwise", "bf16", 10, 40, 33, 16, 16, 17, 17, 1, 3, 11, seed=156),
     P("tc11x9_c136_ragged_x", "depthwise", "bf16", 3, 37, 70, 136, 136, 11, 9, 1, 5, 4, seed=157),
     P("tc9x9_tail_split", "depthwise", "bf16", 8, 20, 24, 152, 152, 9, 9, 1, 4, 4, seed=161),   # 152 planes
+    P("tc31x31_f16", "depthwise", "f16", 3, 20, 20, 16, 16, 31, 31, 1, 15, 15, seed=162),
+    P("tc51x5_f16", "depthwise", "f16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=163),
     P("tc9x21_c64_long_w", "depthwise", "bf16", 9, 66, 45, 64, 64, 9, 21, 1, 4, 10, seed=158),
     P("tc21x9_c192_long_h", "depthwise", "bf16", 2, 45, 67, 192, 192, 21, 9, 1, 10, 4, seed=159),
     P("tc5x51", "depthwise", "bf16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=154),
