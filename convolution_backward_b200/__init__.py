@@ -265,7 +265,7 @@ def depthwise(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, mode="auto",
 
 
 def dense(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=None, stream=None, **kw):
-    """Dense (ungrouped) dgrad on the tensor cores (bf16; dgrad_dense): dY (N,Ho,Wo,K),
+    """Dense (ungrouped) dgrad on the tensor cores (bf16 or f16; dgrad_dense): dY (N,Ho,Wo,K),
     W (KH,KW,K,C) -> dX (N,H,W,C).  H and W_out (alias ``Wd``) are dX's spatial extents."""
     import torch
     if W_out is None:

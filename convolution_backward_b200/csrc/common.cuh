@@ -495,6 +495,13 @@ __device__ __forceinline__ uint32_t float2_to_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t u)
+{
+    __half2 h;
+    *reinterpret_cast<uint32_t*>(&h) = u;
+    return __half22float2(h);
+}
+
 __device__ __forceinline__ uint32_t float2_to_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
@@ -502,5 +509,30 @@ __device__ __forceinline__ uint32_t float2_to_bf16x2(float lo, float hi)
 }
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// Element kinds of the FMA depthwise kernels (dY, W and dX share one): fp32, or a
+// 16-bit format widened to fp32 on load and rounded back on store.
+enum ElemKind : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+
+// One 32-bit word holding a channel pair of 16-bit kind EK, to fp32 and back.
+template <int EK>
+__device__ __forceinline__ float2 h16x2_to_float2(uint32_t u)
+{
+    static_assert(EK == kBF16 || EK == kF16, "16-bit kinds only");
+    if constexpr (EK == kF16)
+        return f16x2_to_float2(u);
+    else
+        return bf16x2_to_float2(u);
+}
+
+template <int EK>
+__device__ __forceinline__ uint32_t float2_to_h16x2(float lo, float hi)
+{
+    static_assert(EK == kBF16 || EK == kF16, "16-bit kinds only");
+    if constexpr (EK == kF16)
+        return float2_to_f16x2(lo, hi);
+    else
+        return float2_to_bf16x2(lo, hi);
+}
 
 }  // namespace dgrad

@@ -93,9 +93,10 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
-// 4-D bf16 NHWC tensor (C innermost), box[4] inner first, no swizzle, zero fill.
-bool encode_nhwc_bf16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H, uint64_t W, uint64_t C,
-                      const unsigned box[4])
+// 4-D 16-bit NHWC tensor (C innermost; bf16, or f16 when f16), box[4] inner
+// first, no swizzle, zero fill.
+bool encode_nhwc_h16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H, uint64_t W, uint64_t C,
+                     const unsigned box[4], bool f16)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -103,7 +104,8 @@ bool encode_nhwc_bf16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H
     const cuuint64_t strides[3] = {C * 2, W * C * 2, H * W * C * 2};
     const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                     const_cast<void*>(base), dims, strides, b, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -503,7 +505,6 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     dgrad_status_t s = validate_common(prob, dtype, &Ho, &Wo, &pw);
     if (s != DGRAD_OK) return s;
     if (mode != DGRAD_DW_AUTO && mode != DGRAD_DW_ROTATED && mode != DGRAD_DW_ROWSTREAM) return DGRAD_ERR_INVALID;
-    if (dtype == DGRAD_F16) return DGRAD_ERR_UNSUPPORTED;
     if (prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
     if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
     if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;
@@ -513,7 +514,7 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     if (prob->H > (1 << 24) || prob->W > (1 << 24) || prob->C > (1 << 24)) return DGRAD_ERR_UNSUPPORTED;
     if (prob->N == 0) return DGRAD_OK;
     if (!dY || !W || !dX) return DGRAD_ERR_INVALID;
-    const int64_t esz = dtype == DGRAD_BF16 ? 2 : 4;
+    const int64_t esz = dtype == DGRAD_F32 ? 4 : 2;
     if (!aligned16(dY) || !aligned16(W) || !aligned16(dX) || (prob->C * esz) % 16) return DGRAD_ERR_ALIGNMENT;
 
     DeviceState* st = nullptr;
@@ -532,6 +533,7 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     a.ph = prob->pad_h;
     a.pw = pw;
     a.bf16 = dtype == DGRAD_BF16;
+    a.f16 = dtype == DGRAD_F16;
     a.dY = dY;
     a.filt = W;
     a.dX = dX;
@@ -545,16 +547,16 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     if (mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box)) {
         // small filters: one halo tile per CTA
         CUtensorMap map;
-        if (!encode_nhwc_bf16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
-                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box))
+        if (!encode_nhwc_h16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
+                             static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box, a.f16))
             return cuda_fail(cudaErrorInvalidValue);
         e = dgrad::launch_dw_tile(a, map, cs);
     } else if (mode == DGRAD_DW_ROTATED) {
         e = dgrad::launch_dw_rotated(a, cs);
     } else if (env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box)) {
         CUtensorMap map;
-        if (!encode_nhwc_bf16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
-                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box))
+        if (!encode_nhwc_h16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
+                             static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box, a.f16))
             return cuda_fail(cudaErrorInvalidValue);
         e = dgrad::launch_dw_rowstream_fast(a, map, 0, cs);
     } else {

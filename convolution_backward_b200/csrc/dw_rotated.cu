@@ -56,34 +56,34 @@ struct RotParams {
     int nA, nB, nC;
 };
 
-template <bool BF16>
+template <int EK>
 struct Chunk {
-    // A 16-byte chunk holds 8 bf16 or 4 f32 channels.
-    static constexpr int kElems = BF16 ? 8 : 4;
+    // A 16-byte chunk holds 8 16-bit or 4 f32 channels.
+    static constexpr int kElems = EK == kF32 ? 4 : 8;
     static constexpr int kPerPos = kCB / kElems;   // chunks per position (32 channels)
     static constexpr int kPairs = kElems / 2;      // channel pairs per chunk
 };
 
-template <bool BF16>
+template <int EK>
 __device__ __forceinline__ void chunk_to_pairs(const uint4& v, float2* dst)
 {
-    if constexpr (BF16) {
-        dst[0] = bf16x2_to_float2(v.x);
-        dst[1] = bf16x2_to_float2(v.y);
-        dst[2] = bf16x2_to_float2(v.z);
-        dst[3] = bf16x2_to_float2(v.w);
+    if constexpr (EK != kF32) {
+        dst[0] = h16x2_to_float2<EK>(v.x);
+        dst[1] = h16x2_to_float2<EK>(v.y);
+        dst[2] = h16x2_to_float2<EK>(v.z);
+        dst[3] = h16x2_to_float2<EK>(v.w);
     } else {
         dst[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
         dst[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
     }
 }
 
-template <int KAI, int TAT, bool BF16>
+template <int KAI, int TAT, int EK>
 __global__ void __launch_bounds__(kThreads, 2)
     dw_rot_kernel(const RotParams p)
 {
-    using Ch = Chunk<BF16>;
-    using T = typename std::conditional<BF16, __nv_bfloat16, float>::type;
+    using Ch = Chunk<EK>;
+    using T = typename std::conditional<EK == kF32, float, uint16_t>::type;
     extern __shared__ float2 sm2[];
     float2* ring = sm2;                                  // [RING][LA][16]
     float2* wbuf = sm2 + p.RING * p.LA * kPairs;         // [2][KAI][16]
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         float2* dst = ring + slot_idx * p.LA * kPairs;
 #pragma unroll
         for (int k = 0; k < kMaxPF; ++k)
-            if ((imask >> k) & 1u) chunk_to_pairs<BF16>(pf[k], dst + soff[k]);
+            if ((imask >> k) & 1u) chunk_to_pairs<EK>(pf[k], dst + soff[k]);
     };
     auto fetch_wline = [&](int jb, uint4 (&pw)[kWPF]) {
         const T* base = wg + (p.KB - 1 - jb) * p.w_sB;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         float2* dst = wbuf + (jb & 1) * KAI * kPairs;
 #pragma unroll
         for (int k = 0; k < kWPF; ++k)
-            if ((wimask >> k) & 1u) chunk_to_pairs<BF16>(pw[k], dst + wsoff[k]);
+            if ((wimask >> k) & 1u) chunk_to_pairs<EK>(pw[k], dst + wsoff[k]);
     };
 
     // Prologue: the first TB dY lines and filter line 0.
@@ -239,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int j = 0; j < TAT; ++j) {
         const int a = a0 + strip * TAT + j;
         if (a < p.OA) {
-            if constexpr (BF16)
-                *reinterpret_cast<uint32_t*>(out + a * p.out_sA) = float2_to_bf16x2(acc[j].x, acc[j].y);
+            if constexpr (EK != kF32)
+                *reinterpret_cast<uint32_t*>(out + a * p.out_sA) = float2_to_h16x2<EK>(acc[j].x, acc[j].y);
             else
                 *reinterpret_cast<float2*>(out + a * p.out_sA) = acc[j];
         }
@@ -254,11 +254,11 @@ constexpr int tat_for() { return KAI <= 7 ? 8 : 16; }
 template <int KAI>
 constexpr int tat_alt() { return KAI <= 7 ? 16 : 32; }
 
-template <int KAI, int TAT, bool BF16>
+template <int KAI, int TAT, int EK>
 cudaError_t launch_one(RotParams& p, long long blocks, cudaStream_t stream)
 {
     const size_t smem = static_cast<size_t>(p.RING * p.LA + 2 * KAI) * kPairs * sizeof(float2);
-    auto kern = dw_rot_kernel<KAI, TAT, BF16>;
+    auto kern = dw_rot_kernel<KAI, TAT, EK>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p);
@@ -285,24 +285,26 @@ void plan_tiles(RotParams& p)
 }
 
 template <int KAI, int TAT>
-cudaError_t dispatch_t(RotParams& p, int N, bool bf16, cudaStream_t stream)
+cudaError_t dispatch_t(RotParams& p, int N, int ek, cudaStream_t stream)
 {
     plan_tiles<TAT, KAI>(p);
     const long long blocks = static_cast<long long>(N) * p.nC * p.nB * p.nA;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    const int per_pos = bf16 ? Chunk<true>::kPerPos : Chunk<false>::kPerPos;
+    const int per_pos = ek == kF32 ? Chunk<kF32>::kPerPos : Chunk<kBF16>::kPerPos;
     if (p.LA * per_pos > kMaxPF * kThreads) return cudaErrorInvalidConfiguration;
-    return bf16 ? launch_one<KAI, TAT, true>(p, blocks, stream) : launch_one<KAI, TAT, false>(p, blocks, stream);
+    if (ek == kF16) return launch_one<KAI, TAT, kF16>(p, blocks, stream);
+    if (ek == kBF16) return launch_one<KAI, TAT, kBF16>(p, blocks, stream);
+    return launch_one<KAI, TAT, kF32>(p, blocks, stream);
 }
 
 // Outputs per thread along A: tat_for<KAI>() by default; DGRAD_ROT_TAT may select tat_alt<KAI>().
 template <int KAI>
-cudaError_t dispatch(RotParams& p, int N, bool bf16, cudaStream_t stream)
+cudaError_t dispatch(RotParams& p, int N, int ek, cudaStream_t stream)
 {
     const char* e = getenv("DGRAD_ROT_TAT");
-    if (e && atoi(e) == tat_alt<KAI>()) return dispatch_t<KAI, tat_alt<KAI>()>(p, N, bf16, stream);
-    return dispatch_t<KAI, tat_for<KAI>()>(p, N, bf16, stream);
+    if (e && atoi(e) == tat_alt<KAI>()) return dispatch_t<KAI, tat_alt<KAI>()>(p, N, ek, stream);
+    return dispatch_t<KAI, tat_for<KAI>()>(p, N, ek, stream);
 }
 
 }  // namespace
@@ -334,22 +336,22 @@ cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream)
     for (int v : kInstKA)
         if (v >= p.KA) { kai = v; break; }
     switch (kai) {
-    case 1: return dispatch<1>(p, a.N, a.bf16, stream);
-    case 3: return dispatch<3>(p, a.N, a.bf16, stream);
-    case 5: return dispatch<5>(p, a.N, a.bf16, stream);
-    case 7: return dispatch<7>(p, a.N, a.bf16, stream);
-    case 9: return dispatch<9>(p, a.N, a.bf16, stream);
-    case 11: return dispatch<11>(p, a.N, a.bf16, stream);
-    case 13: return dispatch<13>(p, a.N, a.bf16, stream);
-    case 15: return dispatch<15>(p, a.N, a.bf16, stream);
-    case 17: return dispatch<17>(p, a.N, a.bf16, stream);
-    case 21: return dispatch<21>(p, a.N, a.bf16, stream);
-    case 25: return dispatch<25>(p, a.N, a.bf16, stream);
-    case 31: return dispatch<31>(p, a.N, a.bf16, stream);
-    case 33: return dispatch<33>(p, a.N, a.bf16, stream);
-    case 41: return dispatch<41>(p, a.N, a.bf16, stream);
-    case 51: return dispatch<51>(p, a.N, a.bf16, stream);
-    case 64: return dispatch<64>(p, a.N, a.bf16, stream);
+    case 1: return dispatch<1>(p, a.N, a.elem_kind(), stream);
+    case 3: return dispatch<3>(p, a.N, a.elem_kind(), stream);
+    case 5: return dispatch<5>(p, a.N, a.elem_kind(), stream);
+    case 7: return dispatch<7>(p, a.N, a.elem_kind(), stream);
+    case 9: return dispatch<9>(p, a.N, a.elem_kind(), stream);
+    case 11: return dispatch<11>(p, a.N, a.elem_kind(), stream);
+    case 13: return dispatch<13>(p, a.N, a.elem_kind(), stream);
+    case 15: return dispatch<15>(p, a.N, a.elem_kind(), stream);
+    case 17: return dispatch<17>(p, a.N, a.elem_kind(), stream);
+    case 21: return dispatch<21>(p, a.N, a.elem_kind(), stream);
+    case 25: return dispatch<25>(p, a.N, a.elem_kind(), stream);
+    case 31: return dispatch<31>(p, a.N, a.elem_kind(), stream);
+    case 33: return dispatch<33>(p, a.N, a.elem_kind(), stream);
+    case 41: return dispatch<41>(p, a.N, a.elem_kind(), stream);
+    case 51: return dispatch<51>(p, a.N, a.elem_kind(), stream);
+    case 64: return dispatch<64>(p, a.N, a.elem_kind(), stream);
     default: return cudaErrorInvalidValue;
     }
 }

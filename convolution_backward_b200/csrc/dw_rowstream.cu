@@ -52,33 +52,33 @@ struct RsParams {
 
 __device__ __forceinline__ int floor_div(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
 
-template <bool BF16>
+template <int EK>
 struct RsChunk {
-    static constexpr int kElems = BF16 ? 8 : 4;
+    static constexpr int kElems = EK == kF32 ? 4 : 8;
     static constexpr int kPerPos = kCB / kElems;
     static constexpr int kPairs = kElems / 2;
 };
 
-template <bool BF16>
+template <int EK>
 __device__ __forceinline__ void rs_chunk_to_pairs(const uint4& v, float2* dst)
 {
-    if constexpr (BF16) {
-        dst[0] = bf16x2_to_float2(v.x);
-        dst[1] = bf16x2_to_float2(v.y);
-        dst[2] = bf16x2_to_float2(v.z);
-        dst[3] = bf16x2_to_float2(v.w);
+    if constexpr (EK != kF32) {
+        dst[0] = h16x2_to_float2<EK>(v.x);
+        dst[1] = h16x2_to_float2<EK>(v.y);
+        dst[2] = h16x2_to_float2<EK>(v.z);
+        dst[3] = h16x2_to_float2<EK>(v.w);
     } else {
         dst[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
         dst[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
     }
 }
 
-template <bool BF16>
+template <int EK>
 __global__ void __launch_bounds__(kThreads)
     dw_rowstream_kernel(const RsParams p)
 {
-    using Ch = RsChunk<BF16>;
-    using T = typename std::conditional<BF16, __nv_bfloat16, float>::type;
+    using Ch = RsChunk<EK>;
+    using T = typename std::conditional<EK == kF32, float, uint16_t>::type;
     extern __shared__ float2 sm2[];
     float2* ring = sm2;                                   // [R][TX][16]
     float2* dyrow = ring + p.R * p.TX * kPairs;           // [LW][16]
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads)
             const int cc = c0 + ch * Ch::kElems;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (cc < p.C) v = __ldg(reinterpret_cast<const uint4*>(wg + tap * C + cc));
-            rs_chunk_to_pairs<BF16>(v, wsm + tap * kPairs + ch * Ch::kPairs);
+            rs_chunk_to_pairs<EK>(v, wsm + tap * kPairs + ch * Ch::kPairs);
         }
     }
 
@@ -145,15 +145,15 @@ __global__ void __launch_bounds__(kThreads)
             if (it < row_items) {
                 const int j = it / Ch::kPerPos;
                 const int ch = it - j * Ch::kPerPos;
-                rs_chunk_to_pairs<BF16>(pf[k], dyrow + j * kPairs + ch * Ch::kPairs);
+                rs_chunk_to_pairs<EK>(pf[k], dyrow + j * kPairs + ch * Ch::kPairs);
             }
         }
     };
     auto weight = [&](int tap) -> float2 {
         if (p.w_in_smem) return wsm[tap * kPairs + cp];
         if (!c_ok) return make_float2(0.f, 0.f);
-        if constexpr (BF16)
-            return bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(wg + tap * C + c)));
+        if constexpr (EK != kF32)
+            return h16x2_to_float2<EK>(__ldg(reinterpret_cast<const uint32_t*>(wg + tap * C + c)));
         else
             return __ldg(reinterpret_cast<const float2*>(wg + tap * C + c));
     };
@@ -169,8 +169,8 @@ __global__ void __launch_bounds__(kThreads)
             *e = make_float2(0.f, 0.f);
             if (x < p.W && c_ok) {
                 T* o = dx + (static_cast<long long>(h) * p.W + x) * C + c;
-                if constexpr (BF16)
-                    *reinterpret_cast<uint32_t*>(o) = float2_to_bf16x2(v.x, v.y);
+                if constexpr (EK != kF32)
+                    *reinterpret_cast<uint32_t*>(o) = float2_to_h16x2<EK>(v.x, v.y);
                 else
                     *reinterpret_cast<float2*>(o) = v;
             }
@@ -214,10 +214,10 @@ __global__ void __launch_bounds__(kThreads)
     for (; next_flush < p.H; ++next_flush) flush_row(next_flush);   // tail
 }
 
-template <bool BF16>
+template <int EK>
 cudaError_t launch_t(const RsParams& p, long long blocks, size_t smem, cudaStream_t stream)
 {
-    auto kern = dw_rowstream_kernel<BF16>;
+    auto kern = dw_rowstream_kernel<EK>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p);
@@ -250,12 +250,14 @@ cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream)
     p.LW = (p.TX - 1 + a.KW - 1) / a.S + 2;
     const size_t smem = smem_for(p.TX, p.w_in_smem);
     if (smem > kSmemBudget) return cudaErrorInvalidConfiguration;
-    const int per_pos = a.bf16 ? RsChunk<true>::kPerPos : RsChunk<false>::kPerPos;
+    const int per_pos = a.elem_kind() == kF32 ? RsChunk<kF32>::kPerPos : RsChunk<kBF16>::kPerPos;
     if (p.LW * per_pos > kMaxPF * kThreads) return cudaErrorInvalidConfiguration;
     const long long blocks = static_cast<long long>(a.N) * p.nC * p.nX;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    return a.bf16 ? launch_t<true>(p, blocks, smem, stream) : launch_t<false>(p, blocks, smem, stream);
+    if (a.f16) return launch_t<kF16>(p, blocks, smem, stream);
+    if (a.bf16) return launch_t<kBF16>(p, blocks, smem, stream);
+    return launch_t<kF32>(p, blocks, smem, stream);
 }
 
 }  // namespace dgrad

@@ -1,4 +1,4 @@
-// dw_rowstream_fast.cu -- row-streaming depthwise dgrad, register-blocked (bf16).
+// dw_rowstream_fast.cu -- row-streaming depthwise dgrad, register-blocked (bf16 or f16).
 //
 // The row-streaming schedule of "channel-packed and large-filter depthwise
 // dgrad" (Technical Details, channel-packed row-streaming dgrad) for strided
@@ -26,7 +26,7 @@
 //   * G dY rows are applied per step, all in registers: they touch
 //     (G-1)*S + KH dX rows, of which the first KH-S come in from the shared
 //     accumulator ring (the rows left open by the previous step), the first
-//     G*S are final afterwards and are rounded to bf16 and stored, and the last
+//     G*S are final afterwards and are rounded to 16 bits and stored, and the last
 //     KH-S go back to the ring.  Ring entries are private to their thread, so
 //     the ring needs no barriers; one __syncthreads per step recycles the TMA
 //     stage.
@@ -46,8 +46,8 @@ constexpr int kStages = 6;
 constexpr int kMaxThreads = 256;
 
 struct FastParams {
-    __nv_bfloat16* dX;
-    const __nv_bfloat16* filt;
+    uint16_t* dX;         // 16-bit elements (bf16 or f16)
+    const uint16_t* filt;
     int* status;
     int N, H, W, C, Ho, Wo, ph, pw;
     int nslot;    // slots per CTA (threads = 16 * nslot), a multiple of 2*S
@@ -68,18 +68,18 @@ struct RsGeom {
 };
 
 // One step with a fixed tap count NT (the thread's column phase has NT taps).
-template <int KH, int KW, int S, int Q, int G, int NT>
+template <int KH, int KW, int S, int Q, int G, int NT, int EK>
 __device__ __forceinline__ void rs_step(float2 (&acc)[RsGeom<KH, KW, S, Q, G>::RB][Q],
                                         const float2 (&wr)[KH][RsGeom<KH, KW, S, Q, G>::NTMAX],
                                         const uint32_t* stage, int LW, int cp, int col0)
 {
-    // stage: [G][LW][32 channels] bf16 -> as uint32 pairs: [G][LW][16]
+    // stage: [G][LW][32 channels] 16-bit -> as uint32 pairs: [G][LW][16]
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         float2 dv[Q + NT - 1];
         const uint32_t* row = stage + (g * LW + col0) * 16 + cp;
 #pragma unroll
-        for (int m = 0; m < Q + NT - 1; ++m) dv[m] = bf16x2_to_float2(row[m * 16]);
+        for (int m = 0; m < Q + NT - 1; ++m) dv[m] = h16x2_to_float2<EK>(row[m * 16]);
         // taps outermost: consecutive FMAs update different accumulators
 #pragma unroll
         for (int i = 0; i < NT; ++i)
@@ -91,7 +91,7 @@ __device__ __forceinline__ void rs_step(float2 (&acc)[RsGeom<KH, KW, S, Q, G>::R
     }
 }
 
-template <int KH, int KW, int S, int Q, int G>
+template <int KH, int KW, int S, int Q, int G, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_fast_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
 {
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);   // TMA destinations 128-byte aligned
     const int nthreads = 16 * p.nslot;
-    const int stage_bytes = G * p.LW * 64;                       // 32 bf16 channels = 64 bytes
+    const int stage_bytes = G * p.LW * 64;                       // 32 16-bit channels = 64 bytes
     const int stage_stride = (stage_bytes + 127) & ~127;         // TMA destinations are 128-byte aligned
     uint32_t* stages = reinterpret_cast<uint32_t*>(smem);
     float4* carry = reinterpret_cast<float4*>(smem + kStages * stage_stride);  // [NC][Q/2][nthreads]
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int col0 = e - (nt - 1) - wo_start;        // staged column of dv[0]
     // store addressing: dX row h of this thread's columns is obase + h*row_elems + xoff[q]
     const long long row_elems = static_cast<long long>(p.W) * p.C;
-    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+    uint16_t* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
     int xoff[Q];
     uint32_t xmask = 0;
 #pragma unroll
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             const int s = s0 + S * i;
             float2 v = make_float2(0.f, 0.f);
             if (s < KW && c_ok)
-                v = bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + s) * p.C + c)));
+                v = h16x2_to_float2<EK>(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + s) * p.C + c)));
             wr[r][i] = v;
         }
     // clear this thread's carried rows
@@ -220,9 +220,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t* stage = reinterpret_cast<const uint32_t*>(reinterpret_cast<uint8_t*>(stages) +
                                                                   sidx * stage_stride);
         if (nt == NTMAX)
-            rs_step<KH, KW, S, Q, G, NTMAX>(acc, wr, stage, p.LW, cp, col0);
+            rs_step<KH, KW, S, Q, G, NTMAX, EK>(acc, wr, stage, p.LW, cp, col0);
         else
-            rs_step<KH, KW, S, Q, G, NTMAX - 1>(acc, wr, stage, p.LW, cp, col0);
+            rs_step<KH, KW, S, Q, G, NTMAX - 1, EK>(acc, wr, stage, p.LW, cp, col0);
 
         // rows hb .. hb+NF-1 are final
         const int hb = hb0 + step * NF;
@@ -230,11 +230,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         for (int i = 0; i < NF; ++i) {
             const int h = hb + i;
             if (h >= h0 && h < h1) {
-                __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
+                uint16_t* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
                 for (int q = 0; q < Q; ++q)
                     if ((xmask >> q) & 1u)
-                        *reinterpret_cast<uint32_t*>(orow + xoff[q]) = float2_to_bf16x2(acc[i][q].x, acc[i][q].y);
+                        *reinterpret_cast<uint32_t*>(orow + xoff[q]) = float2_to_h16x2<EK>(acc[i][q].x, acc[i][q].y);
             }
         }
         // rows hb+NF .. hb+RB-1 stay open: back to the ring
@@ -262,10 +262,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 // nothing is carried through shared memory and there is one barrier per stage.
 // After dY row t of the band the S rows in slots (S*t .. S*t+S-1) mod RS are
 // final: they are stored (if inside the band) and cleared.
-template <int KH, int KW, int S, int Q, int RS, int GT, int NT>
+template <int KH, int KW, int S, int Q, int RS, int GT, int NT, int EK>
 __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 (&wr)[KH][(KW + S - 1) / S],
                                              const uint32_t* stage, int LW, int cp, int col0, int hb, int h0,
-                                             int h1, __nv_bfloat16* obase, long long row_elems,
+                                             int h1, uint16_t* obase, long long row_elems,
                                              const int (&xoff)[Q], uint32_t xmask)
 {
     static_assert((S * GT) % RS == 0 && RS >= KH && KH >= S, "ring geometry");
@@ -274,7 +274,7 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
     auto load_row = [&](int k, float2 (&d)[Q + NT - 1]) {
         const uint32_t* row = stage + (k * LW + col0) * 16 + cp;
 #pragma unroll
-        for (int m = 0; m < Q + NT - 1; ++m) d[m] = bf16x2_to_float2(row[m * 16]);
+        for (int m = 0; m < Q + NT - 1; ++m) d[m] = h16x2_to_float2<EK>(row[m * 16]);
     };
     load_row(0, dv);
 #pragma unroll
@@ -303,12 +303,12 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
             const int slot = (S * k + i) % RS;
             const int h = hb + S * k + i;
             if (h >= h0 && h < h1) {
-                __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
+                uint16_t* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
                 for (int q = 0; q < Q; ++q)
                     if ((xmask >> q) & 1u)
                         *reinterpret_cast<uint32_t*>(orow + xoff[q]) =
-                            float2_to_bf16x2(acc[slot][q].x, acc[slot][q].y);
+                            float2_to_h16x2<EK>(acc[slot][q].x, acc[slot][q].y);
             }
         }
         if (k + 1 < GT)
@@ -317,7 +317,7 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
     }
 }
 
-template <int KH, int KW, int S, int Q, int RS, int GT>
+template <int KH, int KW, int S, int Q, int RS, int GT, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_reg_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
 {
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                                                        : -((-(x0 + p.pw - (KW - 1)) + S - 1) / S);
     const int col0 = e - (nt - 1) - wo_start;
     const long long row_elems = static_cast<long long>(p.W) * p.C;
-    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+    uint16_t* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
     int xoff[Q];
     uint32_t xmask = 0;
 #pragma unroll
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         for (int i = 0; i < NTMAX; ++i) {
             const int sx = s0 + S * i;
             wr[r][i] = (sx < KW && c_ok)
-                           ? bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + sx) * p.C + c)))
+                           ? h16x2_to_float2<EK>(__ldg(reinterpret_cast<const uint32_t*>(p.filt + (r * KW + sx) * p.C + c)))
                            : make_float2(0.f, 0.f);
         }
     if (tid == 0) {
@@ -418,10 +418,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t* stage = reinterpret_cast<const uint32_t*>(smem + sidx * stage_stride);
         const int hb = hb0 + st * GT * S;
         if (nt == NTMAX)
-            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
+            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX, EK>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
                                                       row_elems, xoff, xmask);
         else
-            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX - 1>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
+            rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX - 1, EK>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
                                                           row_elems, xoff, xmask);
         __syncthreads();
     }
@@ -435,8 +435,8 @@ FastParams plan_fast(const DwArgs& a)
 {
     using Geo = RsGeom<KH, KW, S, Q, G>;
     FastParams p{};
-    p.dX = static_cast<__nv_bfloat16*>(a.dX);
-    p.filt = static_cast<const __nv_bfloat16*>(a.filt);
+    p.dX = static_cast<uint16_t*>(a.dX);
+    p.filt = static_cast<const uint16_t*>(a.filt);
     p.status = a.status;
     p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.Ho = a.Ho; p.Wo = a.Wo; p.ph = a.ph; p.pw = a.pw;
     // strip width: pick the slot count (multiple of 2*S, at most 16) that wastes the fewest columns
@@ -462,7 +462,7 @@ FastParams plan_fast(const DwArgs& a)
     const long long base = static_cast<long long>(a.N) * p.nC * p.nX;
     const int sms = device_sm_count();
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dw_rs_fast_kernel<KH, KW, S, Q, G>, 16 * p.nslot,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dw_rs_fast_kernel<KH, KW, S, Q, G, kBF16>, 16 * p.nslot,
                                                       0) != cudaSuccess || per_sm < 1)
         per_sm = 1;
     const long long slots = static_cast<long long>(sms) * per_sm;
@@ -486,7 +486,7 @@ cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     const int nthreads = 16 * p.nslot;
     const size_t smem = static_cast<size_t>(kStages) * ((G * p.LW * 64 + 127) & ~127) +
                         static_cast<size_t>(Geo::NC) * (Q / 2) * nthreads * sizeof(float4) + kStages * 8 + 128;
-    auto kern = dw_rs_fast_kernel<KH, KW, S, Q, G>;
+    auto kern = a.f16 ? dw_rs_fast_kernel<KH, KW, S, Q, G, kF16> : dw_rs_fast_kernel<KH, KW, S, Q, G, kBF16>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
@@ -503,7 +503,7 @@ cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, cudaStream_t str
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const int nthreads = 16 * p.nslot;
     const size_t smem = static_cast<size_t>(kStages) * ((GT * p.LW * 64 + 127) & ~127) + kStages * 8 + 128;
-    auto kern = dw_rs_reg_kernel<KH, KW, S, Q, RS, GT>;
+    auto kern = a.f16 ? dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kF16> : dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kBF16>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
@@ -558,7 +558,7 @@ static int alt_g()
 
 bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4])
 {
-    if (!a.bf16) return false;
+    if (!(a.bf16 || a.f16)) return false;
     if (use_reg_ring()) {
 #define DGRAD_RS_REG_BOX(kh, kw, s, q, rs, gt)                                                     \
         if (a.KH == kh && a.KW == kw && a.S == s) {                                                 \
@@ -588,7 +588,7 @@ bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4])
 cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, int G, cudaStream_t stream)
 {
     (void)G;
-    if (!a.bf16) return cudaErrorNotSupported;
+    if (!(a.bf16 || a.f16)) return cudaErrorNotSupported;
     if (use_reg_ring()) {
 #define DGRAD_RS_REG_LAUNCH(kh, kw, s, q, rs, gt) \
         if (a.KH == kh && a.KW == kw && a.S == s) return launch_reg<kh, kw, s, q, rs, gt>(a, dy_map, stream);

@@ -1,4 +1,4 @@
-// dw_tile.cu -- stride-1 depthwise dgrad for small filters (up to 7 x 7), bf16.
+// dw_tile.cu -- stride-1 depthwise dgrad for small filters (up to 7 x 7), bf16 or f16.
 //
 // The rotated-filter correlation of "channel-packed and large-filter depthwise
 // dgrad" (Technical Details, rotated-filter dgrad):
@@ -11,10 +11,10 @@
 //     load brings its whole halo tile [TH+KH-1][TW+KW-1][32] of dY into shared
 //     memory, the out-of-image part zero-filled by the TMA (that is the padding);
 //   * thread (channel pair, row slot, column slot) computes R rows x TAT columns;
-//     it walks the R+KH-1 input rows it needs once, converting each bf16 pair
+//     it walks the R+KH-1 input rows it needs once, converting each 16-bit pair
 //     to fp32 once, and applies every filter row that input row reaches
 //     (packed fma.rn.f32x2, the rotated filter held in registers);
-//   * results are rounded to bf16 and stored straight to dX (16 threads write
+//   * results are rounded to the I/O format and stored straight to dX (16 threads write
 //     64 contiguous bytes).
 #include "common.cuh"
 #include "host_util.h"
@@ -24,8 +24,8 @@ namespace dgrad {
 namespace {
 
 struct TileParams {
-    __nv_bfloat16* dX;
-    const __nv_bfloat16* filt;
+    uint16_t* dX;         // 16-bit elements (bf16 or f16)
+    const uint16_t* filt;
     int* status;
     int N, H, W, C, ph, pw;
     int CS, RS;       // column and row slots per CTA (threads = 16 * CS * RS)
@@ -33,7 +33,7 @@ struct TileParams {
     int nX, nY, nC;
 };
 
-template <int KH, int KW, int R, int TAT>
+template <int KH, int KW, int R, int TAT, int EK>
 __global__ void __launch_bounds__(256)
     dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const TileParams p)
 {
@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256)
     const int LHt = p.TH + KH - 1;                        // staged rows
     const uint32_t tile_bytes = static_cast<uint32_t>(LWt * LHt * 64);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + ((tile_bytes + 15u) & ~15u));
-    const uint32_t* tile = reinterpret_cast<const uint32_t*>(smem);   // [LHt][LWt][16] bf16 pairs
+    const uint32_t* tile = reinterpret_cast<const uint32_t*>(smem);   // [LHt][LWt][16] 16-bit pairs
 
     int u = blockIdx.x;
     const int xblk = u % p.nX;
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(256)
     for (int r = 0; r < KH; ++r)
 #pragma unroll
         for (int s = 0; s < KW; ++s)
-            wr[r][s] = c_ok ? bf16x2_to_float2(__ldg(reinterpret_cast<const uint32_t*>(
+            wr[r][s] = c_ok ? h16x2_to_float2<EK>(__ldg(reinterpret_cast<const uint32_t*>(
                                   p.filt + ((KH - 1 - r) * KW + (KW - 1 - s)) * p.C + c)))
                             : make_float2(0.f, 0.f);
 
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256)
         float2 x[TAT + KW - 1];
         const uint32_t* src = tile + ((row0 + i) * LWt + col0) * 16 + cp;
 #pragma unroll
-        for (int m = 0; m < TAT + KW - 1; ++m) x[m] = bf16x2_to_float2(src[m * 16]);
+        for (int m = 0; m < TAT + KW - 1; ++m) x[m] = h16x2_to_float2<EK>(src[m * 16]);
         // taps outermost: consecutive FMAs update different accumulators
 #pragma unroll
         for (int s = 0; s < KW; ++s)
@@ -127,18 +127,18 @@ __global__ void __launch_bounds__(256)
 
     if (!c_ok) return;
     const long long row_elems = static_cast<long long>(p.W) * p.C;
-    __nv_bfloat16* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
+    uint16_t* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
 #pragma unroll
     for (int ro = 0; ro < R; ++ro) {
         const int h = h0 + row0 + ro;
         if (h >= p.H || row0 + ro >= p.TH) continue;
-        __nv_bfloat16* orow = obase + static_cast<long long>(h) * row_elems;
+        uint16_t* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
         for (int j = 0; j < TAT; ++j) {
             const int w = w0 + col0 + j;
             if (w < p.W && col0 + j < p.TW)
                 *reinterpret_cast<uint32_t*>(orow + static_cast<long long>(w) * p.C) =
-                    float2_to_bf16x2(acc[ro][j].x, acc[ro][j].y);
+                    float2_to_h16x2<EK>(acc[ro][j].x, acc[ro][j].y);
         }
     }
 }
@@ -147,8 +147,8 @@ template <int KH, int KW, int R, int TAT>
 TileParams plan_tile(const DwArgs& a)
 {
     TileParams p{};
-    p.dX = static_cast<__nv_bfloat16*>(a.dX);
-    p.filt = static_cast<const __nv_bfloat16*>(a.filt);
+    p.dX = static_cast<uint16_t*>(a.dX);
+    p.filt = static_cast<const uint16_t*>(a.filt);
     p.status = a.status;
     p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.ph = a.ph; p.pw = a.pw;
     // columns: as few column slots as cover the row (at most 16), balanced
@@ -179,7 +179,7 @@ cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const size_t tile = static_cast<size_t>(p.TW + KW - 1) * (p.TH + KH - 1) * 64;
     const size_t smem = ((tile + 15) & ~static_cast<size_t>(15)) + 16 + 128;
-    auto kern = dw_tile_kernel<KH, KW, R, TAT>;
+    auto kern = a.f16 ? dw_tile_kernel<KH, KW, R, TAT, kF16> : dw_tile_kernel<KH, KW, R, TAT, kBF16>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), 16 * p.CS * p.RS, smem, stream>>>(map, p);
@@ -195,7 +195,7 @@ cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
 
 bool dw_tile_box(const DwArgs& a, unsigned box[4])
 {
-    if (!a.bf16 || a.S != 1) return false;
+    if (!(a.bf16 || a.f16) || a.S != 1) return false;
 #define DGRAD_TILE_BOX(kh, kw, r, tat)                                                              \
     if (a.KH == kh && a.KW == kw) {                                                                 \
         const TileParams p = plan_tile<kh, kw, r, tat>(a);                                          \
@@ -210,7 +210,7 @@ bool dw_tile_box(const DwArgs& a, unsigned box[4])
 
 cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream)
 {
-    if (!a.bf16 || a.S != 1) return cudaErrorNotSupported;
+    if (!(a.bf16 || a.f16) || a.S != 1) return cudaErrorNotSupported;
 #define DGRAD_TILE_LAUNCH(kh, kw, r, tat) \
     if (a.KH == kh && a.KW == kw) return launch_tile<kh, kw, r, tat>(a, dy_map, stream);
     DGRAD_TILE_SET(DGRAD_TILE_LAUNCH)

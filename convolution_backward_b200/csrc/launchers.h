@@ -77,8 +77,9 @@ void record_cuda_error(cudaError_t e);
 // Depthwise problem (groups = C = K), NHWC, dense.
 struct DwArgs {
     int N, H, W, C, Ho, Wo, KH, KW, S, ph, pw;
-    bool bf16;  // element type of dY, W and dX: bf16 (true) or f32 (false)
-    bool f16;   // f16 instead (tensor-core depthwise only)
+    bool bf16;  // element type of dY, W and dX: bf16 (true), or f32 / f16 (false)
+    bool f16;   // element type f16 (bf16 is false then)
+    int elem_kind() const { return f16 ? 2 : bf16 ? 1 : 0; }   // ElemKind of the device code
     const void* dY;
     const void* filt;  // W[KH][KW][C]
     void* dX;
@@ -88,8 +89,8 @@ struct DwArgs {
 // Stride-1 rotated-filter correlation.  Requires S == 1, KH, KW <= 64.
 cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream);
 
-// Stride-1 depthwise for small filters (3x3, 5x5, 7x7; bf16): one TMA halo tile
-// per CTA.  dy_map covers dY as a 4-D bf16 tensor (C, Wo, Ho, N innermost first)
+// Stride-1 depthwise for small filters (3x3, 5x5, 7x7; bf16 or f16): one TMA halo
+// tile per CTA.  dy_map covers dY as a 4-D 16-bit tensor (C, Wo, Ho, N innermost first)
 // with the box dw_tile_box returns.  cudaErrorNotSupported when not compiled.
 bool dw_tile_box(const DwArgs& a, unsigned box[4]);
 cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream);
@@ -125,7 +126,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
 cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);
 
 // Register-blocked row-streaming kernel for the compiled (KH, KW, S) set, bf16
-// only.  dy_map covers dY as a 4-D bf16 tensor (C, Wo, Ho, N innermost first)
+// or f16.  dy_map covers dY as a 4-D 16-bit tensor (C, Wo, Ho, N innermost first)
 // with no swizzle.  Returns cudaErrorNotSupported when no instantiation fits.
 cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, int G, cudaStream_t stream);
 

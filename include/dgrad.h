@@ -26,8 +26,9 @@
  * Layouts (all dense, channels innermost, no padding between rows):
  *     dY  [N][Ho][Wo][K]      dX [N][H][W][C]
  *     W   pointwise [K][C];   depthwise [KH][KW][C]
- * Element type: DGRAD_F32 (float in, float out) or DGRAD_BF16 (bf16 in, bf16
- * out).  Accumulation is always fp32; a bf16 dX is rounded once, to nearest even.
+ * Element type: DGRAD_F32 (float in, float out), DGRAD_BF16 (bf16 in, bf16 out)
+ * or DGRAD_F16 (f16 in, f16 out).  Accumulation is always fp32; a 16-bit dX is
+ * rounded once, to nearest even.
  *
  * Memory and streams.  Every pointer is device memory the caller owns (for
  * example a PyTorch CUDA tensor's data pointer) on the current device.  Calls
@@ -35,7 +36,7 @@
  * and return without synchronising; the library allocates no device memory per
  * call.  dX is written in full (never accumulated into), so it needs no zeroing.
  * Alignment: every base pointer 16-byte aligned, and K and C multiples of 8
- * (bf16) or 4 (f32), so that every channel row starts on 16 bytes.
+ * (bf16, f16) or 4 (f32), so that every channel row starts on 16 bytes.
  *
  * Errors.  Arguments are validated on the host before anything is launched; a
  * rejected call launches nothing and leaves dX untouched.  A launch failure is
@@ -66,7 +67,8 @@ typedef struct {
 
 /* Element type of dY, W and dX (one type for all three).  DGRAD_F16 is served by
  * dgrad_pointwise, dgrad_dense, dgrad_grouped and dgrad_depthwise_tc (tcgen05
- * f16 operands, fp32 accumulation); other entry points return
+ * f16 operands, fp32 accumulation) and by dgrad_depthwise (f16 widened to fp32
+ * on load, fp32 FMAs); dgrad_pointwise_splitk and its scratch variant return
  * DGRAD_ERR_UNSUPPORTED for it. */
 typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1, DGRAD_F16 = 2 } dgrad_dtype_t;
 
@@ -179,7 +181,8 @@ dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, con
  * Rotated-filter mode requires stride 1, KH and KW <= 64 and
  * 0 <= pad_h <= KH-1, 0 <= pad_w <= KW-1 (the rotated padding KH-1-pad_h and
  * KW-1-pad_w is then non-negative).  Row-streaming requires KH, KW <= 64,
- * stride <= 8, 0 <= pad_h <= KH-1 and 0 <= pad_w <= KW-1. */
+ * stride <= 8, 0 <= pad_h <= KH-1 and 0 <= pad_w <= KW-1.  Any element type:
+ * 16-bit inputs are widened to fp32 on load and dX is rounded once. */
 dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
                                dgrad_dw_mode_t mode,
                                const void* dY, const void* W, void* dX, void* stream);

@@ -233,7 +233,13 @@ def test_grouped_validation():
     assert call(p, 16) == ALIGNMENT         # C/groups = 4 channels: 8-byte rows
     assert call(cb.Problem(0, 8, 8, 64, 128, 3, 3, 1, 1, 1), 4, ptrs=(0, 0, 0)) == OK
     F16 = 2
+    # f16 depthwise: validated like bf16 (16-bit rows), refused before any launch
+    dw = cb.Problem(1, 8, 8, 12, 12, 3, 3, 1, 1, 1)
+    assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE, FAKE, FAKE, None) == ALIGNMENT   # 24-byte rows
     dw = cb.Problem(1, 8, 8, 16, 16, 3, 3, 1, 1, 1)
-    assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE, FAKE, FAKE, None) == UNSUPPORTED
+    assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE, 0, FAKE, None) == INVALID
+    assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE + 8, FAKE, FAKE, None) == ALIGNMENT
+    dw0 = cb.Problem(0, 8, 8, 16, 16, 7, 7, 2, 3, 3)
+    assert L.dgrad_depthwise(ctypes.byref(dw0), F16, 0, 0, 0, 0, None) == OK
     pw = cb.Problem(1, 8, 8, 16, 16, 1, 1, 1, 0, 0)
     assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F16, 0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == UNSUPPORTED

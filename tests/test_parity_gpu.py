@@ -149,6 +149,43 @@ def test_rotated_small_filter_kernels(p, kernel, monkeypatch):
     cb.check_status()
 
 
+DW_F16 = [
+    # stride 1: the halo-tile kernel (3x3, 5x5, 7x7) and the rotated-line kernel
+    (P("f16_tile3x3", "depthwise", "f16", 2, 19, 23, 40, 40, 3, 3, 1, 1, 1, seed=301), {}),
+    (P("f16_tile7x7", "depthwise", "f16", 1, 33, 31, 72, 72, 7, 7, 1, 3, 3, seed=302), {}),
+    (P("f16_line5x5", "depthwise", "f16", 1, 12, 14, 48, 48, 5, 5, 1, 2, 0, seed=303), {"DGRAD_ROT_KERNEL": "line"}),
+    (P("f16_line13x13", "depthwise", "f16", 1, 33, 35, 64, 64, 13, 13, 1, 6, 6, seed=304), {}),
+    (P("f16_line51x5", "depthwise", "f16", 1, 45, 30, 24, 24, 51, 5, 1, 25, 2, seed=305), {}),
+    (P("f16_line5x51", "depthwise", "f16", 1, 30, 45, 24, 24, 5, 51, 1, 2, 25, seed=306), {}),
+    # strided: register ring (two and four columns per thread), shared ring, generic
+    (P("f16_rs7x7s2", "depthwise", "f16", 2, 29, 27, 40, 40, 7, 7, 2, 3, 3, seed=307), {}),
+    (P("f16_rs7x7s2_q4", "depthwise", "f16", 1, 23, 40, 16, 16, 7, 7, 2, 6, 1, seed=308), {"DGRAD_RS_Q": "4"}),
+    (P("f16_rs5x5s2_smem", "depthwise", "f16", 2, 25, 26, 48, 48, 5, 5, 2, 2, 2, seed=309),
+     {"DGRAD_RS_KERNEL": "smem"}),
+    (P("f16_rs3x3s2", "depthwise", "f16", 1, 33, 34, 96, 96, 3, 3, 2, 1, 1, seed=310), {}),
+    (P("f16_rs5x3s3", "depthwise", "f16", 1, 22, 19, 16, 16, 5, 3, 3, 2, 1, seed=311), {}),
+    (P("f16_rs7x7s2_generic", "depthwise", "f16", 1, 30, 31, 32, 32, 7, 7, 2, 0, 0, seed=312),
+     {"DGRAD_RS_GENERIC": "1"}),
+]
+
+
+@pytest.mark.parametrize("p,env", DW_F16, ids=[p.name for p, _ in DW_F16])
+def test_depthwise_f16(p, env, monkeypatch):
+    """fp16 I/O on the FMA depthwise kernels (dgrad_depthwise): every kernel family,
+    f16 widened to fp32 on load, dX rounded once to f16."""
+    h = _h()
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=p.name)
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
 SPLITK = [
     (P("sk_small_m", "pointwise", "bf16", 2, 14, 14, 512, 2048, seed=91), [1, 2, 5, 0]),
     (P("sk_ragged", "pointwise", "bf16", 1, 7, 9, 136, 1000, seed=92), [3, 16, 0]),
