@@ -36,6 +36,7 @@
 #include "host_util.h"
 #include "launchers.h"
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 
@@ -430,10 +431,21 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             if (!mbar_wait(&full[sx % kStages], static_cast<uint32_t>((sx / kStages) & 1))) report_timeout(p.status);
 }
 
-template <int KH, int KW, int S, int Q, int G>
-FastParams plan_fast(const DwArgs& a)
+// Shared memory of one CTA: the TMA stages (G dY rows of LW columns each), their
+// barriers and, for the shared-ring kernel, the carried accumulator rows.
+inline size_t stage_smem(int G, int LW) { return static_cast<size_t>(kStages) * ((G * LW * 64 + 127) & ~127); }
+inline size_t fast_smem(int G, int LW, int NC, int Q, int nthreads)
 {
-    using Geo = RsGeom<KH, KW, S, Q, G>;
+    return stage_smem(G, LW) + static_cast<size_t>(NC) * (Q / 2) * nthreads * sizeof(float4) + kStages * 8 + 128;
+}
+inline size_t reg_smem(int GT, int LW) { return stage_smem(GT, LW) + kStages * 8 + 128; }
+
+// Strip and band plan.  kern / smem (the kernel that will run and its dynamic
+// shared memory per CTA) size the bands; without them one band covers dX.
+template <int KH, int KW, int S, int Q, int G>
+FastParams plan_fast(const DwArgs& a, const void* kern = nullptr, size_t (*smem_of)(int LW, int nthreads) = nullptr)
+{
+    static_assert(KH >= S && KW >= S, "filter must be at least the stride");
     FastParams p{};
     p.dX = static_cast<uint16_t*>(a.dX);
     p.filt = static_cast<const uint16_t*>(a.filt);
@@ -455,20 +467,38 @@ FastParams plan_fast(const DwArgs& a)
     p.LW = (p.TX - 1 + KW - 1) / S + 2;
     p.nX = (a.W + p.TX - 1) / p.TX;
     p.nC = (a.C + 31) / 32;
-    // bands: split the rows only as far as needed to fill one wave of resident
-    // CTAs (longer streams amortise the filter load and the pipeline fill, and
-    // every band re-reads (KH-S)/S halo rows); band rows are a multiple of G*S
-    const int nf = Geo::NF;
+    // Bands: band rows are a multiple of G*S.  Each band streams its BH/S dY rows
+    // plus (KH-S)/S rows of halo above it and pays a fixed start (filter taps,
+    // pipeline fill), so a CTA costs about BH/S + (KH-S)/S + 2 dY rows; the CTAs
+    // run in ceil(CTAs / resident slots) waves.  The band count minimises waves
+    // times CTA cost, which avoids a nearly empty last wave.
+    const int nf = G * S;
     const long long base = static_cast<long long>(a.N) * p.nC * p.nX;
-    const int sms = device_sm_count();
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dw_rs_fast_kernel<KH, KW, S, Q, G, kBF16>, 16 * p.nslot,
-                                                      0) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    const long long slots = static_cast<long long>(sms) * per_sm;
-    int nb = static_cast<int>(slots / base);
-    nb = max(1, min(nb, (a.H + nf - 1) / nf));
-    int bh = (a.H + nb - 1) / nb;
+    const int nthreads = 16 * p.nslot;
+    int per_sm = 1;
+    if (kern && smem_of) {
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, nthreads, smem_of(p.LW, nthreads)) ==
+                cudaSuccess &&
+            occ >= 1)
+            per_sm = occ;
+    }
+    const long long slots = static_cast<long long>(device_sm_count()) * per_sm;
+    const int max_nb = kern ? std::min(16, (a.H + nf - 1) / nf) : 1;
+    int nb_best = 1;
+    double cost_best = 0.0;
+    for (int nb = 1; nb <= max_nb; ++nb) {
+        int bh = (a.H + nb - 1) / nb;
+        bh = ((bh + nf - 1) / nf) * nf;
+        const int bands = (a.H + bh - 1) / bh;
+        const long long waves = (base * bands + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) * (static_cast<double>(bh + KH - S) / S + 2.0);
+        if (nb == 1 || cost < cost_best - 1e-9) {
+            cost_best = cost;
+            nb_best = nb;
+        }
+    }
+    int bh = (a.H + nb_best - 1) / nb_best;
     bh = ((bh + nf - 1) / nf) * nf;
     p.BH = bh;
     p.nB = (a.H + bh - 1) / bh;
@@ -479,14 +509,14 @@ template <int KH, int KW, int S, int Q, int G>
 cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
 {
     using Geo = RsGeom<KH, KW, S, Q, G>;
-    const FastParams p = plan_fast<KH, KW, S, Q, G>(a);
+    auto kern = a.f16 ? dw_rs_fast_kernel<KH, KW, S, Q, G, kF16> : dw_rs_fast_kernel<KH, KW, S, Q, G, kBF16>;
+    auto smem_of = [](int lw, int nthreads) { return fast_smem(G, lw, Geo::NC, Q, nthreads); };
+    const FastParams p = plan_fast<KH, KW, S, Q, G>(a, reinterpret_cast<const void*>(kern), smem_of);
     const long long blocks = static_cast<long long>(a.N) * p.nC * p.nX * p.nB;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const int nthreads = 16 * p.nslot;
-    const size_t smem = static_cast<size_t>(kStages) * ((G * p.LW * 64 + 127) & ~127) +
-                        static_cast<size_t>(Geo::NC) * (Q / 2) * nthreads * sizeof(float4) + kStages * 8 + 128;
-    auto kern = a.f16 ? dw_rs_fast_kernel<KH, KW, S, Q, G, kF16> : dw_rs_fast_kernel<KH, KW, S, Q, G, kBF16>;
+    const size_t smem = fast_smem(G, p.LW, Geo::NC, Q, nthreads);
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
@@ -497,13 +527,14 @@ template <int KH, int KW, int S, int Q, int RS, int GT>
 cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
 {
     // plan as the shared-ring kernel with G = GT (band rows a multiple of S*GT)
-    FastParams p = plan_fast<KH, KW, S, Q, GT>(a);
+    auto kern = a.f16 ? dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kF16> : dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kBF16>;
+    auto smem_of = [](int lw, int) { return reg_smem(GT, lw); };
+    FastParams p = plan_fast<KH, KW, S, Q, GT>(a, reinterpret_cast<const void*>(kern), smem_of);
     const long long blocks = static_cast<long long>(a.N) * p.nC * p.nX * p.nB;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
     const int nthreads = 16 * p.nslot;
-    const size_t smem = static_cast<size_t>(kStages) * ((GT * p.LW * 64 + 127) & ~127) + kStages * 8 + 128;
-    auto kern = a.f16 ? dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kF16> : dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kBF16>;
+    const size_t smem = reg_smem(GT, p.LW);
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);

@@ -514,8 +514,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 // word w of a line holds taps (2w - kOff, 2w + 1 - kOff).  f_words words per
 // channel.  One CTA handles one line ry of 32 channels: the taps are read
 // channel-contiguous (coalesced) into shared memory, then each warp writes whole
-// lines.
-__global__ void __launch_bounds__(256)
+// lines.  A line has at most 64 taps, so each thread issues all of its (at most
+// eight) tap loads before the first store: the CTA waits on one memory latency.
+constexpr int kPackThreads = 256;
+constexpr int kPackPer = 64 * 32 / kPackThreads;   // tap loads per thread
+
+__global__ void __launch_bounds__(kPackThreads)
     dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
                           int KY, int KX, int orient, int half_l, int f_words)
 {
@@ -523,12 +527,20 @@ __global__ void __launch_bounds__(256)
     const int ry = blockIdx.y;
     const int c0 = blockIdx.x * 32;
     const unsigned short* w16 = reinterpret_cast<const unsigned short*>(filt);
-    for (int idx = threadIdx.x; idx < KX * 32; idx += blockDim.x) {
+    unsigned short v[kPackPer];
+#pragma unroll
+    for (int k = 0; k < kPackPer; ++k) {
+        const int idx = threadIdx.x + k * kPackThreads;
         const int rx = idx >> 5;
         const int cl = idx & 31;
         const int r = orient ? (KH - 1 - rx) : (KH - 1 - ry);
         const int s = orient ? (KW - 1 - ry) : (KW - 1 - rx);
-        taps[rx][cl] = c0 + cl < C ? w16[(static_cast<int64_t>(r) * KW + s) * C + c0 + cl] : 0;
+        v[k] = (rx < KX && c0 + cl < C) ? w16[(static_cast<int64_t>(r) * KW + s) * C + c0 + cl] : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < kPackPer; ++k) {
+        const int idx = threadIdx.x + k * kPackThreads;
+        if ((idx >> 5) < KX) taps[idx >> 5][idx & 31] = v[k];
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5;
@@ -894,7 +906,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         }
         if (e != cudaSuccess) return e;
         dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
-        dw_filter_pack_kernel<<<fgrid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
+        dw_filter_pack_kernel<<<fgrid, kPackThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
                                                          a.KW, p.KY, p.KX, p.orient, p.half_l, p.f_words);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
