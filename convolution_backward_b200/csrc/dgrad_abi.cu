@@ -77,9 +77,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 2-D bf16 tensor [rows][cols] (cols contiguous), box box_cols x box_rows, 128B swizzle.
+// 2-D 16-bit tensor [rows][cols] (cols contiguous; bf16, or f16 when f16), box
+// box_cols x box_rows, 128B swizzle.
 bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                    uint32_t box_rows)
+                    uint32_t box_rows, bool f16 = false)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -87,7 +88,8 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -259,8 +261,8 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }
 
-// Shared checks for the split-K entry points: pointwise shape class, bf16, the
-// problem extents the kernels index with 32-bit integers.
+// Shared checks for the split-K entry points: pointwise shape class, bf16 or f16,
+// the problem extents the kernels index with 32-bit integers.
 static dgrad_status_t splitk_prepare(const dgrad_problem_t* prob, dgrad_dtype_t dtype, int splits,
                                      dgrad::PwArgs* a, int* sms)
 {
@@ -270,12 +272,12 @@ static dgrad_status_t splitk_prepare(const dgrad_problem_t* prob, dgrad_dtype_t 
     if (s != DGRAD_OK) return s;
     if (prob->KH != 1 || prob->KW != 1 || prob->stride != 1 || prob->pad_h != 0 || pw != 0)
         return DGRAD_ERR_UNSUPPORTED;
-    if (dtype != DGRAD_BF16) return DGRAD_ERR_UNSUPPORTED;
+    if (dtype != DGRAD_BF16 && dtype != DGRAD_F16) return DGRAD_ERR_UNSUPPORTED;
     if (splits < 0 || splits > 64) return DGRAD_ERR_INVALID;
     const int64_t M = prob->N * prob->H * prob->W;
     if (M > 0x7FFFFFFFLL || prob->K > 65536 || prob->C > 65536) return DGRAD_ERR_UNSUPPORTED;
     if ((prob->K * 2) % 16 || (prob->C * 2) % 16) return DGRAD_ERR_ALIGNMENT;
-    *a = dgrad::PwArgs{M, prob->K, prob->C, nullptr, nullptr, nullptr, nullptr};
+    *a = dgrad::PwArgs{M, prob->K, prob->C, nullptr, nullptr, nullptr, nullptr, dtype == DGRAD_F16};
     *sms = 0;
     return DGRAD_OK;
 }
@@ -321,8 +323,8 @@ dgrad_status_t dgrad_pointwise_splitk(const dgrad_problem_t* prob, dgrad_dtype_t
     a.dX = dX;
     a.status = st->status;
     CUtensorMap map_a, map_b;
-    if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), 64, 128) ||
-        !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.C), 64, 64))
+    if (!encode_2d_bf16(&map_a, dY, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), 64, 128, a.f16) ||
+        !encode_2d_bf16(&map_b, W, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.C), 64, 64, a.f16))
         return cuda_fail(cudaErrorInvalidValue);
     cudaError_t e = dgrad::launch_pointwise_tc_splitk(a, map_a, map_b, splits, static_cast<float*>(workspace),
                                                        st->sms, static_cast<cudaStream_t>(stream));

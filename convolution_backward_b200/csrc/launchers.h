@@ -17,6 +17,7 @@ struct PwArgs {
     const void* W;
     void* dX;
     int* status;  // device status word
+    bool f16;     // 16-bit operands are f16 (split-K path; bf16 otherwise)
 };
 
 // fp32 in / fp32 out, fp32 FMA (no reduced-precision tensor-core path).

@@ -738,10 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // split into S contiguous ranges of k-blocks.  Work unit (m-block, n-block,
 // split) computes a partial tile and writes it as fp32 to the workspace
 // ws[split][m][c]; a second kernel sums the S partials in split order
-// (deterministic: no atomics, nothing to zero) and rounds to bf16.  Structure
-// as the streaming kernel: TMA producer, MMA issuer, 4 epilogue warps, two TMEM
-// accumulators.
-template <int BN, int STAGES>
+// (deterministic: no atomics, nothing to zero) and rounds to bf16 (or f16 when
+// F16: f16 operands, the same fp32 partials).  Structure as the streaming
+// kernel: TMA producer, MMA issuer, 4 epilogue warps, two TMEM accumulators.
+template <int BN, int STAGES, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         float* __restrict__ ws, int M, int C, int K, int S, int* status)
@@ -841,7 +841,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
+            constexpr uint32_t idesc = F16 ? idesc_f16_f32(kBM, BN, /*b_mn_major=*/true)
+                                           : idesc_bf16_f32(kBM, BN, /*b_mn_major=*/true);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -944,9 +945,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// dX[m][c] = bf16(sum over s of ws[s][m][c]), s in increasing order; 8 channels per thread.
+// dX[m][c] = round(sum over s of ws[s][m][c]), s in increasing order, rounded once
+// to bf16 (or f16 when F16); 8 channels per thread.
+template <bool F16>
 __global__ void __launch_bounds__(256)
-    splitk_reduce_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ dX, long long MC, int S)
+    splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dX, long long MC, int S)
 {
     const long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
     if (i >= MC) return;
@@ -958,11 +961,12 @@ __global__ void __launch_bounds__(256)
         a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
         b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
     }
+    constexpr int EK = F16 ? kF16 : kBF16;
     uint4 o;
-    o.x = float2_to_bf16x2(a.x, a.y);
-    o.y = float2_to_bf16x2(a.z, a.w);
-    o.z = float2_to_bf16x2(b.x, b.y);
-    o.w = float2_to_bf16x2(b.z, b.w);
+    o.x = float2_to_h16x2<EK>(a.x, a.y);
+    o.y = float2_to_h16x2<EK>(a.z, a.w);
+    o.z = float2_to_h16x2<EK>(b.x, b.y);
+    o.w = float2_to_h16x2<EK>(b.z, b.w);
     *reinterpret_cast<uint4*>(dX + i) = o;
 }
 
@@ -1059,7 +1063,7 @@ cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a
 {
     if (a.M <= 0) return cudaSuccess;
     using L = PwTcLayout<128, 6>;
-    auto kern = pw_tc_splitk_kernel<128, 6>;
+    auto kern = a.f16 ? pw_tc_splitk_kernel<128, 6, true> : pw_tc_splitk_kernel<128, 6, false>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::kAlloc);
     if (e != cudaSuccess) return e;
     const int num_kb = static_cast<int>((a.K + kBK - 1) / kBK);
@@ -1073,8 +1077,9 @@ cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a
     if (e != cudaSuccess) return e;
     const long long MC = a.M * a.C;
     const long long threads = (MC + 7) / 8;
-    splitk_reduce_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-        ws, static_cast<__nv_bfloat16*>(a.dX), MC, S);
+    auto reduce = a.f16 ? splitk_reduce_kernel<true> : splitk_reduce_kernel<false>;
+    reduce<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(ws, static_cast<uint16_t*>(a.dX), MC,
+                                                                             S);
     return cudaGetLastError();
 }
 

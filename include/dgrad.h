@@ -66,10 +66,10 @@ typedef struct {
 } dgrad_problem_t;
 
 /* Element type of dY, W and dX (one type for all three).  DGRAD_F16 is served by
- * dgrad_pointwise, dgrad_dense, dgrad_grouped and dgrad_depthwise_tc (tcgen05
- * f16 operands, fp32 accumulation) and by dgrad_depthwise (f16 widened to fp32
- * on load, fp32 FMAs); dgrad_pointwise_splitk and its scratch variant return
- * DGRAD_ERR_UNSUPPORTED for it. */
+ * every entry point: dgrad_pointwise, its split-K variants, dgrad_dense,
+ * dgrad_grouped and dgrad_depthwise_tc run tcgen05 MMAs on f16 operands with
+ * fp32 accumulation; dgrad_depthwise widens f16 to fp32 on load and uses fp32
+ * FMAs.  DGRAD_F32 is served by dgrad_pointwise and dgrad_depthwise only. */
 typedef enum { DGRAD_F32 = 0, DGRAD_BF16 = 1, DGRAD_F16 = 2 } dgrad_dtype_t;
 
 /* Depthwise kernel choice.  AUTO: rotated-filter for stride 1, row-streaming
@@ -99,8 +99,8 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
  * long K): each 128 x 128 tile's K-loop is split into `splits` ranges that run
  * on different SMs; partial tiles are written as fp32 to `workspace` and then
  * summed in split order (deterministic: no atomics, nothing to zero) and
- * rounded once to bf16 into dX.  Same shape class and layouts as
- * dgrad_pointwise; DGRAD_BF16 only (else DGRAD_ERR_UNSUPPORTED).  The pages'
+ * rounded once to bf16 (or f16) into dX.  Same shape class and layouts as
+ * dgrad_pointwise; DGRAD_BF16 or DGRAD_F16 (else DGRAD_ERR_UNSUPPORTED).  The pages'
  * implicit-GEMM dgrad has a split-K mode ("add the pointwise fast path dgrad
  * was missing", review-fix commit: split-K sub-GEMMs, dX accumulated
  * atomically).

@@ -241,5 +241,10 @@ def test_grouped_validation():
     assert L.dgrad_depthwise(ctypes.byref(dw), F16, 0, FAKE + 8, FAKE, FAKE, None) == ALIGNMENT
     dw0 = cb.Problem(0, 8, 8, 16, 16, 7, 7, 2, 3, 3)
     assert L.dgrad_depthwise(ctypes.byref(dw0), F16, 0, 0, 0, 0, None) == OK
+    # split-K takes bf16 and f16, not f32; f16 is validated like bf16
     pw = cb.Problem(1, 8, 8, 16, 16, 1, 1, 1, 0, 0)
-    assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F16, 0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == UNSUPPORTED
+    assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F32, 0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == UNSUPPORTED
+    assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F16, 0, FAKE, FAKE, FAKE, 0, 1 << 30, None) == INVALID
+    assert L.dgrad_pointwise_splitk(ctypes.byref(pw), F16, 0, FAKE + 8, FAKE, FAKE, FAKE, 1 << 30, None) == ALIGNMENT
+    pw0 = cb.Problem(0, 8, 8, 16, 16, 1, 1, 1, 0, 0)
+    assert L.dgrad_pointwise_splitk(ctypes.byref(pw0), F16, 0, 0, 0, 0, 0, 0, None) == OK

@@ -191,13 +191,16 @@ SPLITK = [
     (P("sk_ragged", "pointwise", "bf16", 1, 7, 9, 136, 1000, seed=92), [3, 16, 0]),
     (P("sk_one_tile", "pointwise", "bf16", 1, 4, 4, 64, 4096, seed=93), [8, 64, 0]),
     (P("sk_k_lt_64", "pointwise", "bf16", 3, 5, 5, 264, 40, seed=94), [1, 0]),
+    (P("sk_f16_small_m", "pointwise", "f16", 2, 14, 14, 512, 2048, seed=95), [2, 0]),
+    (P("sk_f16_ragged", "pointwise", "f16", 1, 7, 9, 136, 1000, seed=96), [3, 0]),
 ]
 SPLITK_CASES = [(p, s) for p, ss in SPLITK for s in ss]
 
 
 @pytest.mark.parametrize("p,splits", SPLITK_CASES, ids=[f"{p.name}-s{s}" for p, s in SPLITK_CASES])
 def test_pointwise_splitk(p, splits):
-    """Split-K tcgen05 pointwise (NEXT-4): partial tiles in a caller workspace, deterministic reduction."""
+    """Split-K tcgen05 pointwise (NEXT-4), bf16 and f16: partial tiles in a caller workspace,
+    deterministic reduction."""
     h = _h()
     import convolution_backward_b200 as cb
     inp = synthetic.make_inputs(p)
