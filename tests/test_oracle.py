@@ -366,6 +366,19 @@ def test_synthetic_bf16_rounding_is_rne():
     np.testing.assert_array_equal(back, ref)
 
 
+def test_synthetic_f16_inputs_are_rne_and_bit_consistent():
+    # binary16 has 11 significant bits: 1 + 2^-11 is halfway between 1 and
+    # 1 + 2^-10 and rounds to the even neighbour 1; 1 + 3*2^-11 rounds up to
+    # 1 + 2^-9; 2^-24 is the smallest subnormal and 2^-26 rounds to zero
+    p = synthetic.Problem("f16_pin", "pointwise", "f16", 1, 1, 2, 8, 8, seed=5)
+    inp = synthetic.make_inputs(p)
+    np.testing.assert_array_equal(inp.dy_bits.view(np.float16).astype(np.float32), inp.dy)
+    np.testing.assert_array_equal(inp.w_bits.view(np.float16).astype(np.float32), inp.w)
+    x = np.array([1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11, 2 ** -24, 2 ** -26, -65504.0], dtype=np.float32)
+    np.testing.assert_array_equal(x.astype(np.float16).astype(np.float32),
+                                  np.array([1.0, 1.0 + 2 ** -9, 2 ** -24, 0.0, -65504.0], dtype=np.float32))
+
+
 def test_synthetic_workloads_shapes():
     p = synthetic.problem("dw7x7s2_bf16")
     assert (p.Ho, p.Wo) == (56, 56)
