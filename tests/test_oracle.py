@@ -4,7 +4,8 @@ Each routine of oracle/ is checked against mathematics, a library routine or a
 hand-worked fixture, chosen so that a dropped term, a wrong sign or index, or a
 transposed operand fails at least one check:
 
-- hand-worked fixtures (tests/golden/*.txt, each citing its passage);
+- hand-worked fixtures (tests/golden/*.txt, each citing its passage), grouped
+  pointwise included;
 - the adjoint identity <conv_fwd(x), dY> = <x, dgrad(dY)> for every geometry
   the workloads use (reduced sizes), grouped and strided ones included;
 - pointwise dgrad equals numpy's matmul of dY[M,K] and W[K,C];
@@ -54,16 +55,23 @@ def test_golden_fixture(name):
         pytest.skip("not a fixture")
     kind, p, a = _read_golden(os.path.join(GOLDEN, name))
     Ho, Wo = oracle.out_dims(p["H"], p["W"], p["KH"], p["KW"], p["S"], p["ph"], p["pw"])
-    K = p["K"] if kind == "pointwise" else p["C"]
+    K = p["C"] if kind == "depthwise" else p["K"]
     dy = a["dY"].reshape(p["N"], Ho, Wo, K)
-    w = a["W"].reshape((K, p["C"]) if kind == "pointwise" else (p["KH"], p["KW"], p["C"]))
+    extra = {}
+    if kind == "pointwise":
+        w = a["W"].reshape(K, p["C"])
+    elif kind == "depthwise":
+        w = a["W"].reshape(p["KH"], p["KW"], p["C"])
+    else:
+        w = a["W"].reshape(K, p["KH"], p["KW"], p["C"] // p["groups"])
+        extra = dict(groups=p["groups"], C=p["C"])
     dx = oracle.dgrad(dy, w, kind=kind, H=p["H"], W=p["W"], KH=p["KH"], KW=p["KW"], S=p["S"],
-                      ph=p["ph"], pw=p["pw"])
+                      ph=p["ph"], pw=p["pw"], **extra)
     np.testing.assert_array_equal(dx.reshape(-1), a["dX"])
     pts = [(n, h, x, c) for n in range(p["N"]) for h in range(p["H"])
            for x in range(p["W"]) for c in range(p["C"])]
     got = oracle.dgrad_points(dy, w, pts, kind=kind, H=p["H"], W=p["W"], KH=p["KH"], KW=p["KW"],
-                              S=p["S"], ph=p["ph"], pw=p["pw"])
+                              S=p["S"], ph=p["ph"], pw=p["pw"], **extra)
     np.testing.assert_array_equal(got, a["dX"])
 
 
