@@ -116,11 +116,33 @@ def _check(status: int, what: str) -> None:
         raise DgradError(status, what, lib().dgrad_last_cuda_error())
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """The raw cudaStream_t of `stream` (default: the current stream of `device`).
+    A given stream must belong to `device`."""
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device} but the tensors are on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _device_of(*ts):
+    """The one CUDA device every tensor in `ts` lives on.  The C ABI works on the
+    current device, so the wrappers make this device current around each call;
+    tensors on different devices are refused."""
+    devs = {(t.device.type, t.device.index) for t in ts}
+    if len(devs) != 1:
+        raise ValueError("all tensors of one call must be on the same CUDA device, got "
+                         + ", ".join(sorted(f"{d[0]}:{d[1]}" for d in devs)))
+    return ts[0].device
+
+
+def _call(dev, what, fn, *args, stream=None):
+    """Run C entry point `fn` with `dev` current and its stream appended."""
+    import torch
+    with torch.cuda.device(dev):
+        _check(fn(*args, _stream_ptr(stream, dev)), what)
 
 
 def _dtype_code(t) -> int:
@@ -167,8 +189,8 @@ def pointwise(dY, W, out=None, stream=None):
         if tuple(out.shape) != (N, H, Wd, C) or out.dtype != dY.dtype:
             raise ValueError("out has the wrong shape or dtype")
     prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
-    _check(lib().dgrad_pointwise(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
-                                 out.data_ptr(), _stream_ptr(stream)), "dgrad_pointwise")
+    _call(_device_of(dY, W, out), "dgrad_pointwise", lib().dgrad_pointwise, ctypes.byref(prob), _dtype_code(dY),
+          dY.data_ptr(), W.data_ptr(), out.data_ptr(), stream=stream)
     return out
 
 
@@ -190,6 +212,8 @@ def pointwise_splitk(dY, W, splits=0, workspace=None, out=None, stream=None):
     _need_cuda(dY, W)
     if dY.dim() != 4 or W.dim() != 2 or W.shape[0] != dY.shape[3]:
         raise ValueError("expected dY (N,H,W,K) and W (K,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
     N, H, Wd, K = dY.shape
     C = W.shape[1]
     nbytes, used = splitk_workspace_bytes(N, H, Wd, K, C, splits)
@@ -198,10 +222,9 @@ def pointwise_splitk(dY, W, splits=0, workspace=None, out=None, stream=None):
     if out is None:
         out = torch.empty((N, H, Wd, C), dtype=dY.dtype, device=dY.device)
     prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
-    _check(lib().dgrad_pointwise_splitk(ctypes.byref(prob), _dtype_code(dY), int(used), dY.data_ptr(),
-                                        W.data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                                        workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "dgrad_pointwise_splitk")
+    _call(_device_of(dY, W, out, workspace), "dgrad_pointwise_splitk", lib().dgrad_pointwise_splitk,
+          ctypes.byref(prob), _dtype_code(dY), int(used), dY.data_ptr(), W.data_ptr(), out.data_ptr(),
+          workspace.data_ptr(), workspace.numel() * workspace.element_size(), stream=stream)
     return out
 
 
@@ -218,14 +241,16 @@ def pointwise_splitk_noalloc(dY, W, out, splits=0, stream=None):
     _need_cuda(dY, W, out)
     if dY.dim() != 4 or W.dim() != 2 or W.shape[0] != dY.shape[3]:
         raise ValueError("expected dY (N,H,W,K) and W (K,C)")
+    if W.dtype != dY.dtype:
+        raise TypeError("dY and W must have the same dtype")
     N, H, Wd, K = dY.shape
     C = W.shape[1]
     if tuple(out.shape) != (N, H, Wd, C) or out.dtype != dY.dtype:
         raise ValueError("out must be (N,H,W,C) with dY's dtype")
     prob = Problem(N, H, Wd, C, K, 1, 1, 1, 0, 0)
-    _check(lib().dgrad_pointwise_splitk_noalloc(ctypes.byref(prob), _dtype_code(dY), int(splits), dY.data_ptr(),
-                                                W.data_ptr(), out.data_ptr(), _stream_ptr(stream)),
-           "dgrad_pointwise_splitk_noalloc")
+    _call(_device_of(dY, W, out), "dgrad_pointwise_splitk_noalloc", lib().dgrad_pointwise_splitk_noalloc,
+          ctypes.byref(prob), _dtype_code(dY), int(splits), dY.data_ptr(), W.data_ptr(), out.data_ptr(),
+          stream=stream)
     return out
 
 
@@ -259,8 +284,8 @@ def depthwise(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, mode="auto",
         _need_cuda(out)
         if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
             raise ValueError("out has the wrong shape or dtype")
-    _check(lib().dgrad_depthwise(ctypes.byref(prob), _dtype_code(dY), DW_MODES[mode], dY.data_ptr(),
-                                 W.data_ptr(), out.data_ptr(), _stream_ptr(stream)), "dgrad_depthwise")
+    _call(_device_of(dY, W, out), "dgrad_depthwise", lib().dgrad_depthwise, ctypes.byref(prob), _dtype_code(dY),
+          DW_MODES[mode], dY.data_ptr(), W.data_ptr(), out.data_ptr(), stream=stream)
     return out
 
 
@@ -289,8 +314,8 @@ def dense(dY, W, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=None, stream
         if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
             raise ValueError("out has the wrong shape or dtype")
     prob = Problem(N, H, W_out, C, K, KH, KW, stride, pad_h, pad_w)
-    _check(lib().dgrad_dense(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(), out.data_ptr(),
-                             _stream_ptr(stream)), "dgrad_dense")
+    _call(_device_of(dY, W, out), "dgrad_dense", lib().dgrad_dense, ctypes.byref(prob), _dtype_code(dY),
+          dY.data_ptr(), W.data_ptr(), out.data_ptr(), stream=stream)
     return out
 
 
@@ -320,8 +345,8 @@ def grouped(dY, W, groups, *, H, W_out=None, stride=1, pad_h=0, pad_w=-1, out=No
         if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
             raise ValueError("out has the wrong shape or dtype")
     prob = Problem(N, H, W_out, C, K, KH, KW, stride, pad_h, pad_w)
-    _check(lib().dgrad_grouped(ctypes.byref(prob), int(groups), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
-                               out.data_ptr(), _stream_ptr(stream)), "dgrad_grouped")
+    _call(_device_of(dY, W, out), "dgrad_grouped", lib().dgrad_grouped, ctypes.byref(prob), int(groups),
+          _dtype_code(dY), dY.data_ptr(), W.data_ptr(), out.data_ptr(), stream=stream)
     return out
 
 
@@ -364,25 +389,30 @@ def depthwise_tc(dY, W, *, H, W_out=None, pad_h=0, pad_w=-1, workspace=None, out
         _need_cuda(out)
         if tuple(out.shape) != (N, H, W_out, C) or out.dtype != dY.dtype:
             raise ValueError("out has the wrong shape or dtype")
-    _check(lib().dgrad_depthwise_tc(ctypes.byref(prob), _dtype_code(dY), dY.data_ptr(), W.data_ptr(),
-                                    out.data_ptr(), workspace.data_ptr(),
-                                    workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "dgrad_depthwise_tc")
+    _call(_device_of(dY, W, out, workspace), "dgrad_depthwise_tc", lib().dgrad_depthwise_tc, ctypes.byref(prob),
+          _dtype_code(dY), dY.data_ptr(), W.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+          workspace.numel() * workspace.element_size(), stream=stream)
     return out
 
 
 def check_status(stream=None) -> None:
     """Synchronise the stream and raise if a kernel reported a timeout (dgrad_check_status)."""
-    _check(lib().dgrad_check_status(_stream_ptr(stream)), "dgrad_check_status")
+    import torch
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib().dgrad_check_status(_stream_ptr(stream, dev)), "dgrad_check_status")
 
 
 def selftest_timeout(limit_cycles: int = 20_000_000, stream=None) -> None:
     """Launch the diagnostic kernel whose bounded wait runs out (dgrad_selftest_timeout)."""
-    _check(lib().dgrad_selftest_timeout(int(limit_cycles), _stream_ptr(stream)), "dgrad_selftest_timeout")
+    import torch
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib().dgrad_selftest_timeout(int(limit_cycles), _stream_ptr(stream, dev)), "dgrad_selftest_timeout")
 
 
 def fma_probe(blocks: int, iters: int, packed: bool, sink, stream=None) -> int:
     """Launch the fp32 FMA-rate probe; returns the FLOP count it performs."""
-    _check(lib().dgrad_fma_probe(int(blocks), int(iters), 1 if packed else 0, sink.data_ptr(),
-                                 _stream_ptr(stream)), "dgrad_fma_probe")
+    _call(_device_of(sink), "dgrad_fma_probe", lib().dgrad_fma_probe, int(blocks), int(iters), 1 if packed else 0,
+          sink.data_ptr(), stream=stream)
     return int(blocks) * 256 * int(iters) * 16 * 2

@@ -144,8 +144,10 @@ dgrad_status_t dgrad_pointwise_splitk_workspace(const dgrad_problem_t* prob, int
  * Nothing in the buffer has to start at zero and nothing clears it: each split
  * writes its whole partial tile before the reduction reads it.
  * Set-up: the first call on each device (with that device current) looks up
- * the buffer's device address and keeps it; make that first call before any
- * stream capture begins.
+ * the buffer's device address and keeps it for the life of the process; make
+ * that first call before any stream capture begins.  The kept address belongs
+ * to the device's primary context: resetting the device (cudaDeviceReset) or
+ * calling from another context is not supported.
  * Races: there is ONE buffer per device.  Calls whose work may overlap on the
  * same device (issued to different streams, or from several host threads
  * without ordering between their streams) write the same buffer and corrupt

@@ -144,6 +144,44 @@ def test_binding_refuses_cpu_tensors():
         cb.depthwise(x, torch.zeros(3, 3, 8, dtype=torch.bfloat16), H=4, Wd=4, pad_h=1)
 
 
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a machine without a GPU: the binding's
+    argument checks only read these attributes before any library call."""
+
+    def __init__(self, shape, dtype, index=0):
+        import torch
+        self.shape = tuple(shape)
+        self.dtype = dtype
+        self.device = torch.device("cuda", index)
+        self.is_cuda = True
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_binding_refuses_tensors_on_two_devices():
+    torch = pytest.importorskip("torch")
+    a = _FakeCuda((1, 4, 4, 8), torch.bfloat16, 0)
+    b = _FakeCuda((8, 8), torch.bfloat16, 1)
+    with pytest.raises(ValueError, match="same CUDA device"):
+        cb._device_of(a, b)
+    assert cb._device_of(a, _FakeCuda((8, 8), torch.bfloat16, 0)) == torch.device("cuda", 0)
+
+
+def test_splitk_wrappers_refuse_mixed_dtypes():
+    torch = pytest.importorskip("torch")
+    dy = _FakeCuda((1, 4, 4, 64), torch.bfloat16)
+    w = _FakeCuda((64, 64), torch.float32)
+    out = _FakeCuda((1, 4, 4, 64), torch.bfloat16)
+    with pytest.raises(TypeError):
+        cb.pointwise_splitk(dy, w, splits=2)
+    with pytest.raises(TypeError):
+        cb.pointwise_splitk_noalloc(dy, w, out, splits=2)
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(cb, "_LIB_PATH", str(tmp_path / "absent.so"))
     monkeypatch.setattr(cb, "_lib", None)

@@ -133,3 +133,22 @@ def test_noalloc_lowers_automatic_splits_to_fit():
     for out in outs:
         assert _normwise(out, ref) <= 1e-2
         assert torch.equal(out, ref)
+
+
+@pytest.mark.gpu
+def test_noalloc_automatic_count_refuses_when_one_split_does_not_fit():
+    """With splits = 0 the count is lowered until the partial tiles fit; when
+    even one split (M * C * 4 bytes) is over the buffer the call is refused and
+    nothing is launched, so dX keeps its contents."""
+    import torch
+    L = cb.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    big = cb.Problem(8, 28, 28, 512, 512, 1, 1, 1, 0, 0)
+    dy = torch.zeros((8, 28, 28, 512), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((512, 512), dtype=torch.bfloat16, device="cuda")
+    out = torch.full((8, 28, 28, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    st = L.dgrad_pointwise_splitk_noalloc(ctypes.byref(big), BF16, 0, dy.data_ptr(), w.data_ptr(), out.data_ptr(),
+                                          stream)
+    assert st == UNSUPPORTED, cb.STATUS.get(st, st)
+    assert L.dgrad_check_status(stream) == OK
+    assert torch.isnan(out.float()).all()
