@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "dgrad.h"
+#include "host_util.h"
 #include "launchers.h"
 
 namespace {
@@ -77,6 +78,60 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
+// Encoded tensor maps, kept per (type, base, extents, strides, box, swizzle):
+// a caller that repeats a call on the same buffers (the common case) reuses the
+// map instead of encoding it again.  A small table with round-robin replacement.
+struct MapKey {
+    int dtype, rank, swizzle, promo;
+    const void* base;
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5];
+    bool operator==(const MapKey& o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+CUresult encode_cached(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, CUtensorMapDataType dtype,
+                       cuuint32_t rank, void* base, const cuuint64_t* dims, const cuuint64_t* strides,
+                       const cuuint32_t* box, const cuuint32_t* estr, CUtensorMapSwizzle swz,
+                       CUtensorMapL2promotion promo)
+{
+    constexpr int kSlots = 128;
+    static MapKey keys[kSlots];
+    static CUtensorMap maps[kSlots];
+    static bool used[kSlots];
+    static int next = 0;
+    static std::mutex mu;
+    MapKey k;
+    memset(&k, 0, sizeof(k));
+    k.dtype = static_cast<int>(dtype);
+    k.rank = static_cast<int>(rank);
+    k.swizzle = static_cast<int>(swz);
+    k.promo = static_cast<int>(promo);
+    k.base = base;
+    for (cuuint32_t i = 0; i < rank && i < 5; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+        if (i + 1 < rank) k.strides[i] = strides[i];
+    }
+    bool unit_estr = true;
+    for (cuuint32_t i = 0; i < rank; ++i) unit_estr = unit_estr && estr[i] == 1;
+    std::lock_guard<std::mutex> lk(mu);
+    if (unit_estr)
+        for (int i = 0; i < kSlots; ++i)
+            if (used[i] && keys[i] == k) {
+                *map = maps[i];
+                return CUDA_SUCCESS;
+            }
+    CUresult r = enc(map, dtype, rank, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r == CUDA_SUCCESS && unit_estr) {
+        keys[next] = k;
+        maps[next] = *map;
+        used[next] = true;
+        next = (next + 1) % kSlots;
+    }
+    return r;
+}
+
 // 2-D 16-bit tensor [rows][cols] (cols contiguous; bf16, or f16 when f16), box
 // box_cols x box_rows, 128B swizzle.
 bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
@@ -88,10 +143,8 @@ bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                     const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode_cached(enc, map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
     return r == CUDA_SUCCESS;
 }
 
@@ -106,10 +159,8 @@ bool encode_nhwc_h16(CUtensorMap* map, const void* base, uint64_t N, uint64_t H,
     const cuuint64_t strides[3] = {C * 2, W * C * 2, H * W * C * 2};
     const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                     const_cast<void*>(base), dims, strides, b, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode_cached(enc, map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                     const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
     return r == CUDA_SUCCESS;
 }
 
@@ -124,9 +175,7 @@ bool encode_planar_bf16(CUtensorMap* map, const void* base, uint64_t X, uint64_t
     const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
     const cuuint32_t b[4] = {64, 8, nr, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = encode_cached(enc, map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
     return r == CUDA_SUCCESS;
 }
 
@@ -142,9 +191,7 @@ bool encode_nhwc_tr(CUtensorMap* map, const void* base, uint64_t N, uint64_t H, 
     const cuuint64_t strides[3] = {C * 2, W * C * 2, H * W * C * 2};
     const cuuint32_t b[4] = {64, orient ? 1u : 64u, orient ? 64u : 1u, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(enc, map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) == CUDA_SUCCESS;
 }
 
 bool encode_planar_tr(CUtensorMap* map, const void* base, uint64_t X, uint64_t N, uint64_t Y, uint64_t C, uint64_t Xs)
@@ -155,16 +202,14 @@ bool encode_planar_tr(CUtensorMap* map, const void* base, uint64_t X, uint64_t N
     const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
     const cuuint32_t b[4] = {64, 1, 1, 64};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(enc, map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int env_int(const char* name, int dflt)
 {
-    const char* v = getenv(name);
+    const char* v = dgrad::tuning_env(name);
     return v && *v ? atoi(v) : dflt;
 }
 
@@ -239,7 +284,7 @@ dgrad_status_t dgrad_pointwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
             return cuda_fail(cudaErrorInvalidValue);
         // Kernel choice: the SM-pair kernel by default (256-column pair tiles when C > 128);
         // DGRAD_PW_MODE = resident | stream selects the one-SM kernels.
-        const char* mode = getenv("DGRAD_PW_MODE");
+        const char* mode = dgrad::tuning_env("DGRAD_PW_MODE");
         const bool want_stream = mode && strcmp(mode, "stream") == 0;
         const bool want_resident = mode && strcmp(mode, "resident") == 0;
         if (!want_stream && !want_resident) {
@@ -385,9 +430,7 @@ dgrad_status_t dgrad_grouped(const dgrad_problem_t* prob, int64_t groups, dgrad_
         const cuuint64_t strides[4] = {static_cast<cuuint64_t>(Kg) * 2, kb, kb * dims[2], kb * dims[2] * dims[3]};
         const cuuint32_t box[5] = {64, 1, 16, 8, 1};
         const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-        if (enc(&map_a, ty, 5, const_cast<void*>(dY), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        if (encode_cached(enc, &map_a, ty, 5, const_cast<void*>(dY), dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
             return cuda_fail(cudaErrorInvalidValue);
     }
     {
@@ -398,9 +441,7 @@ dgrad_status_t dgrad_grouped(const dgrad_problem_t* prob, int64_t groups, dgrad_
         const cuuint64_t strides[3] = {dims[0] * 2, dims[0] * dims[1] * 2, dims[0] * dims[1] * dims[2] * 2};
         const cuuint32_t box[4] = {64, 64, 1, 1};
         const cuuint32_t estr[4] = {1, 1, 1, 1};
-        if (enc(&map_b, ty, 4, const_cast<void*>(W), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        if (encode_cached(enc, &map_b, ty, 4, const_cast<void*>(W), dims, strides, box, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) != CUDA_SUCCESS)
             return cuda_fail(cudaErrorInvalidValue);
     }
     const int bn = env_int("DGRAD_DENSE_BN", Cg <= 64 ? 64 : 128);
@@ -484,7 +525,7 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
         return cuda_fail(cudaErrorInvalidValue);
     // TMA transposes when every map encodes (DGRAD_TC_TRANSPOSE=cuda selects the CUDA-core ones)
     const void* dXp = static_cast<const uint8_t*>(workspace) + plan.ws_in;
-    const char* trm = getenv("DGRAD_TC_TRANSPOSE");
+    const char* trm = dgrad::tuning_env("DGRAD_TC_TRANSPOSE");
     maps.tma_transpose =
         !(trm && strcmp(trm, "cuda") == 0) &&
         encode_nhwc_tr(&maps.pack_src, dY, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.Ho),
@@ -544,7 +585,7 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     unsigned box[4];
-    const char* rk = getenv("DGRAD_ROT_KERNEL");
+    const char* rk = dgrad::tuning_env("DGRAD_ROT_KERNEL");
     const bool force_line = rk && strcmp(rk, "line") == 0;
     if (mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box)) {
         // small filters: one halo tile per CTA

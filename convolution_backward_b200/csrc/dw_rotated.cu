@@ -272,7 +272,7 @@ void plan_tiles(RotParams& p)
     int ns = 1;
     while (ns < need && ns < 16) ns *= 2;
     // DGRAD_ROT_NS caps the strips per CTA (fewer strips, more lines: less fill per output)
-    const char* e = getenv("DGRAD_ROT_NS");
+    const char* e = dgrad::tuning_env("DGRAD_ROT_NS");
     if (e && atoi(e) >= 1 && atoi(e) < ns) ns = atoi(e);
     p.NS = ns;
     p.TB = 16 / ns;
@@ -302,7 +302,7 @@ cudaError_t dispatch_t(RotParams& p, int N, int ek, cudaStream_t stream)
 template <int KAI>
 cudaError_t dispatch(RotParams& p, int N, int ek, cudaStream_t stream)
 {
-    const char* e = getenv("DGRAD_ROT_TAT");
+    const char* e = dgrad::tuning_env("DGRAD_ROT_TAT");
     if (e && atoi(e) == tat_alt<KAI>()) return dispatch_t<KAI, tat_alt<KAI>()>(p, N, ek, stream);
     return dispatch_t<KAI, tat_for<KAI>()>(p, N, ek, stream);
 }

@@ -559,13 +559,13 @@ cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, cudaStream_t str
 
 static bool reg_q4()
 {
-    const char* e = getenv("DGRAD_RS_Q");
+    const char* e = dgrad::tuning_env("DGRAD_RS_Q");
     return e && atoi(e) == 4;
 }
 
 static bool use_reg_ring()
 {
-    const char* e = getenv("DGRAD_RS_KERNEL");
+    const char* e = dgrad::tuning_env("DGRAD_RS_KERNEL");
     return !(e && strcmp(e, "smem") == 0);
 }
 
@@ -583,7 +583,7 @@ static bool use_reg_ring()
 
 static int alt_g()
 {
-    const char* e = getenv("DGRAD_RS_G");
+    const char* e = dgrad::tuning_env("DGRAD_RS_G");
     return e && *e ? atoi(e) : 0;
 }
 

@@ -783,7 +783,7 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
     static const int cand[][3] = {{2, 32, 1}, {2, 16, 1}, {4, 16, 2}, {4, 8, 2}, {8, 8, 4}, {8, 4, 4}};
     // DGRAD_TC_TILE="orient,P,NH,XT" restricts the plan to that shape (testing and tuning).
     int force[4] = {-1, -1, -1, -1};
-    if (const char* ft = getenv("DGRAD_TC_TILE"))
+    if (const char* ft = dgrad::tuning_env("DGRAD_TC_TILE"))
         if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
     ToepPlan best{};

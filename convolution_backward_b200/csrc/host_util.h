@@ -3,10 +3,24 @@
 
 #include <cuda_runtime.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <vector>
 
 namespace dgrad {
+
+// Kernel-selection overrides (DGRAD_PW_MODE, DGRAD_TC_TILE, ...) exist for tests
+// and tuning only.  They are honoured only when DGRAD_TUNING=1 was set the first
+// time the library looked (once per process); otherwise every override reads as
+// unset and the library's own choices stand, whatever else the environment holds.
+inline const char* tuning_env(const char* name)
+{
+    static const bool on = [] {
+        const char* v = getenv("DGRAD_TUNING");
+        return v != nullptr && v[0] == '1';
+    }();
+    return on ? getenv(name) : nullptr;
+}
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), so
 // repeated launches (and launches under stream capture) make no attribute call.
