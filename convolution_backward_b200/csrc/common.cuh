@@ -108,6 +108,17 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     return true;
 }
 
+// Bounded wait on a barrier that other CTAs of the cluster arrive on (with
+// release at cluster scope).  It polls with the plain CTA-scope test and then
+// takes one cluster-scope acquire fence, so the polling loop itself does not
+// carry cluster-scope acquire semantics on every test.
+__device__ __forceinline__ bool mbar_wait_remote(uint64_t* bar, uint32_t parity, const volatile int* abort = nullptr)
+{
+    if (!mbar_wait(bar, parity, abort)) return false;
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+    return true;
+}
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)
@@ -194,6 +205,22 @@ __device__ __forceinline__ void fence_proxy_async_smem()
 __device__ __forceinline__ void named_barrier_sync(int id, int count)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over `count` threads that also ANDs a predicate across them:
+// every participant gets the same answer.
+__device__ __forceinline__ bool named_barrier_and(int id, int count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // ------------------------------------------------------------------- tcgen05
@@ -480,6 +507,101 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
         : "memory");
+}
+
+// ------------------------------------------------- clusters of up to 16 CTAs
+
+// shared::cluster address of the variable at shared::cta address `addr` in the
+// CTA of the cluster with rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// 16-byte store to shared memory anywhere in the cluster.
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Order this thread's generic-proxy writes to shared memory of the cluster
+// before later async-proxy (tcgen05) reads of it.
+__device__ __forceinline__ void fence_proxy_async_cluster()
+{
+    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
+// Arrive once, on the barrier at this shared-memory offset in every CTA of
+// `cta_mask`, when the tcgen05 operations this thread issued so far complete.
+__device__ __forceinline__ void umma_commit_mc(uint64_t* bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// 16-byte global load that bypasses L1 (data other SMs wrote), and a 16-byte store.
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Column c of an 8 x 8 block of 16-bit elements held as eight 16-byte rows
+// (v[e] holds elements (e, 0..7), two per word): elements (0..7, c), two per word.
+__device__ __forceinline__ uint4 transpose8x8_col(const uint4 (&v)[8], int c)
+{
+    const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t lo = (c >> 1) == 0 ? v[2 * p].x : (c >> 1) == 1 ? v[2 * p].y : (c >> 1) == 2 ? v[2 * p].z : v[2 * p].w;
+        const uint32_t hi = (c >> 1) == 0 ? v[2 * p + 1].x : (c >> 1) == 1 ? v[2 * p + 1].y
+                            : (c >> 1) == 2 ? v[2 * p + 1].z : v[2 * p + 1].w;
+        w[p] = __byte_perm(lo, hi, sel);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 8 x 8 transpose of 16-bit elements held as eight 16-byte rows: on entry row e
+// (v[e]) holds elements (e, 0..7), two per word; on exit o[c] holds elements
+// (0..7, c).  Pairs of rows are interleaved with byte permutes, 32 in all.
+__device__ __forceinline__ void transpose8x8_b16(const uint4 (&v)[8], uint4 (&o)[8])
+{
+    uint32_t w[8][4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        w[e][0] = v[e].x;
+        w[e][1] = v[e].y;
+        w[e][2] = v[e].z;
+        w[e][3] = v[e].w;
+    }
+    uint32_t r[8][4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)          // row pair (2p, 2p+1)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {    // word q: columns 2q, 2q+1
+            r[2 * q][p] = __byte_perm(w[2 * p][q], w[2 * p + 1][q], 0x5410);      // column 2q
+            r[2 * q + 1][p] = __byte_perm(w[2 * p][q], w[2 * p + 1][q], 0x7632);  // column 2q+1
+        }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) o[c] = make_uint4(r[c][0], r[c][1], r[c][2], r[c][3]);
 }
 
 // --------------------------------------------------------------- conversions

@@ -459,7 +459,7 @@ dgrad_status_t dgrad_dense(const dgrad_problem_t* prob, dgrad_dtype_t dtype, con
 // bf16, extents within the kernels' 32-bit indexing and grid limits, and a tile
 // plan that fits one SM.
 static dgrad_status_t toeplitz_prepare(const dgrad_problem_t* prob, dgrad_dtype_t dtype, dgrad::DwArgs* a,
-                                       dgrad::ToepPlan* plan)
+                                       dgrad::ToepPlan* plan, bool nhwc)
 {
     int64_t Ho = 0, Wo = 0;
     int pw = 0;
@@ -485,16 +485,18 @@ static dgrad_status_t toeplitz_prepare(const dgrad_problem_t* prob, dgrad_dtype_
     a->pw = pw;
     a->bf16 = dtype == DGRAD_BF16;
     a->f16 = dtype == DGRAD_F16;
-    if (!dgrad::plan_dw_toeplitz(*a, plan)) return DGRAD_ERR_UNSUPPORTED;
+    if (!dgrad::plan_dw_toeplitz(*a, plan, nhwc)) return DGRAD_ERR_UNSUPPORTED;
     return DGRAD_OK;
 }
+
+
 
 dgrad_status_t dgrad_depthwise_tc_workspace(const dgrad_problem_t* prob, size_t* bytes)
 {
     if (!bytes) return DGRAD_ERR_INVALID;
     dgrad::DwArgs a{};
     dgrad::ToepPlan plan{};
-    dgrad_status_t s = toeplitz_prepare(prob, DGRAD_BF16, &a, &plan);
+    dgrad_status_t s = toeplitz_prepare(prob, DGRAD_BF16, &a, &plan, false);
     if (s != DGRAD_OK) return s;
     *bytes = prob->N == 0 ? 0 : plan.ws_in + plan.ws_out + plan.ws_f;
     return DGRAD_OK;
@@ -505,7 +507,7 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
 {
     dgrad::DwArgs a{};
     dgrad::ToepPlan plan{};
-    dgrad_status_t s = toeplitz_prepare(prob, dtype, &a, &plan);
+    dgrad_status_t s = toeplitz_prepare(prob, dtype, &a, &plan, false);
     if (s != DGRAD_OK) return s;
     if (prob->N == 0) return DGRAD_OK;
     if (!dY || !W || !dX || !workspace) return DGRAD_ERR_INVALID;
@@ -551,6 +553,7 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     if (prob->K != prob->C) return DGRAD_ERR_UNSUPPORTED;
     if (prob->KH > 64 || prob->KW > 64) return DGRAD_ERR_UNSUPPORTED;
     if (prob->pad_h > prob->KH - 1 || pw > prob->KW - 1) return DGRAD_ERR_UNSUPPORTED;
+    const bool auto_mode = mode == DGRAD_DW_AUTO;
     if (mode == DGRAD_DW_AUTO) mode = prob->stride == 1 ? DGRAD_DW_ROTATED : DGRAD_DW_ROWSTREAM;
     if (mode == DGRAD_DW_ROTATED && prob->stride != 1) return DGRAD_ERR_UNSUPPORTED;
     if (prob->stride > 8) return DGRAD_ERR_UNSUPPORTED;
@@ -587,6 +590,15 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
     unsigned box[4];
     const char* rk = dgrad::tuning_env("DGRAD_ROT_KERNEL");
     const bool force_line = rk && strcmp(rk, "line") == 0;
+    if (auto_mode && prob->stride == 1 && dtype != DGRAD_F32 && prob->KH * prob->KW > 49) {
+        // Large stride-1 filters in 16-bit: the tensor-core banded-Toeplitz kernel, when
+        // its tile plan fits (else the FP32 kernels below).
+        dgrad::ToepPlan plan{};
+        if (dgrad::plan_dw_toeplitz(a, &plan, true) && (prob->C % 8) == 0) {
+            e = dgrad::launch_dw_toeplitz_nhwc(a, plan, cs);
+            if (e != cudaErrorNotSupported) return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
+        }
+    }
     if (mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box)) {
         // small filters: one halo tile per CTA
         CUtensorMap map;

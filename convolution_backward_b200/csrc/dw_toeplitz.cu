@@ -59,20 +59,20 @@
 #include <cstdlib>
 
 #include "common.cuh"
+#include "toeplitz_core.cuh"
 #include "host_util.h"
 #include "launchers.h"
 
 namespace dgrad {
 namespace {
+using namespace toep;
 
 constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epilogue
-constexpr int kOff = 72;         // offset of filter tap 0 in a padded filter line (>= 64 + 8)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxA = 4;         // A buffers in tensor memory
 constexpr int kMaxB = 2;         // B blocks in shared memory
 constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 5;
 
-__host__ __device__ inline int floor8(int v) { return v >= 0 ? (v & ~7) : -((-v + 7) & ~7); }
 
 struct ToepArgs {
     const uint32_t* fpack;       // padded filter lines, f_words per channel
@@ -104,60 +104,6 @@ __device__ __forceinline__ Unit decode_unit(const ToepArgs& a, int u)
     t.x0 = xt * a.XT * a.TW;
     t.xb = floor8(t.x0 - a.px);
     return t;
-}
-
-// One thread's row of A_i: taps t0 .. t0 + 2*KQ*8 - 1 of a padded filter line
-// (word w holds taps 2w, 2w+1), i.e. KQ*8 words starting at word t0/2, shifted by
-// one tap when t0 is odd; then written to tensor memory 8 columns at a time.
-template <int KQ>
-__device__ __forceinline__ void store_a_row(uint32_t taddr, const uint32_t* src, bool odd, bool nonzero)
-{
-    uint32_t v[KQ * 8 + 1];
-#pragma unroll
-    for (int k = 0; k < KQ * 8 + 1; ++k) v[k] = nonzero ? src[k] : 0u;
-#pragma unroll
-    for (int q = 0; q < KQ; ++q) {
-        uint32_t w[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) w[k] = odd ? __funnelshift_r(v[q * 8 + k], v[q * 8 + k + 1], 16) : v[q * 8 + k];
-        tmem_st_32x32b_x8(taddr + 8u * q, w);
-    }
-}
-
-__device__ __forceinline__ void store_a(int kq, uint32_t taddr, const uint32_t* src, bool odd, bool nonzero)
-{
-    switch (kq) {
-    case 1: store_a_row<1>(taddr, src, odd, nonzero); break;
-    case 2: store_a_row<2>(taddr, src, odd, nonzero); break;
-    case 3: store_a_row<3>(taddr, src, odd, nonzero); break;
-    case 4: store_a_row<4>(taddr, src, odd, nonzero); break;
-    case 5: store_a_row<5>(taddr, src, odd, nonzero); break;
-    case 6: store_a_row<6>(taddr, src, odd, nonzero); break;
-    case 7: store_a_row<7>(taddr, src, odd, nonzero); break;
-    case 8: store_a_row<8>(taddr, src, odd, nonzero); break;
-    default: store_a_row<9>(taddr, src, odd, nonzero); break;
-    }
-}
-
-// The MMAs of one shift step: for each 16-deep step q and sub-tile sx (sub-tiles
-// innermost, so consecutive MMAs go to different accumulators), D_sx += A[:, 16q..]
-// * B columns sx*TW + 16q ... (TW = 64 / XT).  The B descriptor of the step is
-// precomputed; each MMA only adds a constant to it (start address field, units of
-// 16 bytes: one 64-column panel is pb16, 16 columns are 2).
-template <int KQ, int XT>
-__device__ __forceinline__ void issue_step(const uint32_t (&d_tmem)[4], uint32_t a_tmem, uint64_t desc_i,
-                                           uint32_t pb16, uint32_t idesc, bool first)
-{
-    constexpr int TW = 64 / XT;
-#pragma unroll
-    for (int q = 0; q < KQ; ++q) {
-#pragma unroll
-        for (int sx = 0; sx < XT; ++sx) {
-            const int col = sx * TW + 16 * q;
-            const uint64_t bd = desc_i + static_cast<uint64_t>((col >> 6) * pb16 + ((col & 63) >> 4) * 2);
-            umma_f16_ts(d_tmem[sx], a_tmem + 8u * q, bd, idesc, (first && q == 0) ? 0u : 1u);
-        }
-    }
 }
 
 // Shared-memory barriers and addresses the MMA issuer works with.
@@ -769,7 +715,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
-bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
+bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
 {
     if (!(a.bf16 || a.f16) || a.S != 1) return false;
     // Tile shapes (P row phases, NH row groups, XT sub-tiles of 128/P columns), in the
@@ -829,12 +775,15 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out)
             p.panel_bytes = static_cast<uint32_t>(p.NR) * 1024u;
             p.b_bytes = static_cast<uint32_t>(p.npanels) * p.panel_bytes;
             bool fits = false;
-            for (int nbuf = kMaxB; nbuf >= 1 && !fits; --nbuf) {
-                p.NB = nbuf;
-                p.f_off = static_cast<uint32_t>(nbuf) * p.b_bytes;
-                p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.f_words, 16));
+            // The NHWC kernel keeps one B block (the cluster refills it) and two filter
+            // buffers, or one when two do not fit.
+            for (int nbuf = nhwc ? 2 : kMaxB; nbuf >= 1 && !fits; --nbuf) {
+                p.NB = nhwc ? 1 : nbuf;
+                p.nfb = nhwc ? nbuf : 1;
+                p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
+                p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
                 // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
-                p.smem = p.bar_off + kNumBars * 8 + 16 + 1024;
+                p.smem = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16 + 1024;
                 if (p.smem < 120 * 1024) p.smem = 120 * 1024;
                 fits = p.smem <= 227 * 1024;
             }

@@ -105,7 +105,7 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 // swizzle, zero fill.
 struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
-    int P, TW, XT, NH, Ks, NR, NI, NB, npanels, half_l, f_words, a_col0, a_cols, na;
+    int P, TW, XT, NH, Ks, NR, NI, NB, nfb, npanels, half_l, f_words, a_col0, a_cols, na;
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     size_t smem, ws_in, ws_out, ws_f;
 };
@@ -119,7 +119,10 @@ struct ToepMaps {
     CUtensorMap pack_src, pack_dst, unpack_src, unpack_dst;
     bool tma_transpose;
 };
-bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* p);
+bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* p, bool nhwc = false);
+// The same formulation reading NHWC dY and writing NHWC dX directly, with clusters
+// of 8 CTAs (8 channels) and no workspace; p from plan_dw_toeplitz(a, &p, true).
+cudaError_t launch_dw_toeplitz_nhwc(const DwArgs& a, const ToepPlan& p, cudaStream_t stream);
 cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMaps& maps, void* ws, int num_sms,
                                cudaStream_t stream);
 

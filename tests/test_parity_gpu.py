@@ -490,18 +490,65 @@ def test_depthwise_tensor_core_tile_shapes(tile, monkeypatch):
     cb.check_status()
 
 
-TC_FULL = [p for p in synthetic.all_problems() if p.variant == "tc"]
+TC_AUTO = [q for q in TC_SMALL if q.KH * q.KW > 49]
 
 
-@pytest.mark.parametrize("p", TC_FULL, ids=[p.name for p in TC_FULL])
-def test_full_size_tensor_core_depthwise(p):
-    """The large stride-1 workloads through dgrad_depthwise_tc, as the benchmark's tensor-core
-    variant runs them: sampled oracle points, and every element against cuDNN fp32."""
+@pytest.mark.parametrize("p", TC_AUTO, ids=[q.name for q in TC_AUTO])
+def test_depthwise_auto_tensor_core_nhwc(p):
+    """dgrad_depthwise's automatic choice for large 16-bit stride-1 filters: the tensor-core kernel that
+    reads NHWC dY and writes NHWC dX with no workspace (clusters of 8 channels), against the oracle on
+    every element; dX starts as NaN and a second call gives identical bits."""
     h = _h()
     import convolution_backward_b200 as cb
     inp = synthetic.make_inputs(p)
     dy, w = h.to_dev(inp)
-    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    out = torch.full(p.dx_shape, float("nan"), dtype=dy.dtype, device=dy.device)
+    cb.depthwise(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
+    again = cb.depthwise(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    cb.check_status()
+    assert torch.equal(out, again), f"{p.name}: two calls differ"
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/auto")
+
+
+@pytest.mark.parametrize("tile", TC_TILES)
+def test_depthwise_auto_tensor_core_tile_shapes(tile, monkeypatch):
+    """Every tile shape of the NHWC tensor-core kernel behind dgrad_depthwise (forced through
+    DGRAD_TC_TILE) on a ragged problem: N = 9 (a partial image group), odd extents (a ragged last
+    8-column group), several row tiles for the smaller shapes."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_TILE", tile)
+    p = P("tc_tile_auto", "depthwise", "bf16", 9, 37, 41, 24, 24, 9, 7, 1, 4, 3, seed=160)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = cb.depthwise(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"auto tile {tile}")
+    cb.check_status()
+
+
+TC_FULL = [p for p in synthetic.all_problems() if p.variant == "tc"]
+
+
+@pytest.mark.parametrize("entry", ["tc", "auto"])
+@pytest.mark.parametrize("p", TC_FULL, ids=[p.name for p in TC_FULL])
+def test_full_size_tensor_core_depthwise(p, entry):
+    """The large stride-1 workloads through dgrad_depthwise_tc (planar, with a workspace: what the
+    benchmark runs) and through dgrad_depthwise's automatic choice (NHWC, no workspace): sampled
+    oracle points, and every element against cuDNN fp32."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    if entry == "tc":
+        out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    else:
+        out = cb.depthwise(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
     torch.cuda.synchronize()
     pts = h.sample_points(p, 3000)
     got = out.float()[pts[:, 0], pts[:, 1], pts[:, 2], pts[:, 3]].cpu().numpy().astype(np.float64)
