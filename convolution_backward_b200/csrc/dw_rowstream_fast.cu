@@ -282,14 +282,14 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
     for (int k = 0; k < GT; ++k) {
         float2 nx[Q + NT - 1];
         if (k + 1 < GT) load_row(k + 1, nx);
-        // Filter rows in order r = 0 .. KH-1: rows 0 .. S-1 are the ones that become
-        // final after this dY row, so their last FMAs are issued first.  Rows
-        // r >= KH-S are touched for the first time (their slot was flushed earlier),
-        // so their first tap is a multiply, not an add onto a cleared slot.
+        // Taps outermost: consecutive FMAs go to the KH * Q different accumulators,
+        // so no FMA waits on the one just before it.  Rows r >= KH-S are touched
+        // for the first time (their slot was flushed earlier), so their first tap
+        // is a multiply, not an add onto a cleared slot.
 #pragma unroll
-        for (int r = 0; r < KH; ++r)
+        for (int i = 0; i < NT; ++i)
 #pragma unroll
-            for (int i = 0; i < NT; ++i)
+            for (int r = 0; r < KH; ++r)
 #pragma unroll
                 for (int q = 0; q < Q; ++q) {
                     float2& a = acc[(S * k + r) % RS][q];
