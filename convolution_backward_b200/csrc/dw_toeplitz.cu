@@ -465,13 +465,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 constexpr int kPackThreads = 256;
 constexpr int kPackPer = 64 * 32 / kPackThreads;   // tap loads per thread
 
-__global__ void __launch_bounds__(kPackThreads)
-    dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
-                          int KY, int KX, int orient, int half_l, int f_words)
+__device__ __forceinline__ void pack_filter_block(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst,
+                                                  int C, int KH, int KW, int KY, int KX, int orient, int half_l,
+                                                  int f_words, int bx, int ry)
 {
     __shared__ uint16_t taps[64][34];   // [rx][channel]
-    const int ry = blockIdx.y;
-    const int c0 = blockIdx.x * 32;
+    const int c0 = bx * 32;
     const unsigned short* w16 = reinterpret_cast<const unsigned short*>(filt);
     unsigned short v[kPackPer];
 #pragma unroll
@@ -504,6 +503,13 @@ __global__ void __launch_bounds__(kPackThreads)
         if (ry == KY - 1)   // zero the words that round the channel's block up to f_words
             for (int w = KY * half_l + lane; w < f_words; w += 32) dst[static_cast<int64_t>(c) * f_words + w] = 0u;
     }
+}
+
+__global__ void __launch_bounds__(kPackThreads)
+    dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
+                          int KY, int KX, int orient, int half_l, int f_words)
+{
+    pack_filter_block(filt, dst, C, KH, KW, KY, KX, orient, half_l, f_words, blockIdx.x, blockIdx.y);
 }
 
 // NHWC <-> planar [C][Y][N][Xs] for bf16.  The NHWC side addresses element
@@ -605,6 +611,10 @@ constexpr int kTrStages = 4;
 struct TrArgs {
     int to_planar, orient, N, Y, nxb, ncb, ntiles;
     int* status;
+    int grid_tr;   // CTAs that transpose; CTAs past them pack filter lines (dY launch only)
+    const __nv_bfloat16* filt;
+    uint32_t* fpk;
+    int C, KH, KW, KY, KX, half_l, f_words, pack_ncb;
 };
 
 __device__ __forceinline__ void tr_coords(const TrArgs& a, int t, bool nhwc_side, int (&c)[4])
@@ -632,6 +642,12 @@ __global__ void __launch_bounds__(256)
     dw_transpose_tma_kernel(const __grid_constant__ CUtensorMap src_map, const __grid_constant__ CUtensorMap dst_map,
                             const __grid_constant__ TrArgs a)
 {
+    if (static_cast<int>(blockIdx.x) >= a.grid_tr) {   // the filter-packing CTAs of the dY launch
+        const int b = static_cast<int>(blockIdx.x) - a.grid_tr;
+        pack_filter_block(a.filt, a.fpk, a.C, a.KH, a.KW, a.KY, a.KX, a.orient, a.half_l, a.f_words, b % a.pack_ncb,
+                          b / a.pack_ncb);
+        return;
+    }
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -652,7 +668,7 @@ __global__ void __launch_bounds__(256)
         tma_prefetch_desc(&src_map);
         tma_prefetch_desc(&dst_map);
         for (int s = 0; s < kTrStages; ++s) {
-            const int t = blockIdx.x + s * gridDim.x;
+            const int t = static_cast<int>(blockIdx.x) + s * a.grid_tr;
             if (t >= a.ntiles) break;
             int c[4];
             tr_coords(a, t, src_nhwc, c);
@@ -663,7 +679,7 @@ __global__ void __launch_bounds__(256)
     }
     bool aborted = false;
     int k = 0;
-    for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++k) {
+    for (int t = blockIdx.x; t < a.ntiles; t += a.grid_tr, ++k) {
         const int s = k % kTrStages;
         const int o = k & 1;
         const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((k / kTrStages) & 1));
@@ -694,7 +710,7 @@ __global__ void __launch_bounds__(256)
             tr_coords(a, t, !src_nhwc, c);
             tma_store_4d(&dst_map, out_t + o * 8192, c[0], c[1], c[2], c[3]);
             bulk_commit_group();
-            const int tn = t + kTrStages * gridDim.x;
+            const int tn = t + kTrStages * a.grid_tr;
             if (tn < a.ntiles) {
                 tr_coords(a, tn, src_nhwc, c);
                 mbar_arrive_expect_tx(&full[s], 8192);
@@ -818,7 +834,10 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_transpose_tma_kernel), tr_smem);
         if (e != cudaSuccess) return e;
     }
-    auto tma_transpose = [&](const CUtensorMap& src, const CUtensorMap& dst, bool to_planar, int Y, int X) {
+    static_assert(kPackThreads == 256, "the filter-packing CTAs share the transpose launch's block size");
+    // with pack_to set, CTAs past the transposing ones pack the filter lines into it
+    auto tma_transpose = [&](const CUtensorMap& src, const CUtensorMap& dst, bool to_planar, int Y, int X,
+                             uint32_t* pack_to) {
         TrArgs t{};
         t.to_planar = to_planar ? 1 : 0;
         t.orient = p.orient;
@@ -829,7 +848,22 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.ntiles = a.N * Y * t.nxb * t.ncb;
         t.status = a.status;
         const int grid = t.ntiles < 4 * num_sms ? t.ntiles : 4 * num_sms;   // four CTAs per SM
-        dw_transpose_tma_kernel<<<grid, 256, tr_smem, stream>>>(src, dst, t);
+        t.grid_tr = grid;
+        int pack_blocks = 0;
+        if (pack_to) {
+            t.filt = static_cast<const __nv_bfloat16*>(a.filt);
+            t.fpk = pack_to;
+            t.C = a.C;
+            t.KH = a.KH;
+            t.KW = a.KW;
+            t.KY = p.KY;
+            t.KX = p.KX;
+            t.half_l = p.half_l;
+            t.f_words = p.f_words;
+            t.pack_ncb = (a.C + 31) / 32;
+            pack_blocks = t.pack_ncb * p.KY;
+        }
+        dw_transpose_tma_kernel<<<grid + pack_blocks, 256, tr_smem, stream>>>(src, dst, t);
         return cudaGetLastError();
     };
     if (a.N <= 0) return cudaSuccess;
@@ -845,19 +879,20 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         const int64_t sX = p.orient ? static_cast<int64_t>(a.Wo) * C : C;
         cudaError_t e;
         if (maps.tma_transpose) {
-            e = tma_transpose(maps.pack_src, maps.pack_dst, true, p.Yi, p.Xi);
+            e = tma_transpose(maps.pack_src, maps.pack_dst, true, p.Yi, p.Xi, fpk);   // packs the filters too
         } else {
             dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct),
                       static_cast<unsigned>((p.Yi + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
             dw_transpose_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N,
                                                                 p.Yi, p.Xi, p.Xsi, a.C, sN, sY, sX);
             e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
+            dw_filter_pack_kernel<<<fgrid, kPackThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk,
+                                                                    a.C, a.KH, a.KW, p.KY, p.KX, p.orient, p.half_l,
+                                                                    p.f_words);
+            e = cudaGetLastError();
         }
-        if (e != cudaSuccess) return e;
-        dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
-        dw_filter_pack_kernel<<<fgrid, kPackThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk, a.C, a.KH,
-                                                         a.KW, p.KY, p.KX, p.orient, p.half_l, p.f_words);
-        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     {
@@ -912,7 +947,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         const int64_t sY = p.orient ? C : static_cast<int64_t>(a.W) * C;
         const int64_t sX = p.orient ? static_cast<int64_t>(a.W) * C : C;
         if (maps.tma_transpose) {
-            cudaError_t e = tma_transpose(maps.unpack_src, maps.unpack_dst, false, p.Yo, p.Xo);
+            cudaError_t e = tma_transpose(maps.unpack_src, maps.unpack_dst, false, p.Yo, p.Xo, nullptr);
             if (e != cudaSuccess) return e;
         } else {
             dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct),
