@@ -32,6 +32,16 @@ __device__ __forceinline__ void report_timeout(int* status)
     if (status) atomicExch(status, DEV_TIMEOUT);
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Every kernel is launched so that it may start while the kernel before it on
+// the stream is finishing.  pdl_wait() blocks until that kernel has completed
+// and its memory is visible; a kernel calls it before its first access to
+// global memory, so only set-up (barriers, tensor memory, descriptor
+// prefetch) overlaps.  pdl_trigger() lets the next kernel start once every CTA
+// of this one has called it or exited.  Both are no-ops without a dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     dense_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ DenseArgs d)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using L = DenseLayout<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -320,7 +322,11 @@ cudaError_t launch_dense_bn(DenseArgs d, const CUtensorMap& map_a, const CUtenso
     d.num_tiles = static_cast<int>(tiles);
     if (d.num_tiles == 0) return cudaSuccess;
     const int grid = d.num_tiles < num_sms ? d.num_tiles : num_sms;
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, d);
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, 1,
+                                             map_a, map_b, d);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 

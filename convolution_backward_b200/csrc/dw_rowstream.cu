@@ -77,6 +77,8 @@ template <int EK>
 __global__ void __launch_bounds__(kThreads)
     dw_rowstream_kernel(const RsParams p)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using Ch = RsChunk<EK>;
     using T = typename std::conditional<EK == kF32, float, uint16_t>::type;
     extern __shared__ float2 sm2[];
@@ -220,7 +222,11 @@ cudaError_t launch_t(const RsParams& p, long long blocks, size_t smem, cudaStrea
     auto kern = dw_rowstream_kernel<EK>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(p);
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), smem, stream, 1,
+                                             p);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 

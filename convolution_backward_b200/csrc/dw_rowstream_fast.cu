@@ -96,6 +96,8 @@ template <int KH, int KW, int S, int Q, int G, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_fast_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using Geo = RsGeom<KH, KW, S, Q, G>;
     constexpr int RB = Geo::RB, NF = Geo::NF, NC = Geo::NC, NTMAX = Geo::NTMAX;
     extern __shared__ uint8_t smem_raw[];
@@ -322,6 +324,8 @@ template <int KH, int KW, int S, int Q, int RS, int GT, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_reg_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     constexpr int NTMAX = (KW + S - 1) / S;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -519,7 +523,11 @@ cudaError_t launch_fast(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     const size_t smem = fast_smem(G, p.LW, Geo::NC, Q, nthreads);
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(nthreads), smem, stream, 1,
+                                             map, p);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 
@@ -537,7 +545,11 @@ cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, cudaStream_t str
     const size_t smem = reg_smem(GT, p.LW);
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(blocks), nthreads, smem, stream>>>(map, p);
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(nthreads), smem, stream, 1,
+                                             map, p);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 

@@ -37,6 +37,8 @@ template <int KH, int KW, int R, int TAT, int EK>
 __global__ void __launch_bounds__(256)
     dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const TileParams p)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
@@ -182,7 +184,11 @@ cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     auto kern = a.f16 ? dw_tile_kernel<KH, KW, R, TAT, kF16> : dw_tile_kernel<KH, KW, R, TAT, kBF16>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(blocks), 16 * p.CS * p.RS, smem, stream>>>(map, p);
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(16 * p.CS * p.RS), smem, stream, 1,
+                                             map, p);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 

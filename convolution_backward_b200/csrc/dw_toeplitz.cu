@@ -45,6 +45,12 @@
 // padded filter lines of every channel, and dw_transpose_kernel writes the planar
 // output of the MMA epilogue back to NHWC dX.
 //
+// Launch order.  Like every kernel here, these wait for the kernel before them
+// (griddepcontrol.wait) before touching global memory.  Unlike the others, they
+// do not let the next kernel start early: the MMA kernel and a transpose fit on
+// one SM together, and a transpose CTA waiting next to the MMA kernel slowed
+// the 51x5 problem by 6% (measured), while the early start saved nothing here.
+//
 // Roles (448 threads, one CTA per SM, a contiguous range of tiles per CTA so
 // that the image groups of one channel follow each other):
 //   warp 0      producer: filter lines (bulk copy) and B panels (TMA)
@@ -196,6 +202,7 @@ __device__ __forceinline__ void unit_range(const ToepArgs& a, int* u_begin, int*
 __global__ void __launch_bounds__(kThreadsT, 1)
     dw_toeplitz_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ ToepArgs a)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -509,6 +516,7 @@ __global__ void __launch_bounds__(kPackThreads)
     dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
                           int KY, int KX, int orient, int half_l, int f_words)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
     pack_filter_block(filt, dst, C, KH, KW, KY, KX, orient, half_l, f_words, blockIdx.x, blockIdx.y);
 }
 
@@ -526,6 +534,7 @@ __global__ void __launch_bounds__(256)
     dw_transpose_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int N, int Y, int X,
                         int Xs, int C, int64_t sN, int64_t sY, int64_t sX)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
     __shared__ uint32_t tile[64][33];   // [row][pair]: rows are x (to planar) or c (from planar)
     const int nct = (C + 63) >> 6;
     const int ct = blockIdx.x % nct;
@@ -642,6 +651,7 @@ __global__ void __launch_bounds__(256)
     dw_transpose_tma_kernel(const __grid_constant__ CUtensorMap src_map, const __grid_constant__ CUtensorMap dst_map,
                             const __grid_constant__ TrArgs a)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
     if (static_cast<int>(blockIdx.x) >= a.grid_tr) {   // the filter-packing CTAs of the dY launch
         const int b = static_cast<int>(blockIdx.x) - a.grid_tr;
         pack_filter_block(a.filt, a.fpk, a.C, a.KH, a.KW, a.KY, a.KX, a.orient, a.half_l, a.f_words, b % a.pack_ncb,
@@ -863,7 +873,11 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
             t.pack_ncb = (a.C + 31) / 32;
             pack_blocks = t.pack_ncb * p.KY;
         }
-        dw_transpose_tma_kernel<<<grid + pack_blocks, 256, tr_smem, stream>>>(src, dst, t);
+        {
+            const cudaError_t le_ = launch_kernel(dw_transpose_tma_kernel, dim3(grid + pack_blocks), dim3(256), tr_smem, stream, 1,
+                                                 src, dst, t);
+            if (le_ != cudaSuccess) return le_;
+        }
         return cudaGetLastError();
     };
     if (a.N <= 0) return cudaSuccess;
@@ -883,14 +897,22 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         } else {
             dim3 grid(static_cast<unsigned>(((p.Xi + 63) / 64) * nct),
                       static_cast<unsigned>((p.Yi + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
-            dw_transpose_kernel<true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N,
+            {
+                const cudaError_t le_ = launch_kernel(dw_transpose_kernel<true>, dim3(grid), dim3(256), 0, stream, 1,
+                                                     static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N,
                                                                 p.Yi, p.Xi, p.Xsi, a.C, sN, sY, sX);
+                if (le_ != cudaSuccess) return le_;
+            }
             e = cudaGetLastError();
             if (e != cudaSuccess) return e;
             dim3 fgrid(static_cast<unsigned>((a.C + 31) / 32), static_cast<unsigned>(p.KY));
-            dw_filter_pack_kernel<<<fgrid, kPackThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.filt), fpk,
+            {
+                const cudaError_t le_ = launch_kernel(dw_filter_pack_kernel, dim3(fgrid), dim3(kPackThreads), 0, stream, 1,
+                                                     static_cast<const __nv_bfloat16*>(a.filt), fpk,
                                                                     a.C, a.KH, a.KW, p.KY, p.KX, p.orient, p.half_l,
                                                                     p.f_words);
+                if (le_ != cudaSuccess) return le_;
+            }
             e = cudaGetLastError();
         }
         if (e != cudaSuccess) return e;
@@ -937,7 +959,11 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));
         if (e != cudaSuccess) return e;
         const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-        dw_toeplitz_kernel<<<grid, kThreadsT, p.smem, stream>>>(map_b, t);
+        {
+            const cudaError_t le_ = launch_kernel(dw_toeplitz_kernel, dim3(grid), dim3(kThreadsT), p.smem, stream, 1,
+                                                 map_b, t);
+            if (le_ != cudaSuccess) return le_;
+        }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -952,8 +978,12 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         } else {
             dim3 grid(static_cast<unsigned>(((p.Xo + 63) / 64) * nct),
                       static_cast<unsigned>((p.Yo + kRowsPerCta - 1) / kRowsPerCta), static_cast<unsigned>(a.N));
-            dw_transpose_kernel<false><<<grid, 256, 0, stream>>>(dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo,
+            {
+                const cudaError_t le_ = launch_kernel(dw_transpose_kernel<false>, dim3(grid), dim3(256), 0, stream, 1,
+                                                     dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo,
                                                                  p.Xo, p.Xso, a.C, sN, sY, sX);
+                if (le_ != cudaSuccess) return le_;
+            }
         }
     }
     return cudaGetLastError();

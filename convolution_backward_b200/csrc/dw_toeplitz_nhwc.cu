@@ -563,6 +563,7 @@ __device__ __forceinline__ void ec_role(const ToepNArgs& a, const KCtx& k, int w
 __global__ void __launch_bounds__(kThreadsN, 1)
     dw_toeplitz_nhwc_kernel(const __grid_constant__ ToepNArgs a)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -785,19 +786,8 @@ cudaError_t launch_dw_toeplitz_nhwc(const DwArgs& a, const ToepPlan& p, cudaStre
     const int ncl_max = max_active_clusters(p.smem);
     if (ncl_max < 1) return cudaErrorNotSupported;
     const int ncl = static_cast<int>(nsu < ncl_max ? nsu : ncl_max);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ncl * kCluster));
-    cfg.blockDim = dim3(kThreadsN);
-    cfg.dynamicSmemBytes = p.smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = kCluster;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, dw_toeplitz_nhwc_kernel, t);
+    e = launch_kernel(dw_toeplitz_nhwc_kernel, dim3(static_cast<unsigned>(ncl * kCluster)), dim3(kThreadsN), p.smem,
+                      stream, kCluster, t);
     return e;
 }
 

@@ -5,6 +5,7 @@
 
 #include <cstdlib>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 namespace dgrad {
@@ -48,6 +49,36 @@ inline cudaError_t ensure_smem_limit(const void* kernel, int bytes)
         }
     done.push_back({kernel, dev, bytes});
     return cudaSuccess;
+}
+
+// Launch `kernel` on `stream` with programmatic stream serialisation (it may
+// begin while the previous kernel on the stream finishes; the kernel itself
+// waits for it with griddepcontrol.wait before touching global memory) and,
+// when cluster_x > 1, clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 int cluster_x, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    int n = 0;
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        at[n].id = cudaLaunchAttributeClusterDimension;
+        at[n].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        at[n].val.clusterDim.y = 1;
+        at[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = at;
+    cfg.numAttrs = static_cast<unsigned>(n);
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace dgrad

@@ -10,6 +10,7 @@
 // short K (the small problems this kernel serves) costs one memory latency.
 // Requires K % 4 == 0 and C % 4 == 0 (16-byte rows), checked by the caller.
 #include "common.cuh"
+#include "host_util.h"
 #include "launchers.h"
 
 namespace dgrad {
@@ -23,6 +24,8 @@ __global__ void __launch_bounds__(kThreads)
     pw_f32_kernel(const float* __restrict__ dY, const float* __restrict__ W, float* __restrict__ dX, int M,
                   int K, int C)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     __shared__ __align__(16) float As[kTK][kTM + 4];   // dY slice, stored k-major (rows of 272 bytes)
     __shared__ __align__(16) float Bs[kTK][kTC];       // W slice
     const int tid = threadIdx.x;
@@ -93,9 +96,13 @@ cudaError_t launch_pointwise_f32(const PwArgs& a, cudaStream_t stream)
 {
     if (a.M <= 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>((a.M + kTM - 1) / kTM), static_cast<unsigned>((a.C + kTC - 1) / kTC));
-    pw_f32_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const float*>(a.dY), static_cast<const float*>(a.W),
+    {
+        const cudaError_t le_ = launch_kernel(pw_f32_kernel, dim3(grid), dim3(kThreads), 0, stream, 1,
+                                             static_cast<const float*>(a.dY), static_cast<const float*>(a.W),
                                             static_cast<float*>(a.dX), static_cast<int>(a.M),
                                             static_cast<int>(a.K), static_cast<int>(a.C));
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 

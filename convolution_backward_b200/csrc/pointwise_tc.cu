@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                  __nv_bfloat16* __restrict__ dX, int M, int C, int K, int* status)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using L = PwTcLayout<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -280,6 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_res_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const __grid_constant__ CUtensorMap map_d, int M, int C, int K, int* status)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using L = PwResLayout;
     constexpr int BN = 128;
     extern __shared__ uint8_t smem_raw[];
@@ -525,6 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_d, int M, int C, int K, int* status)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using L = PwPairLayout<BN, STAGES>;
     constexpr int kPairStages = STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -746,6 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         float* __restrict__ ws, int M, int C, int K, int S, int* status)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     using L = PwTcLayout<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -951,6 +959,8 @@ template <bool F16>
 __global__ void __launch_bounds__(256)
     splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dX, long long MC, int S)
 {
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     const long long i = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
     if (i >= MC) return;
     float4 a = *reinterpret_cast<const float4*>(ws + i);
@@ -981,9 +991,13 @@ cudaError_t launch_bn(const PwArgs& a, const CUtensorMap& map_a, const CUtensorM
     if (e != cudaSuccess) return e;
     const int num_tiles = static_cast<int>(((a.M + kBM - 1) / kBM) * ((a.C + BN - 1) / BN));
     const int grid = num_tiles < num_sms ? num_tiles : num_sms;
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, static_cast<__nv_bfloat16*>(a.dX),
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, 1,
+                                             map_a, map_b, static_cast<__nv_bfloat16*>(a.dX),
                                                  static_cast<int>(a.M), static_cast<int>(a.C),
                                                  static_cast<int>(a.K), a.status);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 
@@ -999,9 +1013,13 @@ cudaError_t launch_res(const PwArgs& a, const CUtensorMap& map_a, const CUtensor
     int per_n = num_sms / num_n;
     if (per_n > num_m) per_n = num_m;
     const int grid = per_n * num_n;
-    pw_tc_res_kernel<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, map_d, static_cast<int>(a.M),
+    {
+        const cudaError_t le_ = launch_kernel(pw_tc_res_kernel, dim3(grid), dim3(kThreads), L::kAlloc, stream, 1,
+                                             map_a, map_b, map_d, static_cast<int>(a.M),
                                                             static_cast<int>(a.C), static_cast<int>(a.K),
                                                             a.status);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 
@@ -1035,9 +1053,8 @@ cudaError_t launch_pair(const PwArgs& a, const CUtensorMap& map_a, const CUtenso
         max_clusters = n;
     }
     int pairs = max_clusters < num_tiles ? max_clusters : num_tiles;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    return cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_d, static_cast<int>(a.M),
-                              static_cast<int>(a.C), static_cast<int>(a.K), a.status);
+    return launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), L::kAlloc, stream, 2, map_a,
+                         map_b, map_d, static_cast<int>(a.M), static_cast<int>(a.C), static_cast<int>(a.K), a.status);
 }
 
 }  // namespace
@@ -1071,15 +1088,23 @@ cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a
     const int S = (num_kb + kb_per - 1) / kb_per;   // no empty split
     const long long units = ((a.M + kBM - 1) / kBM) * ((a.C + 127) / 128) * S;
     const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(map_a, map_b, ws, static_cast<int>(a.M), static_cast<int>(a.C),
+    {
+        const cudaError_t le_ = launch_kernel(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, 1,
+                                             map_a, map_b, ws, static_cast<int>(a.M), static_cast<int>(a.C),
                                                 static_cast<int>(a.K), S, a.status);
+        if (le_ != cudaSuccess) return le_;
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long MC = a.M * a.C;
     const long long threads = (MC + 7) / 8;
     auto reduce = a.f16 ? splitk_reduce_kernel<true> : splitk_reduce_kernel<false>;
-    reduce<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(ws, static_cast<uint16_t*>(a.dX), MC,
+    {
+        const cudaError_t le_ = launch_kernel(reduce, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, stream, 1,
+                                             ws, static_cast<uint16_t*>(a.dX), MC,
                                                                              S);
+        if (le_ != cudaSuccess) return le_;
+    }
     return cudaGetLastError();
 }
 
