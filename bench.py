@@ -40,6 +40,7 @@ METRIC = "dgrad effective TFLOP/s and HBM GB/s on 1 B200, % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 FP32_LANES_PER_SM = 128
+KERN_REPS = 10   # separately timed replays per kernel graph; the median is reported
 
 
 def load_peaks():
@@ -231,13 +232,47 @@ def describe_plan(plan):
 
 
 def cpu_baseline(problems, inputs, budget_s=15.0):
+    """The oracle on the host cores over a bounded sample: the suite rate, the
+    rate of each problem, and (on a smaller sample) the rate of one thread."""
+    import oracle
     plan, threads = oracle_sample_plan(problems, inputs, budget_s)
-    flops, secs = run_oracle_sample(plan, inputs)
+    flops, secs = 0, 0.0
+    per_problem = []
+    for item in plan:
+        f, t = run_oracle_sample([item], inputs)
+        flops += f
+        secs += t
+        per_problem.append({"problem": item[0].name, "tflops": round(f / t / 1e12, 6), "seconds": round(t, 3)})
+    # one thread: the same problems on a sample `threads` times smaller (one image, or 1/threads of the rows)
+    small = []
+    for p, n, c in plan:
+        if p.kind == "pointwise":
+            small.append((p, n, max(1, c // threads)))
+        else:
+            small.append((p, 1, c))
+    oracle.set_threads(1)
+    try:
+        f1, t1 = run_oracle_sample(small, inputs)
+    finally:
+        oracle.set_threads(threads)
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": describe_plan(plan), "seconds": round(secs, 3), "flops": flops}
+            "sample": describe_plan(plan), "seconds": round(secs, 3), "flops": flops,
+            "per_problem": per_problem,
+            "single_thread": {"value": round(f1 / t1 / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                              "sample": describe_plan(small), "seconds": round(t1, 3)}}
 
 
 # ---------------------------------------------------------------------- ours
+
+def inbounds_flops(p) -> int:
+    """FLOPs of the taps that land inside dX (zero padding skipped): the nominal
+    count is 2*N*Ho*Wo*K*(C/groups)*KH*KW, padded taps included; here each of the
+    two spatial axes counts only the (output, tap) pairs whose dX position
+    ho*S - pad + r lies in [0, H) (and likewise for columns)."""
+    rows = sum(1 for ho in range(p.Ho) for r in range(p.KH) if 0 <= ho * p.stride - p.pad_h + r < p.H)
+    cols = sum(1 for wo in range(p.Wo) for s in range(p.KW) if 0 <= wo * p.stride - p.pad_w + s < p.W)
+    return 2 * p.N * rows * cols * p.K * (p.C // p.groups)
+
 
 def traffic_record():
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
@@ -354,6 +389,7 @@ def run_ours(args, world, rank, local):
             step(args.warmup + i)
     reps = {}
     g_kern = []
+    g_warm = []   # the same buffers every launch: a warm-L2 figure, reported separately
     for j, p in enumerate(problems):
         r = max(8, len(sets[p.name]))
         reps[j] = r
@@ -363,9 +399,14 @@ def run_ours(args, world, rank, local):
                 dy, w, out = sets[p.name][i % len(sets[p.name])]
                 call(p, dy, w, out)
         g_kern.append(g)
+        gw = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gw):
+            for i in range(r):
+                call(p, *sets[p.name][0])
+        g_warm.append(gw)
     for _ in range(2):
         g_steps.replay()
-        for g in g_kern:
+        for g in g_kern + g_warm:
             g.replay()
     torch.cuda.synchronize()
     cb.check_status()
@@ -382,23 +423,33 @@ def run_ours(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     step_ms = e0.elapsed_time(e1) / args.steps
-    kern_ms = []
-    kern_iters = max(1, args.steps // 4)
-    for j, g in enumerate(g_kern):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(kern_iters):
+    # per kernel: KERN_REPS separately timed replays of its graph, median (and min)
+    kern_ms, kern_min_ms, warm_ms = [], [], []
+
+    def timed_replays(g, r):
+        out = []
+        for _ in range(KERN_REPS):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
             g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        kern_ms.append(a.elapsed_time(b) / (kern_iters * reps[j]))
+            b.record(stream)
+            torch.cuda.synchronize()
+            out.append(a.elapsed_time(b) / r)
+        return out
+
+    for j in range(len(problems)):
+        t = timed_replays(g_kern[j], reps[j])
+        kern_ms.append(statistics.median(t))
+        kern_min_ms.append(min(t))
+        warm_ms.append(statistics.median(timed_replays(g_warm[j], reps[j])))
+    kern_iters = KERN_REPS
     clocks = sampler.stop()
     barrier(world)
     cb.check_status()
     # kernels one call launches: the tensor-core depthwise call runs pack, filter pack, MMA and
     # unpack kernels; split-K runs the GEMM and the reduction; every other call is one kernel
     per_call = [4 if p.variant == "tc" else 2 if p.variant == "splitk" else 1 for p in problems]
-    n_launches = sum((args.steps + kern_iters * reps[j]) * per_call[j] for j in range(len(problems)))
+    n_launches = sum((args.steps + 2 * kern_iters * reps[j]) * per_call[j] for j in range(len(problems)))
 
     step_ms_max = max_over_ranks(world, step_ms, dev)
     flops_step = sum(p.nominal_flops() for p in problems)
@@ -412,8 +463,9 @@ def run_ours(args, world, rank, local):
     bf16_peak = peaks["bf16_tflops"]
     traffic = traffic_record()
     per_kernel = []
-    for p, ms in zip(problems, kern_ms):
+    for p, ms, ms_min, ms_warm in zip(problems, kern_ms, kern_min_ms, warm_ms):
         fl = p.nominal_flops()
+        fl_in = inbounds_flops(p)
         by = p.algorithmic_bytes()
         tf = fl / (ms * 1e-3) / 1e12
         gbs = by / (ms * 1e-3) / 1e9
@@ -440,6 +492,15 @@ def run_ours(args, world, rank, local):
             "frac_of_tensor_peak": round(tf / bf16_peak, 4) if bound == "tensor" else None,
             "frac_of_hbm": round(gbs / hbm, 4),
             "fp32_floor_us": round(fl / (fp32_peak * 1e12) * 1e6, 3) if p.kind == "depthwise" else None,
+            # the depthwise roofline as the benchmark's target defines it (bytes at HBM
+            # bandwidth against nominal FMAs at the FP32 peak), for every depthwise kernel,
+            # tensor-core ones included
+            "frac_hbm_fp32_roofline": (round(max(t_bytes, fl / (fp32_peak * 1e12)) / (ms * 1e-3), 4)
+                                       if p.kind == "depthwise" else None),
+            "inbounds_flop": fl_in, "nominal_flop": fl, "inbounds_tflops": round(fl_in / (ms * 1e-3) / 1e12, 3),
+            "us_min": round(ms_min * 1e3, 3), "replays": KERN_REPS,
+            "warm_l2_us": round(ms_warm * 1e3, 3),
+            "warm_l2_tflops": round(fl / (ms_warm * 1e-3) / 1e12, 3),
             "dram_bytes_per_launch": tr})
     dom = max(range(len(problems)), key=lambda j: kern_ms[j])
     dp = problems[dom]
@@ -453,6 +514,11 @@ def run_ours(args, world, rank, local):
     else:
         roof = {"bound": "alu", "achieved": dk["tflops"], "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
                 "frac": round(dk["tflops"] / fp32_peak, 4), "traffic": dk["dram_bytes_per_launch"]}
+    if dp.variant == "tc":
+        roof["basis"] = ("nominal FLOPs against the bf16 tensor peak (the kernel runs on the tensor cores); "
+                         "frac_hbm_fp32_roofline is the depthwise roofline of the benchmark's target: "
+                         "max(bytes / HBM, nominal FLOPs / FP32 peak) / time")
+        roof["frac_hbm_fp32_roofline"] = dk["frac_hbm_fp32_roofline"]
     roof.update({"kernel": dk["kernel"], "problem": dp.name,
                  "peak_source": (f"{peak_src} (MEASURED_PEAKS.json)" if roof["bound"] != "alu" else
                                  f"derived: {sms} SMs x {FP32_LANES_PER_SM} FMA/clk x 2 x {sm_max:.0f} MHz")})
@@ -520,7 +586,10 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": n_launches,
-        "timing": "CUDA graphs replayed on the launching stream, CUDA events around the replay",
+        "timing": ("CUDA graphs replayed on the launching stream, CUDA events around the replay; the step "
+                   "is one graph of `steps` steps; per_kernel us = median of 10 separately timed replays of "
+                   "a graph of back-to-back launches over rotating cold copies (warm_l2_us: the same buffers "
+                   "every launch, so inputs that fit stay in L2)"),
         "peaks": {"source": peak_src, "hbm_gbs": hbm, "bf16_tflops": bf16_peak,
                   "fp32_tflops_at_max_clock": round(fp32_peak, 2)},
     }
