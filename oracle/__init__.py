@@ -9,7 +9,9 @@ which holds none of the method's arithmetic.
 The arithmetic lives in ``dgrad_oracle.c`` (plain fp64 loops, OpenMP over the
 batch).  This module builds it with gcc, loads it with ctypes and marshals numpy
 arrays.  Each wrapper names the C routine it calls; the C file cites the
-passages each routine follows.
+passages each routine follows.  Two whole-array fp64 forms written with numpy
+(``pointwise_matmul``, ``depthwise_taps``) serve comparisons of every element of
+full-size problems; both are pinned to the C scatter loop.
 
 Layouts (NHWC, channels innermost):
   dY  (N, Ho, Wo, K)           dX (N, H, W, C)
@@ -227,4 +229,54 @@ def dw_rowstream(dy, w, *, H: int, W: int, S: int, ph: int, pw: int) -> np.ndarr
     dx = np.empty((N, H, W, C), dtype=np.float64)
     if _load().oracle_dw_rowstream(ctypes.byref(g), _dptr(dy), _dptr(w), _dptr(dx)):
         raise ValueError("oracle_dw_rowstream rejected the geometry")
+    return dx
+
+
+# --- Whole-array fp64 forms (numpy), for comparing every element of full-size
+# problems in seconds.  Each is the definition written with array slices; each is
+# pinned to the scatter loop above on small problems (tests/test_oracle.py).
+
+def pointwise_matmul(dy, w) -> np.ndarray:
+    """Pointwise dgrad as the plain product dX[M, C] = dY[M, K] . W[K, C] in fp64,
+    M = N*H*W ("add the pointwise fast path dgrad was missing", Technical Details:
+    dY offset m*K + k, W offset k*C + c)."""
+    dy = np.asarray(dy, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    N, H, W, K = dy.shape
+    return (dy.reshape(-1, K) @ w).reshape(N, H, W, w.shape[1])
+
+
+def depthwise_taps(dy, w, *, H: int, W: int, S: int = 1, ph: int = 0, pw: int = 0) -> np.ndarray:
+    """Depthwise dgrad (groups = C) in fp64 as one strided slice update per filter tap.
+
+    The scatter form of the adjoint: dY[n, ho, wo, c] * W[r][s][c] adds into
+    dX[n, ho*S - ph + r, wo*S - pw + s, c]; for a fixed tap (r, s) the targets of
+    all (ho, wo) form a strided slice of dX, so each tap is one array update.
+    Targets outside [0, H) x [0, W) are dropped ("channel-packed and large-filter
+    depthwise dgrad", Technical Details: the stride / padding geometry and the
+    row-streaming schedule apply exactly these scatter targets)."""
+    dy = np.asarray(dy, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    N, Ho, Wo, C = dy.shape
+    KH, KW = w.shape[:2]
+    dx = np.zeros((N, H, W, C), dtype=np.float64)
+
+    def span(extent_out, extent_in, off):
+        # ho values whose target ho*S + off lies in [0, extent_in)
+        lo = max(0, -(-(0 - off) // S))
+        hi = min(extent_out, (extent_in - 1 - off) // S + 1) if extent_in - 1 - off >= 0 else 0
+        return lo, max(lo, hi)
+
+    for r in range(KH):
+        h_lo, h_hi = span(Ho, H, r - ph)
+        if h_lo >= h_hi:
+            continue
+        for s in range(KW):
+            w_lo, w_hi = span(Wo, W, s - pw)
+            if w_lo >= w_hi:
+                continue
+            h0 = h_lo * S - ph + r
+            w0 = w_lo * S - pw + s
+            dx[:, h0:h0 + (h_hi - h_lo - 1) * S + 1:S, w0:w0 + (w_hi - w_lo - 1) * S + 1:S, :] += \
+                dy[:, h_lo:h_hi, w_lo:w_hi, :] * w[r, s, :]
     return dx

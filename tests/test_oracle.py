@@ -398,3 +398,54 @@ def test_synthetic_workloads_shapes():
     # the same seed gives the same draws
     again = synthetic.make_inputs(synthetic.problem("dw3x3_bf16"))
     np.testing.assert_array_equal(inp.dy_bits, again.dy_bits)
+
+
+# --- the whole-array fp64 forms used for full-size comparisons -----------------
+
+WHOLE_ARRAY_GEOMS = [
+    # N, H, W, C, KH, KW, S, ph, pw
+    (2, 7, 9, 3, 3, 3, 1, 1, 1),      # 3x3 'same'
+    (1, 11, 10, 2, 7, 7, 2, 3, 3),    # 7x7 stride 2
+    (2, 9, 8, 4, 5, 2, 3, 2, 1),      # stride 3, per-axis padding
+    (1, 12, 5, 3, 4, 4, 2, 0, 3),     # even filter, unequal pads
+    (1, 9, 9, 2, 2, 2, 3, 0, 0),      # filter smaller than the stride (gaps)
+    (2, 13, 9, 3, 13, 5, 1, 6, 2),    # non-square stride-1 ('same')
+    (1, 6, 6, 2, 1, 1, 1, 0, 0),      # 1x1
+]
+
+
+@pytest.mark.parametrize("geom", WHOLE_ARRAY_GEOMS)
+def test_depthwise_taps_equals_scatter_loop(geom):
+    """The per-tap slice form is the same sum as the scatter loop (up to fp64 rounding order)."""
+    N, H, W, C, KH, KW, S, ph, pw = geom
+    Ho = (H + 2 * ph - KH) // S + 1
+    Wo = (W + 2 * pw - KW) // S + 1
+    rng = np.random.default_rng(hash(geom) % 2**32)
+    dy = rng.standard_normal((N, Ho, Wo, C))
+    w = rng.standard_normal((KH, KW, C))
+    got = oracle.depthwise_taps(dy, w, H=H, W=W, S=S, ph=ph, pw=pw)
+    ref = oracle.dgrad(dy, w, kind="depthwise", H=H, W=W, KH=KH, KW=KW, S=S, ph=ph, pw=pw)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12 * (1 + np.abs(ref).max()))
+
+
+def test_depthwise_taps_catches_a_dropped_tap():
+    """A slice form that skips one tap must not pass the comparison above."""
+    N, H, W, C, KH, KW, S, ph, pw = WHOLE_ARRAY_GEOMS[1]
+    Ho = (H + 2 * ph - KH) // S + 1
+    rng = np.random.default_rng(7)
+    dy = rng.standard_normal((N, Ho, Ho, C))
+    w = rng.standard_normal((KH, KW, C))
+    w_dropped = w.copy()
+    w_dropped[3, 4, :] = 0.0
+    got = oracle.depthwise_taps(dy, w_dropped, H=H, W=W, S=S, ph=ph, pw=pw)
+    ref = oracle.dgrad(dy, w, kind="depthwise", H=H, W=W, KH=KH, KW=KW, S=S, ph=ph, pw=pw)
+    assert np.abs(got - ref).max() > 1e-3
+
+
+def test_pointwise_matmul_equals_scatter_loop():
+    rng = np.random.default_rng(11)
+    dy = rng.standard_normal((2, 5, 7, 24))
+    w = rng.standard_normal((24, 40))
+    got = oracle.pointwise_matmul(dy, w)
+    ref = oracle.dgrad(dy, w, kind="pointwise", H=5, W=7)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12 * (1 + np.abs(ref).max()))

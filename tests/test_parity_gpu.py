@@ -628,3 +628,88 @@ def test_streams_are_respected():
     ref = h.oracle_full(p, inp.dy, inp.w)
     absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
     h.check(p, h.gpu_to_np(out), ref, absref, what="side stream")
+
+
+# --- every element of the full-size workloads against the oracle ----------------
+
+EVERY = [p for p in synthetic.all_problems() if p.name in ("pw_bf16", "dw3x3_bf16", "dw7x7s2_bf16")]
+
+
+def _oracle_whole(p, dy, w):
+    import oracle
+    if p.kind == "pointwise":
+        return oracle.pointwise_matmul(dy, w)
+    return oracle.depthwise_taps(dy, w, H=p.H, W=p.W, S=p.stride, ph=p.pad_h, pw=p.pad_w)
+
+
+@pytest.mark.parametrize("p", EVERY, ids=[p.name for p in EVERY])
+def test_full_size_every_element(p):
+    """The benchmark's pointwise bf16, depthwise 3x3 and 7x7 stride-2 problems at full size, every
+    element of dX against the fp64 oracle (whole-array form, pinned to the scatter loop) under the
+    normwise bar and the elementwise bound."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = h.run_gpu(p, dy, w)
+    cb.check_status()
+    got = h.gpu_to_np(out)
+    ref = _oracle_whole(p, inp.dy, inp.w)
+    absref = _oracle_whole(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name} every element")
+
+
+TC_EVERY_CHANNELS = (0, 1, 2, 3, 4, 5, 6, 7, 200, 201, 202, 203, 204, 205, 206, 207, -8, -7, -6, -5, -4, -3, -2, -1)
+
+
+@pytest.mark.parametrize("entry", ["tc", "auto"])
+@pytest.mark.parametrize("p", TC_FULL, ids=[p.name for p in TC_FULL])
+def test_full_size_tensor_core_channel_subset(p, entry):
+    """The large-filter workloads at full size: every image and every spatial position of 24 channels
+    (the first, a middle and the last 8-channel block) against the fp64 oracle, through the planar
+    tensor-core entry point and through dgrad_depthwise's automatic choice.  Depthwise channels are
+    independent, so a channel subset is an exact sub-problem."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    if entry == "tc":
+        out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    else:
+        out = cb.depthwise(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    cb.check_status()
+    ch = np.array([c % p.C for c in TC_EVERY_CHANNELS])
+    got = out.float()[..., torch.from_numpy(ch).cuda()].cpu().numpy().astype(np.float64)
+    sub = p.replace(C=len(ch), K=len(ch))
+    dys, ws = inp.dy[..., ch], inp.w[..., ch]
+    ref = _oracle_whole(sub, dys, ws)
+    absref = _oracle_whole(sub, np.abs(dys), np.abs(ws))
+    h.check(sub, got, ref, absref, what=f"{p.name}/{entry} channels {list(ch[:3])}..")
+
+
+def test_planted_dy_stride_mistake_is_caught():
+    """The pages' lesson for the pointwise fast path (a mutated dY pixel stride must fail the numeric
+    suite): dgrad_pointwise is handed a dY whose rows really lie K + 8 elements apart while the
+    problem says K, as a kernel with a wrong stride would read it.  The parity check must fail."""
+    h = _h()
+    import ctypes
+    import convolution_backward_b200 as cb
+    p = P("pw_planted", "pointwise", "bf16", 2, 14, 14, 64, 64, seed=77)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    M = p.N * p.H * p.W
+    wide = torch.zeros((M, p.K + 8), dtype=dy.dtype, device=dy.device)
+    wide[:, :p.K] = dy.reshape(M, p.K)
+    out = torch.empty(p.dx_shape, dtype=dy.dtype, device=dy.device)
+    prob = cb.Problem(p.N, p.H, p.W, p.C, p.K, 1, 1, 1, 0, 0)
+    L = cb.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.dgrad_pointwise(ctypes.byref(prob), 1, wide.data_ptr(), w.data_ptr(), out.data_ptr(), stream) == 0
+    cb.check_status()
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    with pytest.raises(AssertionError):
+        h.check(p, got, ref, absref, what="planted dY stride")
+    # and the same buffers read with the right layout pass
+    h.check(p, h.gpu_to_np(cb.pointwise(dy, w)), ref, absref, what="right dY stride")
