@@ -23,12 +23,15 @@ __all__ = ["pointwise", "pointwise_splitk", "pointwise_splitk_noalloc", "depthwi
            "Problem", "lib", "library_path", "selftest_timeout", "fma_probe", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "libdgrad.so")
+# DGRAD_LIBRARY=debug loads libdgrad_debug.so: the same kernels built with index
+# checks on every hand-indexed store (a failed check skips the store and makes
+# check_status raise with DGRAD_ERR_BOUNDS).
+_LIB_PATH = os.path.join(_PKG, "libdgrad_debug.so" if os.environ.get("DGRAD_LIBRARY") == "debug" else "libdgrad.so")
 _lock = threading.Lock()
 _lib = None
 
 STATUS = {0: "DGRAD_OK", 1: "DGRAD_ERR_INVALID", 2: "DGRAD_ERR_UNSUPPORTED", 3: "DGRAD_ERR_ALIGNMENT",
-          4: "DGRAD_ERR_CUDA", 5: "DGRAD_ERR_TIMEOUT"}
+          4: "DGRAD_ERR_CUDA", 5: "DGRAD_ERR_TIMEOUT", 6: "DGRAD_ERR_BOUNDS"}
 DW_MODES = {"auto": 0, "rotated": 1, "rowstream": 2}
 DTYPES = {"f32": 0, "bf16": 1, "f16": 2}
 SPLITK_SCRATCH_BYTES = 8 << 20   # DGRAD_SPLITK_SCRATCH_BYTES: the fixed per-device split-K buffer

@@ -1,9 +1,12 @@
-"""Build libdgrad.so in-tree with nvcc for sm_100a.
+"""Build libdgrad.so (and libdgrad_debug.so) in-tree with nvcc for sm_100a.
 
 Every .cu file under csrc/ is compiled to an object in _build/ (in parallel),
 then linked into convolution_backward_b200/libdgrad.so with the CUDA runtime
-linked statically.  ptxas register/spill reports go to _build/ptxas.log.
-Rebuilds only when a source, header or this file is newer than the library.
+linked statically.  ptxas register/spill reports go to _build/ptxas.log.  The
+same sources built with -DDGRAD_DEBUG (objects in _build/debug/) give
+libdgrad_debug.so, whose kernels check every hand-indexed store against its
+output buffer.  Rebuilds only when a source, header or this file is newer than
+a library.
 """
 from __future__ import annotations
 
@@ -19,6 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdgrad.so")
+LIB_DEBUG = os.path.join(PKG, "libdgrad_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v",
@@ -40,10 +44,10 @@ def _inputs():
 
 
 def needs_build() -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(LIB_DEBUG):
         return True
     _, deps = _inputs()
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(LIB_DEBUG))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
@@ -54,26 +58,33 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs, _ = _inputs()
 
-    def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [nvcc, *CFLAGS, "-c", src, "-o", obj]
+    debug_dir = os.path.join(BUILD, "debug")
+    os.makedirs(debug_dir, exist_ok=True)
+
+    def compile_one(job):
+        src, debug = job
+        obj = os.path.join(debug_dir if debug else BUILD, os.path.basename(src) + ".o")
+        cmd = [nvcc, *CFLAGS, *(["-DDGRAD_DEBUG"] if debug else []), "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         return obj, r.stderr
 
-    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 4)) as ex:
-        results = list(ex.map(compile_one, srcs))
+    jobs = [(s, False) for s in srcs] + [(s, True) for s in srcs]
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+        results = list(ex.map(compile_one, jobs))
+    release, debug = results[:len(srcs)], results[len(srcs):]
     with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
-        for (obj, log), src in zip(results, srcs):
+        for (obj, log), src in zip(release, srcs):
             f.write(f"==== {os.path.basename(src)}\n{log}\n")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *[o for o, _ in results],
-           "-ldl", "-lpthread", "-lrt"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    for lib, objs in ((LIB, release), (LIB_DEBUG, debug)):
+        tmp = lib + f".tmp{os.getpid()}"
+        cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *[o for o, _ in objs],
+               "-ldl", "-lpthread", "-lrt"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, lib)
     if verbose:
         print(f"built {LIB}")
     return LIB

@@ -17,7 +17,7 @@
 namespace dgrad {
 
 // Device status word values (the host maps DEV_TIMEOUT to DGRAD_ERR_TIMEOUT).
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 5 };
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 5, DEV_BOUNDS = 6 };
 
 // A wait gives up after this many SM cycles (about one second at 2 GHz).
 constexpr long long kWaitCycles = 2000000000LL;
@@ -30,6 +30,25 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p)
 __device__ __forceinline__ void report_timeout(int* status)
 {
     if (status) atomicExch(status, DEV_TIMEOUT);
+}
+
+// Index checks of the debug build (compiled with -DDGRAD_DEBUG into
+// libdgrad_debug.so): a hand-indexed store of n bytes at p must lie inside the
+// buffer [base, base + bytes).  One that would not is skipped and DEV_BOUNDS is
+// recorded in the status word (dgrad_check_status reports DGRAD_ERR_BOUNDS).
+// Release builds compile the check to `true`.
+__device__ __forceinline__ bool store_ok(const void* base, long long bytes, const void* p, int n, int* status)
+{
+#ifdef DGRAD_DEBUG
+    const long long off = static_cast<const char*>(p) - static_cast<const char*>(base);
+    if (off < 0 || off + n > bytes) {
+        if (status) atomicExch(status, DEV_BOUNDS);
+        return false;
+    }
+#else
+    (void)base, (void)bytes, (void)p, (void)n, (void)status;
+#endif
+    return true;
 }
 
 // ------------------------------------------------- programmatic dependent launch

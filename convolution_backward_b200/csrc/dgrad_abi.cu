@@ -636,7 +636,7 @@ dgrad_status_t dgrad_check_status(void* stream)
         e = cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return cuda_fail(e);
     }
-    return v == dgrad::DEV_TIMEOUT ? DGRAD_ERR_TIMEOUT : DGRAD_OK;
+    return v == dgrad::DEV_TIMEOUT ? DGRAD_ERR_TIMEOUT : v == dgrad::DEV_BOUNDS ? DGRAD_ERR_BOUNDS : DGRAD_OK;
 }
 
 const char* dgrad_status_string(dgrad_status_t s)
@@ -648,6 +648,7 @@ const char* dgrad_status_string(dgrad_status_t s)
     case DGRAD_ERR_ALIGNMENT: return "pointer or channel row not 16-byte aligned";
     case DGRAD_ERR_CUDA: return "CUDA error";
     case DGRAD_ERR_TIMEOUT: return "a kernel gave up waiting (timeout)";
+    case DGRAD_ERR_BOUNDS: return "a debug-build index check failed (a store was skipped)";
     }
     return "unknown status";
 }

@@ -53,6 +53,8 @@ struct RotParams {
     long long out_sA, out_sB, out_sN;
     int w_sA, w_sB;           // filter strides along A and B (W is [KH][KW][C])
     int NS, TB, TAC, LA, RING;
+    long long dx_bytes;       // size of dX (index checks of the debug build)
+    int* status;
     int nA, nB, nC;
 };
 
@@ -240,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int j = 0; j < TAT; ++j) {
         const int a = a0 + strip * TAT + j;
-        if (a < p.OA) {
+        if (a < p.OA && store_ok(p.dX, p.dx_bytes, out + a * p.out_sA, EK != kF32 ? 4 : 8, p.status)) {
             if constexpr (EK != kF32)
                 *reinterpret_cast<uint32_t*>(out + a * p.out_sA) = float2_to_h16x2<EK>(acc[j].x, acc[j].y);
             else
@@ -337,6 +339,8 @@ cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream)
     }
     p.in_sN = static_cast<long long>(a.Ho) * a.Wo * C;
     p.out_sN = static_cast<long long>(a.H) * a.W * C;
+    p.dx_bytes = p.out_sN * a.N * (a.elem_kind() == kF32 ? 4 : 2);
+    p.status = a.status;
 
     int kai = 0;
     for (int v : kInstKA)

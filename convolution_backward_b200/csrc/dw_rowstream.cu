@@ -48,6 +48,8 @@ struct RsParams {
     int nX, nC;   // column strips, channel blocks
     int LW;       // dY columns staged per row
     bool w_in_smem;
+    long long dx_bytes;   // size of dX (index checks of the debug build)
+    int* status;
 };
 
 __device__ __forceinline__ int floor_div(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
@@ -169,8 +171,8 @@ __global__ void __launch_bounds__(kThreads)
             float2* e = ring + (sl * p.TX + xl) * kPairs + cp;
             const float2 v = *e;
             *e = make_float2(0.f, 0.f);
-            if (x < p.W && c_ok) {
-                T* o = dx + (static_cast<long long>(h) * p.W + x) * C + c;
+            T* o = dx + (static_cast<long long>(h) * p.W + x) * C + c;
+            if (x < p.W && c_ok && store_ok(p.dX, p.dx_bytes, o, EK != kF32 ? 4 : 8, p.status)) {
                 if constexpr (EK != kF32)
                     *reinterpret_cast<uint32_t*>(o) = float2_to_h16x2<EK>(v.x, v.y);
                 else
@@ -240,6 +242,8 @@ cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream)
     p.dX = a.dX;
     p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.Ho = a.Ho; p.Wo = a.Wo;
     p.KH = a.KH; p.KW = a.KW; p.S = a.S; p.ph = a.ph; p.pw = a.pw;
+    p.dx_bytes = static_cast<long long>(a.N) * a.H * a.W * a.C * (a.elem_kind() == kF32 ? 4 : 2);
+    p.status = a.status;
     p.R = a.KH > a.S ? a.KH : a.S;
     p.nC = (a.C + kCB - 1) / kCB;
     // Widest strip (64, 48, 32 or 16 columns) whose ring and staged row fit the

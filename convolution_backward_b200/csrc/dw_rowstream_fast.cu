@@ -56,6 +56,7 @@ struct FastParams {
     int LW;       // dY columns per staged row
     int BH;       // dX rows per band (multiple of G*S)
     int nX, nC, nB;
+    long long dx_bytes;   // size of dX (index checks of the debug build)
 };
 
 template <int KH, int KW, int S, int Q, int G>
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                 uint16_t* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
                 for (int q = 0; q < Q; ++q)
-                    if ((xmask >> q) & 1u)
+                    if (((xmask >> q) & 1u) && store_ok(p.dX, p.dx_bytes, orow + xoff[q], 4, p.status))
                         *reinterpret_cast<uint32_t*>(orow + xoff[q]) = float2_to_h16x2<EK>(acc[i][q].x, acc[i][q].y);
             }
         }
@@ -269,7 +270,8 @@ template <int KH, int KW, int S, int Q, int RS, int GT, int NT, int EK>
 __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 (&wr)[KH][(KW + S - 1) / S],
                                              const uint32_t* stage, int LW, int cp, int col0, int hb, int h0,
                                              int h1, uint16_t* obase, long long row_elems,
-                                             const int (&xoff)[Q], uint32_t xmask)
+                                             const int (&xoff)[Q], uint32_t xmask, const void* dx_base,
+                                             long long dx_bytes, int* status)
 {
     static_assert((S * GT) % RS == 0 && RS >= KH && KH >= S, "ring geometry");
     // dY row k of the stage, converted to fp32 pairs; row k+1 is loaded while row k computes
@@ -309,7 +311,7 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
                 uint16_t* orow = obase + static_cast<long long>(h) * row_elems;
 #pragma unroll
                 for (int q = 0; q < Q; ++q)
-                    if ((xmask >> q) & 1u)
+                    if (((xmask >> q) & 1u) && store_ok(dx_base, dx_bytes, orow + xoff[q], 4, status))
                         *reinterpret_cast<uint32_t*>(orow + xoff[q]) =
                             float2_to_h16x2<EK>(acc[slot][q].x, acc[slot][q].y);
             }
@@ -424,10 +426,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const int hb = hb0 + st * GT * S;
         if (nt == NTMAX)
             rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX, EK>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
-                                                      row_elems, xoff, xmask);
+                                                      row_elems, xoff, xmask, p.dX, p.dx_bytes, p.status);
         else
             rs_reg_stage<KH, KW, S, Q, RS, GT, NTMAX - 1, EK>(acc, wr, stage, p.LW, cp, col0, hb, h0, h1, obase,
-                                                          row_elems, xoff, xmask);
+                                                          row_elems, xoff, xmask, p.dX, p.dx_bytes, p.status);
         __syncthreads();
     }
     if (tid == 0)
@@ -455,6 +457,7 @@ FastParams plan_fast(const DwArgs& a, const void* kern = nullptr, size_t (*smem_
     p.filt = static_cast<const uint16_t*>(a.filt);
     p.status = a.status;
     p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.Ho = a.Ho; p.Wo = a.Wo; p.ph = a.ph; p.pw = a.pw;
+    p.dx_bytes = static_cast<long long>(a.N) * a.H * a.W * a.C * 2;
     // strip width: pick the slot count (multiple of 2*S, at most 16) that wastes the fewest columns
     int best = -1, best_waste = 1 << 30;
     for (int ns = 16; ns >= 2 * S; ns -= 2 * S) {

@@ -31,6 +31,7 @@ struct TileParams {
     int CS, RS;       // column and row slots per CTA (threads = 16 * CS * RS)
     int TH, TW;       // output tile
     int nX, nY, nC;
+    long long dx_bytes;   // size of dX (index checks of the debug build)
 };
 
 template <int KH, int KW, int R, int TAT, int EK>
@@ -138,7 +139,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int j = 0; j < TAT; ++j) {
             const int w = w0 + col0 + j;
-            if (w < p.W && col0 + j < p.TW)
+            if (w < p.W && col0 + j < p.TW &&
+                store_ok(p.dX, p.dx_bytes, orow + static_cast<long long>(w) * p.C, 4, p.status))
                 *reinterpret_cast<uint32_t*>(orow + static_cast<long long>(w) * p.C) =
                     float2_to_h16x2<EK>(acc[ro][j].x, acc[ro][j].y);
         }
@@ -153,6 +155,7 @@ TileParams plan_tile(const DwArgs& a)
     p.filt = static_cast<const uint16_t*>(a.filt);
     p.status = a.status;
     p.N = a.N; p.H = a.H; p.W = a.W; p.C = a.C; p.ph = a.ph; p.pw = a.pw;
+    p.dx_bytes = static_cast<long long>(a.N) * a.H * a.W * a.C * 2;
     // columns: as few column slots as cover the row (at most 16), balanced
     int cs = (a.W + TAT - 1) / TAT;
     if (cs > 16) {

@@ -91,6 +91,7 @@ struct ToepArgs {
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
     int f16;                     // operands and output are f16 (else bf16)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
+    long long dxp_bytes;         // size of the planar output (index checks of the debug build)
 };
 
 struct Unit {
@@ -388,6 +389,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         const int hcols = (a.XT * ncol_sub) >> 1;   // columns per half: at most 128
         const int nch = hcols >> 5;                  // 32-column chunks per half: 1 .. 4
         const int64_t img_stride = a.Xso;
+        // a 16-bit store into the planar output (checked against its size in the debug build)
+        auto put16 = [&](uint16_t* d, uint32_t v) {
+            if (store_ok(a.dXp, a.dxp_bytes, d, 2, a.status)) d[0] = static_cast<uint16_t>(v);
+        };
         const int64_t hrow_stride = static_cast<int64_t>(a.P) * a.N * a.Xso;
         uint32_t ub = 0;
         bool ok = true;
@@ -434,11 +439,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                             uint16_t* dst = base + hp * hrow_stride + img * img_stride;
                             const uint32_t v = pk[cc * 16 + k];
                             if (full) {
-                                dst[0] = static_cast<uint16_t>(v & 0xFFFFu);
-                                dst[img_stride] = static_cast<uint16_t>(v >> 16);
+                                put16(dst, v & 0xFFFFu);
+                                put16(dst + img_stride, v >> 16);
                             } else if (t.Y0 + a.P * (hp0 + hp) + p < a.Yo) {
-                                if (8 * t.g + img < a.N) dst[0] = static_cast<uint16_t>(v & 0xFFFFu);
-                                if (8 * t.g + img + 1 < a.N) dst[img_stride] = static_cast<uint16_t>(v >> 16);
+                                if (8 * t.g + img < a.N) put16(dst, v & 0xFFFFu);
+                                if (8 * t.g + img + 1 < a.N) put16(dst + img_stride, v >> 16);
                             }
                         }
                     }
@@ -532,7 +537,7 @@ constexpr int kRowsPerCta = 4;
 template <bool TO_PLANAR>
 __global__ void __launch_bounds__(256)
     dw_transpose_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int N, int Y, int X,
-                        int Xs, int C, int64_t sN, int64_t sY, int64_t sX)
+                        int Xs, int C, int64_t sN, int64_t sY, int64_t sX, long long dst_bytes, int* status)
 {
     pdl_wait();      // the previous kernel on the stream has finished
     __shared__ uint32_t tile[64][33];   // [row][pair]: rows are x (to planar) or c (from planar)
@@ -595,13 +600,13 @@ __global__ void __launch_bounds__(256)
                 w[j] = lo | (hi << 16);
             }
             if (TO_PLANAR) {
-                if (c0 + orow < C && x0 + ocol < X)
-                    *reinterpret_cast<uint4*>(dst + ((static_cast<int64_t>(c0 + orow) * Y + y) * N + n) * Xs + x0 +
-                                              ocol) = make_uint4(w[0], w[1], w[2], w[3]);
+                __nv_bfloat16* d = dst + ((static_cast<int64_t>(c0 + orow) * Y + y) * N + n) * Xs + x0 + ocol;
+                if (c0 + orow < C && x0 + ocol < X && store_ok(dst, dst_bytes, d, 16, status))
+                    *reinterpret_cast<uint4*>(d) = make_uint4(w[0], w[1], w[2], w[3]);
             } else {
-                if (x0 + orow < X && c0 + ocol < C)
-                    *reinterpret_cast<uint4*>(dst + n * sN + y * sY + static_cast<int64_t>(x0 + orow) * sX + c0 +
-                                              ocol) = make_uint4(w[0], w[1], w[2], w[3]);
+                __nv_bfloat16* d = dst + n * sN + y * sY + static_cast<int64_t>(x0 + orow) * sX + c0 + ocol;
+                if (x0 + orow < X && c0 + ocol < C && store_ok(dst, dst_bytes, d, 16, status))
+                    *reinterpret_cast<uint4*>(d) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
     }
@@ -900,7 +905,8 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
             {
                 const cudaError_t le_ = launch_kernel(dw_transpose_kernel<true>, dim3(grid), dim3(256), 0, stream, 1,
                                                      static_cast<const __nv_bfloat16*>(a.dY), dYp, a.N,
-                                                                p.Yi, p.Xi, p.Xsi, a.C, sN, sY, sX);
+                                                                p.Yi, p.Xi, p.Xsi, a.C, sN, sY, sX,
+                                                                static_cast<long long>(p.ws_in), a.status);
                 if (le_ != cudaSuccess) return le_;
             }
             e = cudaGetLastError();
@@ -956,6 +962,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;
         t.f_off = p.f_off;
         t.bar_off = p.bar_off;
+        t.dxp_bytes = static_cast<long long>(p.ws_out);
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));
         if (e != cudaSuccess) return e;
         const int grid = static_cast<int>(units < num_sms ? units : num_sms);
@@ -981,7 +988,9 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
             {
                 const cudaError_t le_ = launch_kernel(dw_transpose_kernel<false>, dim3(grid), dim3(256), 0, stream, 1,
                                                      dXp, static_cast<__nv_bfloat16*>(a.dX), a.N, p.Yo,
-                                                                 p.Xo, p.Xso, a.C, sN, sY, sX);
+                                                                 p.Xo, p.Xso, a.C, sN, sY, sX,
+                                                                 static_cast<long long>(a.N) * a.H * a.W * a.C * 2,
+                                                                 a.status);
                 if (le_ != cudaSuccess) return le_;
             }
         }

@@ -77,6 +77,7 @@ struct ToepNArgs {
     int f16, full_plane;
     int nfb;                   // filter-line buffers: 2, or 1 when two do not fit
     uint32_t panel_bytes, b_bytes, f_words, f_off, bar_off;
+    long long dx_bytes;        // size of dX (index checks of the debug build)
 };
 
 struct Tile {
@@ -197,6 +198,8 @@ __device__ void fill_window(const ToepNArgs& a, const Tile& t, int rank, int e, 
                              (static_cast<uint32_t>((xg & 7) ^ (R & 7)) << 4);
         // channel k of the 8 columns, stored to CTA k as soon as it is formed
 #pragma unroll
+        if (!store_ok(nullptr, a.b_bytes, reinterpret_cast<const void*>(static_cast<uintptr_t>(off)), 16, a.status))
+            continue;   // debug build: outside the B block (recorded)
         for (int k = 0; k < kCluster; ++k)
             st_cluster_v4(mapa_shared(b_local + off, static_cast<uint32_t>(k)), transpose8x8_col(v, k));
     }
@@ -221,6 +224,9 @@ __device__ void transpose_tile_out(const ToepNArgs& a, const Tile& t, int rank, 
         const int y = t.Y0 + q % nrow;
         const int img = 8 * t.g + q / nrow;
         uint16_t* base = a.dX + out_off(a, img, y, 8 * xg, t.cb);
+        if (!store_ok(a.dX, a.dx_bytes, base, 16, a.status) ||
+            !store_ok(a.dX, a.dx_bytes, base + 7 * a.sXo, 16, a.status))
+            continue;   // debug build: outside dX (recorded)
         uint4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) v[u] = ld_cg_v4(base + u * a.sXo);
@@ -537,8 +543,10 @@ __device__ __forceinline__ void ec_role(const ToepNArgs& a, const KCtx& k, int w
                         const uint32_t v = pk[cc * 16 + k];
                         if (y < a.Yo) {
                             uint16_t* d = colbase + img * a.sNo + y * a.sYo;
-                            if (img_full || 8 * tl.g + img < a.N) d[0] = static_cast<uint16_t>(v & 0xFFFFu);
-                            if (img_full || 8 * tl.g + img + 1 < a.N)
+                            if ((img_full || 8 * tl.g + img < a.N) && store_ok(a.dX, a.dx_bytes, d, 2, a.status))
+                                d[0] = static_cast<uint16_t>(v & 0xFFFFu);
+                            if ((img_full || 8 * tl.g + img + 1 < a.N) &&
+                                store_ok(a.dX, a.dx_bytes, d + a.sNo, 2, a.status))
                                 d[a.sNo] = static_cast<uint16_t>(v >> 16);
                         }
                     }
@@ -775,6 +783,7 @@ cudaError_t launch_dw_toeplitz_nhwc(const DwArgs& a, const ToepPlan& p, cudaStre
     t.f16 = a.f16 ? 1 : 0;
     t.full_plane = (t.num_xt == 1 && t.num_yt == 1) ? 1 : 0;
     t.nfb = p.nfb;
+    t.dx_bytes = static_cast<long long>(a.N) * a.H * a.W * a.C * 2;
     t.panel_bytes = p.panel_bytes;
     t.b_bytes = p.b_bytes;
     t.f_words = static_cast<uint32_t>(p.f_words);

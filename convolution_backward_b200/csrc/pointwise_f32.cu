@@ -22,7 +22,7 @@ constexpr int kLd = kTM * kTK / 4 / kThreads;   // float4 loads per thread per o
 
 __global__ void __launch_bounds__(kThreads)
     pw_f32_kernel(const float* __restrict__ dY, const float* __restrict__ W, float* __restrict__ dX, int M,
-                  int K, int C)
+                  int K, int C, int* status)
 {
     pdl_wait();      // the previous kernel on the stream has finished
     pdl_trigger();   // the next one may start its set-up
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int m = m0 + ty * 4 + i;
-        if (m < M)
+        if (m < M && store_ok(dX, static_cast<long long>(M) * C * 4, dX + static_cast<int64_t>(m) * C + c, 16, status))
             *reinterpret_cast<float4*>(dX + static_cast<int64_t>(m) * C + c) =
                 make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     }
@@ -100,7 +100,7 @@ cudaError_t launch_pointwise_f32(const PwArgs& a, cudaStream_t stream)
         const cudaError_t le_ = launch_kernel(pw_f32_kernel, dim3(grid), dim3(kThreads), 0, stream, 1,
                                              static_cast<const float*>(a.dY), static_cast<const float*>(a.W),
                                             static_cast<float*>(a.dX), static_cast<int>(a.M),
-                                            static_cast<int>(a.K), static_cast<int>(a.C));
+                                            static_cast<int>(a.K), static_cast<int>(a.C), a.status);
         if (le_ != cudaSuccess) return le_;
     }
     return cudaGetLastError();

@@ -957,7 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // to bf16 (or f16 when F16); 8 channels per thread.
 template <bool F16>
 __global__ void __launch_bounds__(256)
-    splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dX, long long MC, int S)
+    splitk_reduce_kernel(const float* __restrict__ ws, uint16_t* __restrict__ dX, long long MC, int S, int* status)
 {
     pdl_wait();      // the previous kernel on the stream has finished
     pdl_trigger();   // the next one may start its set-up
@@ -977,7 +977,7 @@ __global__ void __launch_bounds__(256)
     o.y = float2_to_h16x2<EK>(a.z, a.w);
     o.z = float2_to_h16x2<EK>(b.x, b.y);
     o.w = float2_to_h16x2<EK>(b.z, b.w);
-    *reinterpret_cast<uint4*>(dX + i) = o;
+    if (store_ok(dX, MC * 2, dX + i, 16, status)) *reinterpret_cast<uint4*>(dX + i) = o;
 }
 
 template <int BN, int STAGES>
@@ -1102,7 +1102,7 @@ cudaError_t launch_pointwise_tc_splitk(const PwArgs& a, const CUtensorMap& map_a
     {
         const cudaError_t le_ = launch_kernel(reduce, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, stream, 1,
                                              ws, static_cast<uint16_t*>(a.dX), MC,
-                                                                             S);
+                                                                             S, a.status);
         if (le_ != cudaSuccess) return le_;
     }
     return cudaGetLastError();

@@ -83,7 +83,8 @@ typedef enum {
     DGRAD_ERR_UNSUPPORTED = 2,  /* valid geometry this entry point does not serve */
     DGRAD_ERR_ALIGNMENT = 3,    /* base pointer or channel row not 16-byte aligned */
     DGRAD_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
-    DGRAD_ERR_TIMEOUT = 5       /* a kernel gave up waiting (reported by dgrad_check_status) */
+    DGRAD_ERR_TIMEOUT = 5,      /* a kernel gave up waiting (reported by dgrad_check_status) */
+    DGRAD_ERR_BOUNDS = 6        /* libdgrad_debug.so only: a store index check failed (dgrad_check_status) */
 } dgrad_status_t;
 
 /* Pointwise dgrad, dX[M,C] = dY[M,K] . W[K,C] with M = N*H*W.
@@ -219,7 +220,10 @@ dgrad_status_t dgrad_out_dims(const dgrad_problem_t* prob, int64_t* Ho, int64_t*
 
 /* Synchronise `stream`, then report (and clear) the device status word of the
  * current device: DGRAD_ERR_TIMEOUT if any kernel gave up waiting since the
- * last check, DGRAD_ERR_CUDA if the stream reported an error, else DGRAD_OK. */
+ * last check, DGRAD_ERR_BOUNDS if (in the debug build, libdgrad_debug.so, built
+ * from the same sources with -DDGRAD_DEBUG) a hand-indexed store fell outside
+ * its output buffer and was skipped, DGRAD_ERR_CUDA if the stream reported an
+ * error, else DGRAD_OK. */
 dgrad_status_t dgrad_check_status(void* stream);
 
 /* Static, human-readable text for a status code. */
