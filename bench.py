@@ -306,6 +306,8 @@ def kernel_of(p):
         return "dw_toeplitz_kernel", KERNEL_SOURCE["toeplitz"]
     if p.kind == "dense":
         return "dense_tc_kernel", KERNEL_SOURCE["dense"]
+    if p.variant == "rotated" and p.KH * p.KW > 49:
+        return "dw_rot_kernel", KERNEL_SOURCE["rotated"]
     if p.kind == "pointwise":
         return ("pw_tc_pair_kernel" if p.dtype == "bf16" else "pw_f32_kernel"), KERNEL_SOURCE["pointwise"][p.dtype]
     if p.stride == 1 and p.dtype == "bf16" and p.KH <= 7 and p.KW <= 7 and p.KH == p.KW and p.KH % 2 == 1 \
@@ -362,7 +364,8 @@ def run_ours(args, world, rank, local):
         elif p.kind == "dense":
             cb.dense(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
         else:
-            cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
+            cb.depthwise(dy, w, H=p.H, Wd=p.W, stride=p.stride, pad_h=p.pad_h, pad_w=p.pad_w, out=out,
+                         mode="rotated" if p.variant == "rotated" else "auto")
 
     def step(i, evs=None):
         for j, p in enumerate(problems):
@@ -446,9 +449,10 @@ def run_ours(args, world, rank, local):
     clocks = sampler.stop()
     barrier(world)
     cb.check_status()
-    # kernels one call launches: the tensor-core depthwise call runs pack, filter pack, MMA and
-    # unpack kernels; split-K runs the GEMM and the reduction; every other call is one kernel
-    per_call = [4 if p.variant == "tc" else 2 if p.variant == "splitk" else 1 for p in problems]
+    # kernels one call launches: the tensor-core depthwise call runs the dY transpose (whose extra
+    # CTAs pack the filter), the MMA kernel and the dX transpose; split-K runs the GEMM and the
+    # reduction; every other call is one kernel
+    per_call = [3 if p.variant == "tc" else 2 if p.variant == "splitk" else 1 for p in problems]
     n_launches = sum((args.steps + 2 * kern_iters * reps[j]) * per_call[j] for j in range(len(problems)))
 
     step_ms_max = max_over_ranks(world, step_ms, dev)

@@ -255,8 +255,11 @@ constexpr int kInstKA[] = {1, 3, 5, 7, 9, 11, 13, 15, 17, 21, 25, 31, 33, 41, 51
 
 template <int KAI>
 constexpr int tat_for() { return KAI <= 7 ? 8 : 16; }
+// The alternative (tuning) width: 16 for short lines, 8 for long ones.  32 outputs
+// per thread were measured slower for long lines and spilled registers at KA >= 13,
+// so they are not built.
 template <int KAI>
-constexpr int tat_alt() { return KAI <= 7 ? 16 : 32; }
+constexpr int tat_alt() { return KAI <= 7 ? 16 : 8; }
 
 template <int KAI, int TAT, int EK>
 cudaError_t launch_one(RotParams& p, long long blocks, cudaStream_t stream)

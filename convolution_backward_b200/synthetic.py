@@ -46,7 +46,8 @@ class Problem:
     dy_var: float = 1.0
     w_dist: str = "normal"
     w_var: float = 1.0
-    variant: str = ""    # "splitk": split-K pointwise entry point; "tc": tensor-core depthwise entry point
+    variant: str = ""    # "splitk": split-K pointwise entry point; "tc": tensor-core depthwise entry point;
+    #                      "rotated": dgrad_depthwise forced to the FP32 rotated-filter kernels
     ngroups: int = 1     # groups of a "grouped" problem (K and C multiples of it)
 
     @property
@@ -140,9 +141,10 @@ EXTRA_WORKLOADS: dict[str, list[Problem]] = {
     "dense3x3s2_bf16": [Problem("dense3x3s2_bf16", "dense", "bf16", N=32, H=56, W=56, C=128, K=256, KH=3, KW=3,
                                 stride=2, pad_h=1, pad_w=1, seed=7, w_var=1.0 / 2304)],
     # the large stride-1 depthwise problems through the FP32 rotated-filter kernel (dgrad_depthwise)
-    "dw_large_fp32": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_fp32", variant=""),
-                      WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_fp32", variant=""),
-                      WORKLOADS["dw_nonsquare_strided_bf16"][1].replace(name="dw5x51_bf16_fp32", variant="")],
+    "dw_large_fp32": [WORKLOADS["dw31x31_bf16"][0].replace(name="dw31x31_bf16_fp32", variant="rotated"),
+                      WORKLOADS["dw_nonsquare_strided_bf16"][0].replace(name="dw51x5_bf16_fp32", variant="rotated"),
+                      WORKLOADS["dw_nonsquare_strided_bf16"][1].replace(name="dw5x51_bf16_fp32",
+                                                                        variant="rotated")],
 }
 
 
