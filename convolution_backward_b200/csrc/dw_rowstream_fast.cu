@@ -326,8 +326,6 @@ template <int KH, int KW, int S, int Q, int RS, int GT, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_reg_kernel(const __grid_constant__ CUtensorMap dy_map, const FastParams p)
 {
-    pdl_wait();      // the previous kernel on the stream has finished
-    pdl_trigger();   // the next one may start its set-up
     constexpr int NTMAX = (KW + S - 1) / S;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -376,6 +374,15 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int hb0 = ho_lo * S - p.ph;
     const int nrows = (h1 - hb0 + S - 1) / S;          // dY rows until every band row is final
     const int nstages = (nrows + GT - 1) / GT;
+    if (tid == 0) {
+        // While the previous kernel may still run, only L2 prefetches of the first stages'
+        // tiles (L2 is the point of coherence, so the loads still see that kernel's writes).
+        tma_prefetch_desc(&dy_map);
+        for (int st = 0; st < kStages - 1 && st < nstages; ++st)
+            tma_prefetch_l2_4d(&dy_map, c0, wo_start, ho_lo + st * GT, n);
+    }
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
 
     float2 wr[KH][NTMAX];
 #pragma unroll
@@ -403,10 +410,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             : "memory");
     };
     int issued = 0;
-    if (tid == 0) {
-        tma_prefetch_desc(&dy_map);
+    if (tid == 0)
         for (; issued < kStages - 1 && issued < nstages; ++issued) issue(issued);
-    }
 
     float2 acc[RS][Q];
 #pragma unroll

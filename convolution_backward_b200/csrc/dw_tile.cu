@@ -38,8 +38,6 @@ template <int KH, int KW, int R, int TAT, int EK>
 __global__ void __launch_bounds__(256)
     dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const TileParams p)
 {
-    pdl_wait();      // the previous kernel on the stream has finished
-    pdl_trigger();   // the next one may start its set-up
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 127u) & ~127u) - raw);
@@ -67,12 +65,18 @@ __global__ void __launch_bounds__(256)
     const int w0 = xblk * p.TW;
 
     if (tid == 0) {
+        // While the previous kernel may still run, only an L2 prefetch of this CTA's halo
+        // tile: L2 is the point of coherence, so the load below still sees that kernel's
+        // writes; the DRAM reads overlap its tail.
+        tma_prefetch_desc(&dy_map);
+        tma_prefetch_l2_4d(&dy_map, c0, w0 - (KW - 1 - p.pw), h0 - (KH - 1 - p.ph), n);
         mbar_init(bar, 1);
         fence_mbar_init();
     }
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     __syncthreads();
     if (tid == 0) {
-        tma_prefetch_desc(&dy_map);
         mbar_arrive_expect_tx(bar, tile_bytes);
         asm volatile(
             "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
