@@ -512,6 +512,48 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   * cluster barriers order barrier initialisation before any remote arrive
 //     and keep both CTAs alive until all cross-CTA traffic has landed.
 // BN is the pair tile width (256 or 128); each CTA holds BN/2 columns of W.
+// The units of one SM pair.  Every pair takes R = tiles / pairs whole tiles
+// (t = pair, pair + pairs, ...).  When the L tiles left over fit twice into the
+// pairs (2L <= pairs), they are split into 2L halves of BN/2 columns, one per
+// pair, so the last round takes about half a tile instead of a whole one on a
+// third of the pairs; otherwise the first L pairs take one more whole tile.
+struct PwUnit {
+    int m_blk, n0, ncols;
+};
+
+struct PwSched {
+    int num_n, pairs, R, L;
+    bool split;
+    __device__ __forceinline__ PwSched(int num_tiles, int num_n_, int pairs_, int BN)
+    {
+        num_n = num_n_;
+        pairs = pairs_;
+        R = num_tiles / pairs;
+        L = num_tiles - R * pairs;
+        split = BN == 256 && L > 0 && 2 * L <= pairs;
+    }
+    __device__ __forceinline__ int count(int pair) const
+    {
+        return R + (split ? (pair < 2 * L ? 1 : 0) : (pair < L ? 1 : 0));
+    }
+    __device__ __forceinline__ PwUnit unit(int pair, int k, int BN) const
+    {
+        PwUnit u;
+        if (k < R || !split) {
+            const int t = pair + k * pairs;
+            u.m_blk = t / num_n;
+            u.n0 = (t - u.m_blk * num_n) * BN;
+            u.ncols = BN;
+        } else {
+            const int t = R * pairs + (pair >> 1);
+            u.m_blk = t / num_n;
+            u.n0 = (t - u.m_blk * num_n) * BN + (pair & 1) * (BN / 2);
+            u.ncols = BN / 2;
+        }
+        return u;
+    }
+};
+
 template <int BN, int STAGES>
 struct PwPairLayout {
     static constexpr int kBHalf = (BN / 2) * kBK * 2;         // this CTA's W columns, one k-block
@@ -554,6 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_kb = (K + kBK - 1) / kBK;
     const int pair = blockIdx.x >> 1;
     const int num_pairs = gridDim.x >> 1;
+    const PwSched sched(num_tiles, num_n, num_pairs, BN);
+    const int nunits = sched.count(pair);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPairStages; ++s) {
@@ -589,22 +633,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             long long issued = 0;
             bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-                const int m_blk = t / num_n;
-                const int n_blk = t - m_blk * num_n;
+            for (int k = 0; k < nunits && ok; ++k) {
+                const PwUnit un = sched.unit(pair, k, BN);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStage);
+                    // both CTAs' A halves (16 KB each) and W columns (ncols/2 each, 128 bytes per k row)
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (16384 + un.ncols * kBK));
                     uint8_t* a_tile = smem + L::kA + stage * L::kStage;
                     uint8_t* b_tile = a_tile + 16384;
                     const uint32_t fb = full0 + static_cast<uint32_t>(stage * 8);
-                    tma_load_2d_pair(a_tile, &map_a, fb, kb * kBK, m_blk * 256 + static_cast<int>(rank) * 128);
-                    const int ncol = n_blk * BN + static_cast<int>(rank) * (BN / 2);
-#pragma unroll
-                    for (int j = 0; j < BN / 128; ++j)
+                    tma_load_2d_pair(a_tile, &map_a, fb, kb * kBK, un.m_blk * 256 + static_cast<int>(rank) * 128);
+                    const int ncol = un.n0 + static_cast<int>(rank) * (un.ncols / 2);
+                    for (int j = 0; j < un.ncols / 128; ++j)
                         tma_load_2d_pair(b_tile + j * 8192, &map_b, fb, ncol + j * 64, kb * kBK);
                     ++issued;
                     if (++stage == kPairStages) {
@@ -627,13 +670,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(256, BN, /*b_mn_major=*/true);
+            constexpr uint32_t idesc_full = idesc_bf16_f32(256, BN, /*b_mn_major=*/true);
+            constexpr uint32_t idesc_half = idesc_bf16_f32(256, BN / 2, /*b_mn_major=*/true);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
-            for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+            for (int k = 0; k < nunits && ok; ++k) {
+                const uint32_t idesc = sched.unit(pair, k, BN).ncols == BN ? idesc_full : idesc_half;
                 if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -682,16 +727,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int t = pair; t < num_tiles; t += num_pairs) {
-            const int m_blk = t / num_n;
-            const int n_blk = t - m_blk * num_n;
+        for (int k = 0; k < nunits; ++k) {
+            const PwUnit un = sched.unit(pair, k, BN);
             if (!mbar_wait_cluster(&tfull[acc], acc_phase, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int chunk = 0; chunk < BN / 64; ++chunk) {
+            for (int chunk = 0; chunk < un.ncols / 64; ++chunk) {
                 uint8_t* buf = smem + L::kEpi + (chunk & 1) * 16384;
                 if (issuer) bulk_wait_group_read<1>();
                 named_barrier_sync(1, 128);
@@ -714,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 named_barrier_sync(1, 128);
                 if (issuer) {
-                    tma_store_2d(&map_d, buf, n_blk * BN + chunk * 64, m_blk * 256 + static_cast<int>(rank) * 128);
+                    tma_store_2d(&map_d, buf, un.n0 + chunk * 64, un.m_blk * 256 + static_cast<int>(rank) * 128);
                     bulk_commit_group();
                 }
             }

@@ -123,6 +123,29 @@ def test_pointwise_kernels(mode, bn, shape, monkeypatch):
     cb.check_status()
 
 
+# Shapes where the SM-pair kernel has more tiles than pairs and splits the leftover ones in N:
+# (N, H, W, C, K) with 75 tiles of 256 x 256 (one leftover tile, two halves), and with 80 tiles over
+# two column blocks of which the second is ragged (C = 320: the upper halves of its leftover tiles
+# lie wholly past C, so they load zeros and store nothing).
+PW_SPLIT = [(2, 95, 100, 256, 136), (5, 40, 50, 320, 72)]
+
+
+@pytest.mark.parametrize("shape", PW_SPLIT, ids=["75_tiles", "80_tiles_ragged_C"])
+def test_pointwise_pair_split_last_round(shape):
+    """The default pair kernel (256 x 256 tiles) where the last round's tiles are split in N."""
+    h = _h()
+    N, H, W, C, K = shape
+    p = P("pw_bf16_split", "pointwise", "bf16", N, H, W, C, K, seed=61)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what="pair, split last round")
+    import convolution_backward_b200 as cb
+    cb.check_status()
+
+
 ROT_SMALL = [
     P("tile3x3", "depthwise", "bf16", 2, 19, 23, 40, 40, 3, 3, 1, 1, 1, seed=81),
     P("tile3x3_wide", "depthwise", "bf16", 1, 9, 150, 32, 32, 3, 3, 1, 0, 2, seed=82),
