@@ -39,11 +39,13 @@
 // with zeros and packed two taps per word, from shared memory; the producer
 // brings them in with one bulk copy whenever the channel changes.
 //
-// Three helper kernels run around the MMA kernel, all through the caller's
-// workspace: dw_transpose_kernel writes NHWC dY as planes [C][Yi][N][Xs] (channels
-// outermost, images between rows and columns), dw_filter_pack_kernel writes the
-// padded filter lines of every channel, and dw_transpose_kernel writes the planar
-// output of the MMA epilogue back to NHWC dX.
+// Two transposes run around the MMA kernel, all through the caller's workspace:
+// the first writes NHWC dY as planes [C][Yi][N][Xs] (channels outermost, images
+// between rows and columns), and extra CTAs of the same launch write the padded
+// filter lines of every channel; the second writes the planar output of the MMA
+// epilogue back to NHWC dX.  Both are dw_transpose_tma_kernel (TMA on both
+// sides); when a tensor map cannot be encoded, dw_transpose_kernel (CUDA cores)
+// and a separate dw_filter_pack_kernel launch do the same.
 //
 // Launch order.  Like every kernel here, these wait for the kernel before them
 // (griddepcontrol.wait) before touching global memory.  Unlike the others, they
