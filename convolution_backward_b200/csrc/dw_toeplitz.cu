@@ -65,6 +65,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 #include "toeplitz_core.cuh"
@@ -92,6 +93,7 @@ struct ToepArgs {
     int num_xt, num_yt, num_g, num_units;
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
     int f16;                     // operands and output are f16 (else bf16)
+    int clip;                    // one tile spans the row: B starts at input column 0 (xb = 0)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
     long long dxp_bytes;         // size of the planar output (index checks of the debug build)
 };
@@ -111,7 +113,7 @@ __device__ __forceinline__ Unit decode_unit(const ToepArgs& a, int u)
     t.c = r / a.num_g;
     t.Y0 = yt * a.P * a.NH;
     t.x0 = xt * a.XT * a.TW;
-    t.xb = floor8(t.x0 - a.px);
+    t.xb = a.clip ? 0 : floor8(t.x0 - a.px);
     return t;
 }
 
@@ -762,6 +764,9 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     static const int cand[][3] = {{2, 32, 1}, {2, 16, 1}, {4, 16, 2}, {4, 8, 2}, {8, 8, 4}, {8, 4, 4}};
     // DGRAD_TC_TILE="orient,P,NH,XT" restricts the plan to that shape (testing and tuning).
     int force[4] = {-1, -1, -1, -1};
+    // DGRAD_TC_CLIP=0 keeps the full Toeplitz band for single-tile rows (testing and tuning).
+    const char* clp = dgrad::tuning_env("DGRAD_TC_CLIP");
+    const bool no_clip = clp && strcmp(clp, "0") == 0;
     if (const char* ft = dgrad::tuning_env("DGRAD_TC_TILE"))
         if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
@@ -789,14 +794,25 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             p.NH = cd[1];
             p.XT = cd[2];
             p.TW = 128 / p.P;
-            p.Ks = (p.TW + p.KX - 1 + mis + 15) & ~15;
+            // When one tile of one sub-tile spans the whole output row, the K range (input
+            // columns j) is clipped to the columns inside the image, starting at j = 0: the
+            // columns outside are the zero padding, whose B rows are zero and add nothing.  For
+            // 64-wide planes this takes K from 96 to 64 at 31x31 and from 128 to 64 at 51x5, and
+            // one 64-column panel then fits twice in shared memory.
+            p.clip = !nhwc && p.XT == 1 && p.Xo <= p.TW && !no_clip ? 1 : 0;
+            if (p.clip)
+                p.Ks = (std::max(std::min(p.Xi, p.TW + p.KX - 1 - p.px), 16) + 15) & ~15;
+            else
+                p.Ks = (p.TW + p.KX - 1 + mis + 15) & ~15;
             if (p.Ks > 144) continue;
             const int span = (p.XT - 1) * p.TW + p.Ks;
             p.npanels = (span + 63) / 64;
             p.NR = p.P * p.NH + p.KY - 1;
             if (p.NR > 256) continue;
             p.NI = p.KY + p.P - 1;
-            p.half_l = (p.Ks + kOff + 8) / 2;
+            // a line holds every tap a row reads: from word t0/2, Ks/2 + 1 words, t0 at most
+            // px + kOff when clipped (xb = x0 = 0, xl = 0), kOff - mis otherwise
+            p.half_l = p.clip ? ((p.px + kOff) >> 1) + (p.Ks >> 1) + 1 : (p.Ks + kOff + 8) / 2;
             p.f_words = static_cast<int>(round_up(static_cast<size_t>(p.KY) * p.half_l, 4));
             p.a_cols = ((p.Ks / 2) + 31) & ~31;
             const int ncols_d = p.XT * 8 * p.NH;
@@ -963,6 +979,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.f_words = static_cast<uint32_t>(p.f_words);
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;
         t.f_off = p.f_off;
+        t.clip = p.clip;
         t.bar_off = p.bar_off;
         t.dxp_bytes = static_cast<long long>(p.ws_out);
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));

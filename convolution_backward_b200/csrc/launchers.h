@@ -106,6 +106,7 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
     int P, TW, XT, NH, Ks, NR, NI, NB, nfb, npanels, half_l, f_words, a_col0, a_cols, na;
+    int clip;   // one tile spans the row: K clipped to the input columns inside the image
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     size_t smem, ws_in, ws_out, ws_f;
 };
