@@ -799,7 +799,7 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             // columns outside are the zero padding, whose B rows are zero and add nothing.  For
             // 64-wide planes this takes K from 96 to 64 at 31x31 and from 128 to 64 at 51x5, and
             // one 64-column panel then fits twice in shared memory.
-            p.clip = !nhwc && p.XT == 1 && p.Xo <= p.TW && !no_clip ? 1 : 0;
+            p.clip = p.XT == 1 && p.Xo <= p.TW && !no_clip ? 1 : 0;
             if (p.clip)
                 p.Ks = (std::max(std::min(p.Xi, p.TW + p.KX - 1 - p.px), 16) + 15) & ~15;
             else

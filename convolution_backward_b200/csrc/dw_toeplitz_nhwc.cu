@@ -75,6 +75,7 @@ struct ToepNArgs {
     int num_xt, num_yt, num_g, num_su;
     int a_col0, a_cols, na;
     int f16, full_plane;
+    int clip;                  // one tile spans the row: the window starts at input column 0
     int nfb;                   // filter-line buffers: 2, or 1 when two do not fit
     uint32_t panel_bytes, b_bytes, f_words, f_off, bar_off;
     long long dx_bytes;        // size of dX (index checks of the debug build)
@@ -95,7 +96,7 @@ __device__ __forceinline__ Tile decode_tile(const ToepNArgs& a, int su)
     t.cb = r / a.num_g;
     t.Y0 = yt * a.P * a.NH;
     t.x0 = xt * a.XT * a.TW;
-    t.xb = floor8(t.x0 - a.px);
+    t.xb = a.clip ? 0 : floor8(t.x0 - a.px);
     return t;
 }
 
@@ -771,6 +772,7 @@ cudaError_t launch_dw_toeplitz_nhwc(const DwArgs& a, const ToepPlan& p, cudaStre
     t.NI = p.NI;
     t.half_l = p.half_l;
     t.npanels = p.npanels;
+    t.clip = p.clip;
     t.num_xt = (p.Xo + p.XT * p.TW - 1) / (p.XT * p.TW);
     t.num_yt = (p.Yo + p.P * p.NH - 1) / (p.P * p.NH);
     t.num_g = (a.N + 7) / 8;
