@@ -205,6 +205,19 @@ bool encode_planar_tr(CUtensorMap* map, const void* base, uint64_t X, uint64_t N
     return encode_cached(enc, map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) == CUDA_SUCCESS;
 }
 
+// The planar dX of the tensor-core depthwise path as the MMA epilogue stores it:
+// dims (X, N, Y, C) of [C][Y][N][Xs], box (64, 8, 8, 1), no swizzle.
+bool encode_planar_store(CUtensorMap* map, const void* base, uint64_t X, uint64_t N, uint64_t Y, uint64_t C, uint64_t Xs)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {X, N, Y, C};
+    const cuuint64_t strides[3] = {Xs * 2, N * Xs * 2, Y * N * Xs * 2};
+    const cuuint32_t b[4] = {64, 8, 8, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode_cached(enc, map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, b, estr, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int env_int(const char* name, int dflt)
@@ -538,6 +551,10 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
                          static_cast<uint64_t>(plan.Yo), static_cast<uint64_t>(a.C), static_cast<uint64_t>(plan.Xso)) &&
         encode_nhwc_tr(&maps.unpack_dst, dX, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.H),
                        static_cast<uint64_t>(a.W), static_cast<uint64_t>(a.C), plan.orient);
+    maps.tma_epi = plan.tma_epi &&
+                   encode_planar_store(&maps.d_store, dXp, static_cast<uint64_t>(plan.Xo), static_cast<uint64_t>(a.N),
+                                       static_cast<uint64_t>(plan.Yo), static_cast<uint64_t>(a.C),
+                                       static_cast<uint64_t>(plan.Xso));
     cudaError_t e = dgrad::launch_dw_toeplitz(a, plan, maps, workspace, st->sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
 }

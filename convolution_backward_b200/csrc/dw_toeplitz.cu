@@ -94,6 +94,8 @@ struct ToepArgs {
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
     int f16;                     // operands and output are f16 (else bf16)
     int clip;                    // one tile spans the row: B starts at input column 0 (xb = 0)
+    int tma_epi;                 // the epilogue stages 8 x 8 x 64 boxes in shared memory and stores them by TMA
+    uint32_t stg_off;            // two 8 KB staging boxes (one per epilogue half)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
     long long dxp_bytes;         // size of the planar output (index checks of the debug build)
 };
@@ -205,7 +207,8 @@ __device__ __forceinline__ void unit_range(const ToepArgs& a, int* u_begin, int*
 }
 
 __global__ void __launch_bounds__(kThreadsT, 1)
-    dw_toeplitz_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ ToepArgs a)
+    dw_toeplitz_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_d,
+                       const __grid_constant__ ToepArgs a)
 {
     pdl_wait();      // the previous kernel on the stream has finished
     extern __shared__ uint8_t smem_raw[];
@@ -402,7 +405,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         bool ok = true;
         for (int u = u_begin; u < u_end; ++u) {
             const Unit t = decode_unit(a, u);
-            if (!mbar_wait(d_full, ub & 1u, abort_flag)) {
+            const bool w = mbar_wait(d_full, ub & 1u, abort_flag);
+            // with staging boxes the half's 128 threads meet at named barriers, so they agree
+            // on whether to go on
+            if (a.tma_epi ? !named_barrier_and(1 + half, 128, w) : !w) {
                 ok = false;
                 break;
             }
@@ -422,6 +428,38 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             }
             tc_fence_before();
             mbar_arrive(d_empty);   // the accumulator may be overwritten now
+            if (a.tma_epi) {
+                // P = 2, one sub-tile: the 128 threads of this half hold every row m = (p, xl)
+                // of their 32-column chunks, i.e. 8 output rows (4 h' x 2 phases) x 8 images
+                // x 64 columns of one channel's planes; they stage that box in shared memory
+                // and one thread stores it with TMA, which clips the ragged edges.
+                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + a.stg_off + half * 8192);
+                const bool issuer = lane == 0 && (warp & 3) == 2;   // warps 6 and 10
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    if (cc < nch) {
+                        if (issuer) bulk_wait_group_read<0>();   // the previous box has been read
+                        named_barrier_sync(1 + half, 128);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int hp = (2 * k) >> 3;            // h' offset inside the chunk
+                            const int img = (2 * k) & 7;
+                            const uint32_t v = pk[cc * 16 + k];
+                            stg[((2 * hp + p) * 8 + img) * 64 + xl] = static_cast<uint16_t>(v & 0xFFFFu);
+                            stg[((2 * hp + p) * 8 + img + 1) * 64 + xl] = static_cast<uint16_t>(v >> 16);
+                        }
+                        fence_proxy_async_smem();
+                        named_barrier_sync(1 + half, 128);
+                        if (issuer) {
+                            const int hp0 = (half * hcols + cc * 32) >> 3;
+                            tma_store_4d(&map_d, stg, t.x0, 8 * t.g, t.Y0 + 2 * hp0, t.c);
+                            bulk_commit_group();
+                        }
+                    }
+                }
+                ++ub;
+                continue;
+            }
             const bool full = t.Y0 + a.P * a.NH <= a.Yo && 8 * t.g + 8 <= a.N;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -459,6 +497,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             report_timeout(a.status);
             *abort_flag = 1;
         }
+        if (a.tma_epi && lane == 0 && (warp & 3) == 2) bulk_wait_group<0>();   // the boxes have been written
     }
 
     tc_fence_before();
@@ -767,6 +806,9 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     // DGRAD_TC_CLIP=0 keeps the full Toeplitz band for single-tile rows (testing and tuning).
     const char* clp = dgrad::tuning_env("DGRAD_TC_CLIP");
     const bool no_clip = clp && strcmp(clp, "0") == 0;
+    // DGRAD_TC_EPI=store keeps the epilogue's direct 16-bit stores (testing and tuning).
+    const char* epi = dgrad::tuning_env("DGRAD_TC_EPI");
+    const bool no_tma_epi = epi && strcmp(epi, "store") == 0;
     if (const char* ft = dgrad::tuning_env("DGRAD_TC_TILE"))
         if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
@@ -825,14 +867,27 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             p.b_bytes = static_cast<uint32_t>(p.npanels) * p.panel_bytes;
             bool fits = false;
             // The NHWC kernel keeps one B block (the cluster refills it) and two filter
-            // buffers, or one when two do not fit.
-            for (int nbuf = nhwc ? 2 : kMaxB; nbuf >= 1 && !fits; --nbuf) {
+            // buffers, or one when two do not fit.  The planar kernel takes two B blocks when
+            // they fit and, for P = 2 with one sub-tile, 16 KB of epilogue staging boxes when
+            // they fit as well.
+            const bool stg_ok = !nhwc && p.P == 2 && p.XT == 1 && !no_tma_epi;
+            for (int opt = 0; opt < 4 && !fits; ++opt) {
+                const int nbuf = nhwc ? 2 - opt : kMaxB - opt / 2;
+                if (nbuf < 1) break;
                 p.NB = nhwc ? 1 : nbuf;
                 p.nfb = nhwc ? nbuf : 1;
+                p.tma_epi = stg_ok && (nhwc || opt % 2 == 0) ? 1 : 0;
+                if (!nhwc && opt % 2 == 1 && !stg_ok) continue;   // the same layout as the option before
                 p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
                 p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
+                size_t end = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16;
+                p.stg_off = 0;
+                if (p.tma_epi) {
+                    p.stg_off = static_cast<uint32_t>(round_up(end, 1024));
+                    end = p.stg_off + 2 * 8192;
+                }
                 // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
-                p.smem = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16 + 1024;
+                p.smem = end + 1024;
                 if (p.smem < 120 * 1024) p.smem = 120 * 1024;
                 fits = p.smem <= 227 * 1024;
             }
@@ -980,6 +1035,8 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;
         t.f_off = p.f_off;
         t.clip = p.clip;
+        t.tma_epi = p.tma_epi && maps.tma_epi ? 1 : 0;
+        t.stg_off = p.stg_off;
         t.bar_off = p.bar_off;
         t.dxp_bytes = static_cast<long long>(p.ws_out);
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));
@@ -987,7 +1044,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         const int grid = static_cast<int>(units < num_sms ? units : num_sms);
         {
             const cudaError_t le_ = launch_kernel(dw_toeplitz_kernel, dim3(grid), dim3(kThreadsT), p.smem, stream, 1,
-                                                 map_b, t);
+                                                 map_b, maps.tma_epi ? maps.d_store : map_b, t);
             if (le_ != cudaSuccess) return le_;
         }
         e = cudaGetLastError();

@@ -107,6 +107,8 @@ struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
     int P, TW, XT, NH, Ks, NR, NI, NB, nfb, npanels, half_l, f_words, a_col0, a_cols, na;
     int clip;   // one tile spans the row: K clipped to the input columns inside the image
+    int tma_epi;          // the MMA epilogue stores staged boxes by TMA (needs ToepMaps::d_store)
+    uint32_t stg_off;     // its staging boxes in shared memory
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     size_t smem, ws_in, ws_out, ws_f;
 };
@@ -119,6 +121,10 @@ struct ToepMaps {
     CUtensorMap b;
     CUtensorMap pack_src, pack_dst, unpack_src, unpack_dst;
     bool tma_transpose;
+    // the planar dX [C][Yo][N][Xso] (dims Xo, N, Yo, C), box (64, 8, 8, 1), no swizzle:
+    // the MMA epilogue's stores when the plan has tma_epi
+    CUtensorMap d_store;
+    bool tma_epi;
 };
 bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* p, bool nhwc = false);
 // The same formulation reading NHWC dY and writing NHWC dX directly, with clusters
