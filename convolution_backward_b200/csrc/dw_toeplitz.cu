@@ -80,7 +80,7 @@ constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epi
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxA = 4;         // A buffers in tensor memory
 constexpr int kMaxB = 2;         // B blocks in shared memory
-constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 5;
+constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 7;   // + d_full, d_empty, drain, f_full[2], f_empty[2]
 
 
 struct ToepArgs {
@@ -94,6 +94,7 @@ struct ToepArgs {
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
     int f16;                     // operands and output are f16 (else bf16)
     int clip;                    // one tile spans the row: B starts at input column 0 (xb = 0)
+    int nfb;                     // filter-line buffers: 2 when they fit, so the next channel's lines load early
     int tma_epi;                 // the epilogue stages 8 x 8 x 64 boxes in shared memory and stores them by TMA
     uint32_t stg_off;            // two 8 KB staging boxes (one per epilogue half)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
 
     uint8_t* bblk = smem;                                               // NB blocks of B panels (128-byte swizzle)
-    uint32_t* fwords = reinterpret_cast<uint32_t*>(smem + a.f_off);     // padded filter lines
+    uint32_t* fwords = reinterpret_cast<uint32_t*>(smem + a.f_off);     // nfb buffers of padded filter lines
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
     uint64_t* b_full = bars;                          // [kMaxB]
     uint64_t* b_empty = bars + kMaxB;                 // [kMaxB]
@@ -224,9 +225,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     uint64_t* a_empty = a_full + kMaxA;               // [kMaxA]
     uint64_t* d_full = a_empty + kMaxA;
     uint64_t* d_empty = d_full + 1;
-    uint64_t* f_full = d_full + 2;
-    uint64_t* f_empty = d_full + 3;
-    uint64_t* drain = d_full + 4;
+    uint64_t* drain = d_full + 2;
+    uint64_t* f_full = d_full + 3;                    // [2]
+    uint64_t* f_empty = d_full + 5;                   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -249,8 +250,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         }
         mbar_init(d_full, 1);
         mbar_init(d_empty, 256);
-        mbar_init(f_full, 1);
-        mbar_init(f_empty, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&f_full[b], 1);
+            mbar_init(&f_empty[b], 128);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -267,21 +270,26 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // Per unit: the filter lines when the channel changes (one bulk copy),
-        // then the B panels (one TMA box per 64 columns) into the next B block.
+        // Per unit: the filter lines when the channel changes (one bulk copy into
+        // the next of nfb buffers, so with two the next channel's lines load while
+        // the builders still use the current ones), then the B panels (one TMA box
+        // per 64 columns) into the next B block.
         if (lane == 0) {
+            const uint32_t nfb = static_cast<uint32_t>(a.nfb);
             uint32_t ub = 0, fe = 0;
             int prev_c = -1;
             bool ok = true;
             for (int u = u_begin; u < u_end; ++u) {
                 const Unit t = decode_unit(a, u);
                 if (t.c != prev_c) {
-                    if (!mbar_wait(f_empty, (fe & 1u) ^ 1u, abort_flag)) {
+                    const uint32_t fb = fe % nfb;
+                    if (!mbar_wait(&f_empty[fb], ((fe / nfb) & 1u) ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(f_full, a.f_bytes);
-                    bulk_load(fwords, a.fpack + static_cast<int64_t>(t.c) * a.f_words, a.f_bytes, f_full);
+                    mbar_arrive_expect_tx(&f_full[fb], a.f_bytes);
+                    bulk_load(fwords + fb * a.f_words, a.fpack + static_cast<int64_t>(t.c) * a.f_words, a.f_bytes,
+                              &f_full[fb]);
                     ++fe;
                     prev_c = t.c;
                 }
@@ -307,7 +315,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                     report_timeout(a.status);
                     *abort_flag = 1;
                 }
-            if (fe > 0 && !mbar_wait(f_full, (fe - 1u) & 1u)) {
+            if (fe > 0 && !mbar_wait(&f_full[(fe - 1u) % nfb], ((fe - 1u) / nfb) & 1u)) {
                 report_timeout(a.status);
                 *abort_flag = 1;
             }
@@ -337,13 +345,15 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         const int p = m / a.TW;
         const int xl = m % a.TW;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t ab = 0, aph = 0, fe = 0;
+        const uint32_t nfb = static_cast<uint32_t>(a.nfb);
+        uint32_t ab = 0, aph = 0, fe = 0, fb = 0;
         int prev_c = -1;
         bool ok = true;
         for (int u = u_begin; u < u_end && ok; ++u) {
             const Unit t = decode_unit(a, u);
             if (t.c != prev_c) {
-                if (!mbar_wait(f_full, fe & 1u, abort_flag)) {
+                fb = fe % nfb;
+                if (!mbar_wait(&f_full[fb], (fe / nfb) & 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -353,7 +363,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             // A_i[m][j] = F[i-p][j + e], e = xb - x0 + px - xl (the same for every sub-tile);
             // padded tap index t0 = e + kOff >= 0.
             const int t0 = t.xb - t.x0 + a.px - xl + kOff;
-            const uint32_t* rowbase = fwords + (t0 >> 1);
+            const uint32_t* rowbase = fwords + fb * a.f_words + (t0 >> 1);
             const bool odd = (t0 & 1) != 0;
             for (int i = 0; i < a.NI; ++i) {
                 const uint32_t b = ab;
@@ -377,7 +387,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             }
             // Done with this channel's filter lines: let the producer replace them.
             const bool last = u + 1 >= u_end || decode_unit(a, u + 1).c != t.c;
-            if (ok && last) mbar_arrive(f_empty);
+            if (ok && last) mbar_arrive(&f_empty[fb]);
         }
         if (!ok) {
             report_timeout(a.status);
@@ -870,14 +880,22 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             // buffers, or one when two do not fit.  The planar kernel takes two B blocks when
             // they fit and, for P = 2 with one sub-tile, 16 KB of epilogue staging boxes when
             // they fit as well.
+            // Then two filter-line buffers when they fit as well.
             const bool stg_ok = !nhwc && p.P == 2 && p.XT == 1 && !no_tma_epi;
-            for (int opt = 0; opt < 4 && !fits; ++opt) {
-                const int nbuf = nhwc ? 2 - opt : kMaxB - opt / 2;
-                if (nbuf < 1) break;
-                p.NB = nhwc ? 1 : nbuf;
-                p.nfb = nhwc ? nbuf : 1;
-                p.tma_epi = stg_ok && (nhwc || opt % 2 == 0) ? 1 : 0;
-                if (!nhwc && opt % 2 == 1 && !stg_ok) continue;   // the same layout as the option before
+            for (int opt = 0; opt < 8 && !fits; ++opt) {
+                int nbuf;
+                if (nhwc) {
+                    if (opt >= 2) break;
+                    p.NB = 1;
+                    p.nfb = 2 - opt;
+                    p.tma_epi = 0;
+                } else {
+                    nbuf = kMaxB - opt / 4;                 // B blocks: 2, then 1
+                    p.NB = nbuf;
+                    p.tma_epi = stg_ok && (opt / 2) % 2 == 0 ? 1 : 0;   // staging, then none
+                    p.nfb = opt % 2 == 0 ? 2 : 1;           // filter buffers: 2, then 1
+                    if (!stg_ok && (opt / 2) % 2 == 1) continue;   // the same layouts as the options before
+                }
                 p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
                 p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
                 size_t end = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16;
@@ -1034,6 +1052,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.f_words = static_cast<uint32_t>(p.f_words);
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;
         t.f_off = p.f_off;
+        t.nfb = p.nfb;
         t.clip = p.clip;
         t.tma_epi = p.tma_epi && maps.tma_epi ? 1 : 0;
         t.stg_off = p.stg_off;
