@@ -31,9 +31,16 @@
 // atom.  Row (h', img) of B_i is row (2*h' + i, img), so B_i is that block seen
 // through a descriptor whose start moves by one atom per shift step and whose
 // row-group stride is two atoms: one TMA load of the planar input per 64
-// columns serves every shift.  A_i is a 128 x K bf16 tile written by four warps
-// straight into tensor memory (up to four buffers), so the MMA reads only B
-// from shared memory.  bf16 or f16 operands: the transposes, the filter packing
+// columns serves every shift.  A_i is Toeplitz along both of its axes at the
+// granularity of 8 x 8 core matrices when each 8-row group holds 4 columns of
+// both row phases, so for P = 2 it is stored as a table of a_slots distinct
+// 128-byte core matrices (3.75 KB at K = 64) that the MMA's no-swizzle
+// descriptor walks with overlapping strides (build_a_tables); four warps write
+// the tables into a ring of shared-memory buffers and tensor memory holds two
+// accumulator sets, so one tile's epilogue overlaps the next tile's MMAs.
+// Other tiles (P = 4, 8), or tables that do not fit, keep A_i as a 128 x K tile
+// written by the four warps straight into tensor memory (up to four buffers)
+// after one accumulator set.  bf16 or f16 operands: the transposes, the filter packing
 // and the TMA copies move 16-bit patterns, only the MMA's operand format and the
 // output rounding depend on the type.  The A builders read the channel's filter lines, padded
 // with zeros and packed two taps per word, from shared memory; the producer
@@ -57,9 +64,10 @@
 // that the image groups of one channel follow each other):
 //   warp 0      producer: filter lines (bulk copy) and B panels (TMA)
 //   warp 1      TMEM allocation (512 columns) and the MMA issuer (one lane)
-//   warps 2-5   A builders: each thread writes its row of A_i with tcgen05.st
-//   warps 6-13  epilogue: two warps per TMEM lane quarter drain the accumulator
-//               into registers, release it, then round to bf16 and store planes
+//   warps 2-5   A builders: A_i tables in shared memory, or each thread's row of
+//               A_i in tensor memory with tcgen05.st
+//   warps 6-13  epilogue: two warps per TMEM lane quarter drain an accumulator
+//               set into registers, release it, then round to bf16 and store planes
 // Every wait is bounded; a timeout is recorded in the status word, raises the
 // CTA's abort flag, lets issued copies and MMAs finish and frees TMEM.
 #include <algorithm>
@@ -78,9 +86,9 @@ using namespace toep;
 
 constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxA = 4;         // A buffers in tensor memory
+constexpr int kMaxA = 6;         // A buffers (tensor memory: at most 4; shared memory: at most 6)
 constexpr int kMaxB = 2;         // B blocks in shared memory
-constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 7;   // + d_full, d_empty, drain, f_full[2], f_empty[2]
+constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 9;   // + d_full[2], d_empty[2], drain, f_full[2], f_empty[2]
 
 
 struct ToepArgs {
@@ -92,6 +100,10 @@ struct ToepArgs {
     int P, TW, XT, NH, Ks, NR, NI, half_l, NB;
     int num_xt, num_yt, num_g, num_units;
     int a_col0, a_cols, na;      // TMEM column of A buffer 0, columns per buffer, buffer count
+    int a_smem;                  // A_i lives in shared memory as a table of 8 x 8 core matrices (below)
+    int a_slots;                 // 128-byte core matrices per table: 16 + P*(Ks/8 - 1)
+    uint32_t a_off, a_bytes;     // offset of table 0 and the stride between tables
+    int nacc;                    // accumulator sets in tensor memory: 2 when A is in shared memory
     int f16;                     // operands and output are f16 (else bf16)
     int clip;                    // one tile spans the row: B starts at input column 0 (xb = 0)
     int nfb;                     // filter-line buffers: 2 when they fit, so the next channel's lines load early
@@ -126,18 +138,39 @@ struct MmaCtx {
     uint64_t* b_empty;
     uint64_t* a_full;
     uint64_t* a_empty;
-    uint64_t* d_full;
-    uint64_t* d_empty;
+    uint64_t* d_full;            // [nacc]
+    uint64_t* d_empty;           // [nacc]
     const volatile int* abort_flag;
     uint32_t tmem_base;
     uint32_t bblk_addr;
+    uint32_t a_addr;             // A table 0 (A in shared memory)
 };
+
+// The MMAs of one shift step with A_i in shared memory: as issue_step, with the
+// A descriptor advancing by two core matrices along K (2 * LBO = 256*P bytes)
+// per 16-deep step.
+template <int KQ, int XT>
+__device__ __forceinline__ void issue_step_ss(const uint32_t (&d_tmem)[4], uint64_t a_desc_i, uint64_t desc_i,
+                                              uint32_t pb16, uint32_t a_q16, uint32_t idesc, bool first)
+{
+    constexpr int TW = 64 / XT;
+#pragma unroll
+    for (int q = 0; q < KQ; ++q) {
+#pragma unroll
+        for (int sx = 0; sx < XT; ++sx) {
+            const int col = sx * TW + 16 * q;
+            const uint64_t bd = desc_i + static_cast<uint64_t>((col >> 6) * pb16 + ((col & 63) >> 4) * 2);
+            umma_f16(d_tmem[sx], a_desc_i + static_cast<uint64_t>(q) * a_q16, bd, idesc,
+                     (first && q == 0) ? 0u : 1u);
+        }
+    }
+}
 
 // The MMA issuer's loop over its units, compiled per (16-deep steps per tile,
 // sub-tiles) so that each shift step is a short straight run of MMAs: buffer
 // indices and phases advance incrementally and the B descriptor moves by one
 // swizzle atom per step.  Returns false when a wait gave up.
-template <int KQ, int XT>
+template <int KQ, int XT, bool AS>
 __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
 {
     const int ncol_sub = 8 * a.NH;
@@ -145,58 +178,160 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
         a.f16 ? idesc_f16_f32(128, ncol_sub, /*b_mn_major=*/false) : idesc_bf16_f32(128, ncol_sub, false);
     const uint32_t sbo = static_cast<uint32_t>(a.P) * 1024u;
     const uint32_t pb16 = a.panel_bytes >> 4;
+    // accumulator set s of sub-tile sx at column s*XT*ncol_sub + sx*ncol_sub
+    const uint32_t set_cols = static_cast<uint32_t>(a.XT * ncol_sub);
     uint32_t d_tmem[4];
 #pragma unroll
     for (int sx = 0; sx < 4; ++sx) d_tmem[sx] = c.tmem_base + static_cast<uint32_t>(sx * ncol_sub);
     const uint32_t a_first = c.tmem_base + static_cast<uint32_t>(a.a_col0);
-    const uint32_t a_last = a_first + static_cast<uint32_t>((a.na - 1) * a.a_cols);
-    uint32_t bb = 0, bph = 0, ab = 0, aph = 0, dph = 0;
+    // A tables: no swizzle, K-major; core matrix (g, kc) at slot g + P*kc, i.e. SBO = 128
+    // bytes between 8-row groups and LBO = 128*P bytes between 8-column steps of K
+    const uint64_t a_desc0 = noswz_desc(c.a_addr, 128u * static_cast<uint32_t>(a.P), 128u);
+    const uint32_t a_q16 = 16u * static_cast<uint32_t>(a.P);
+    const uint32_t a_buf16 = a.a_bytes >> 4;
+    // Everything the loop reads lives in registers: the MMA and commit statements clobber
+    // memory, so fields read through `a` or `c` would be loaded again after each of them,
+    // and this single thread's issue rate bounds the tensor pipe's.
+    const int NI = a.NI;
+    const uint32_t na = static_cast<uint32_t>(a.na), nb = static_cast<uint32_t>(a.NB);
+    const uint32_t a_cols = static_cast<uint32_t>(a.a_cols), b_bytes = a.b_bytes, bblk_addr = c.bblk_addr;
+    const bool two_acc = a.nacc == 2;
+    uint64_t* const b_full = c.b_full;
+    uint64_t* const b_empty = c.b_empty;
+    uint64_t* const a_full = c.a_full;
+    uint64_t* const a_empty = c.a_empty;
+    uint64_t* const d_full = c.d_full;
+    uint64_t* const d_empty = c.d_empty;
+    const volatile int* const abort_flag = c.abort_flag;
+    uint32_t bb = 0, bph = 0, ab = 0, aph = 0;
     uint32_t a_tmem = a_first;
     for (int u = u_begin; u < u_end; ++u) {
-        if (!mbar_wait(&c.b_full[bb], bph, c.abort_flag) || !mbar_wait(c.d_empty, dph ^ 1u, c.abort_flag))
+        const uint32_t k = static_cast<uint32_t>(u - u_begin);
+        const uint32_t acc = two_acc ? (k & 1u) : 0u;
+        const uint32_t use = two_acc ? (k >> 1) : k;
+        if (!mbar_wait(&b_full[bb], bph, abort_flag) || !mbar_wait(&d_empty[acc], (use & 1u) ^ 1u, abort_flag))
             return false;
         tc_fence_after();
-        uint64_t desc = sw128_desc(c.bblk_addr + bb * a.b_bytes, 16, sbo);
-        for (int i = 0; i < a.NI; ++i) {
-            if (!mbar_wait(&c.a_full[ab], aph, c.abort_flag)) return false;
+        uint32_t d_set[4];
+#pragma unroll
+        for (int sx = 0; sx < 4; ++sx) d_set[sx] = d_tmem[sx] + acc * set_cols;
+        uint64_t desc = sw128_desc(bblk_addr + bb * b_bytes, 16, sbo);
+        uint64_t a_desc = a_desc0 + static_cast<uint64_t>(ab * a_buf16);
+        for (int i = 0; i < NI; ++i) {
+            if (!mbar_wait(&a_full[ab], aph, abort_flag)) return false;
             tc_fence_after();
-            issue_step<KQ, XT>(d_tmem, a_tmem, desc, pb16, idesc, i == 0);
-            umma_commit(&c.a_empty[ab]);   // A buffer free once these MMAs have read it
-            desc += 64;                     // next shift step: one 1024-byte atom
-            if (a_tmem == a_last) {
+            if (AS)
+                issue_step_ss<KQ, XT>(d_set, a_desc, desc, pb16, a_q16, idesc, i == 0);
+            else
+                issue_step<KQ, XT>(d_set, a_tmem, desc, pb16, idesc, i == 0);
+            umma_commit(&a_empty[ab]);   // A buffer free once these MMAs have read it
+            desc += 64;                   // next shift step: one 1024-byte atom
+            if (++ab == na) {
                 a_tmem = a_first;
+                a_desc = a_desc0;
                 ab = 0;
                 aph ^= 1u;
             } else {
-                a_tmem += static_cast<uint32_t>(a.a_cols);
-                ++ab;
+                a_tmem += a_cols;
+                a_desc += a_buf16;
             }
         }
-        umma_commit(c.d_full);
-        umma_commit(&c.b_empty[bb]);
-        if (++bb == static_cast<uint32_t>(a.NB)) {
+        umma_commit(&d_full[acc]);
+        umma_commit(&b_empty[bb]);
+        if (++bb == nb) {
             bb = 0;
             bph ^= 1u;
         }
-        dph ^= 1u;
     }
     return true;
 }
 
-template <int XT>
+template <int XT, bool AS>
 __device__ __forceinline__ bool mma_role_x(int kq, const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
 {
     switch (kq) {
-    case 1: return mma_role<1, XT>(a, c, u_begin, u_end);
-    case 2: return mma_role<2, XT>(a, c, u_begin, u_end);
-    case 3: return mma_role<3, XT>(a, c, u_begin, u_end);
-    case 4: return mma_role<4, XT>(a, c, u_begin, u_end);
-    case 5: return mma_role<5, XT>(a, c, u_begin, u_end);
-    case 6: return mma_role<6, XT>(a, c, u_begin, u_end);
-    case 7: return mma_role<7, XT>(a, c, u_begin, u_end);
-    case 8: return mma_role<8, XT>(a, c, u_begin, u_end);
-    default: return mma_role<9, XT>(a, c, u_begin, u_end);
+    case 1: return mma_role<1, XT, AS>(a, c, u_begin, u_end);
+    case 2: return mma_role<2, XT, AS>(a, c, u_begin, u_end);
+    case 3: return mma_role<3, XT, AS>(a, c, u_begin, u_end);
+    case 4: return mma_role<4, XT, AS>(a, c, u_begin, u_end);
+    case 5: return mma_role<5, XT, AS>(a, c, u_begin, u_end);
+    case 6: return mma_role<6, XT, AS>(a, c, u_begin, u_end);
+    case 7: return mma_role<7, XT, AS>(a, c, u_begin, u_end);
+    case 8: return mma_role<8, XT, AS>(a, c, u_begin, u_end);
+    default: return mma_role<9, XT, AS>(a, c, u_begin, u_end);
     }
+}
+
+// A_i in shared memory (P = 2).  Row m of the MMA tile is m = 8g + r with r = 4p
+// + xr: output row phase p, output column xl = 4*(15 - g) + xr.  Core matrix (g,
+// kc) of A_i (rows 8g.., K columns 8kc..) then holds, in row r and column e,
+// F[i-p][c0 + 8kc + e - xl] with c0 = xb - x0 + px, which depends on g and kc only
+// through 4*(g + 2kc): every core matrix is one of a_slots = 16 + 2*(K/8 - 1)
+// distinct 128-byte blocks, and block s = g + 2kc holds in row r taps w(s, xr) =
+// c0 - 60 + 4s - xr .. +7 of line i-p.  The MMA's descriptor walks the blocks with
+// SBO = 128 bytes (8-row groups) and LBO = 256 bytes (8-column steps of K), so A_i
+// takes a_slots*128 bytes (3.75 KB at K = 64) instead of a 16 KB tile.  A builder
+// thread owns pairs (s, xr), q = tb and tb + 128: row xr of block s takes line i's
+// window, row 4 + xr line i-1's, which is the window the thread loaded for row xr
+// at the step before, so each step reads one window per pair.  A line outside the
+// filter reads as zeros.  Returns false when a wait gave up.
+constexpr int kMaxAPairs = 2;   // (block, column) pairs per builder thread: a_slots <= 64
+__device__ __forceinline__ uint4 load_window(const uint32_t* src, bool odd)
+{
+    const uint32_t w0 = src[0], w1 = src[1], w2 = src[2], w3 = src[3];
+    const uint32_t w4 = odd ? src[4] : 0u;
+    const uint32_t sh = odd ? 16u : 0u;
+    return make_uint4(__funnelshift_r(w0, w1, sh), __funnelshift_r(w1, w2, sh), __funnelshift_r(w2, w3, sh),
+                      __funnelshift_r(w3, w4, sh));
+}
+
+__device__ __forceinline__ bool build_a_tables(const ToepArgs& a, const Unit& t, const uint32_t* lines,
+                                               uint8_t* tables, uint64_t* a_full, uint64_t* a_empty,
+                                               const volatile int* abort_flag, int tb, uint32_t& ab, uint32_t& aph)
+{
+    const int c0 = t.xb - t.x0 + a.px;
+    const int npairs = 4 * a.a_slots;
+    const int NI = a.NI, KY = a.KY, half_l = a.half_l;   // registers (the loop's statements clobber memory)
+    const uint32_t na = static_cast<uint32_t>(a.na), a_bytes = a.a_bytes;
+    int wo[kMaxAPairs], off[kMaxAPairs];
+    bool odd[kMaxAPairs];
+    uint4 prev[kMaxAPairs];
+#pragma unroll
+    for (int k = 0; k < kMaxAPairs; ++k) {
+        const int q = tb + 128 * k;
+        const int sl = q >> 2;
+        const int xr = q & 3;
+        const int t0 = c0 - 60 + 4 * sl - xr + kOff;   // >= 2: c0 >= -7, kOff = 72
+        wo[k] = t0 >> 1;
+        odd[k] = (t0 & 1) != 0;
+        off[k] = 128 * sl + 16 * xr;
+        prev[k] = make_uint4(0u, 0u, 0u, 0u);          // line -1
+    }
+    for (int i = 0; i < NI; ++i) {
+        uint4 cur[kMaxAPairs];
+#pragma unroll
+        for (int k = 0; k < kMaxAPairs; ++k) {
+            cur[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (tb + 128 * k < npairs && i < KY) cur[k] = load_window(lines + i * half_l + wo[k], odd[k]);
+        }
+        if (!mbar_wait(&a_empty[ab], aph ^ 1u, abort_flag)) return false;
+        uint8_t* tab = tables + ab * a_bytes;
+#pragma unroll
+        for (int k = 0; k < kMaxAPairs; ++k) {
+            if (tb + 128 * k < npairs) {
+                *reinterpret_cast<uint4*>(tab + off[k]) = cur[k];        // phase 0: line i
+                *reinterpret_cast<uint4*>(tab + off[k] + 64) = prev[k];  // phase 1: line i-1
+            }
+            prev[k] = cur[k];
+        }
+        fence_proxy_async_smem();   // the tensor core reads the table through the async proxy
+        mbar_arrive(&a_full[ab]);
+        if (++ab == na) {
+            ab = 0;
+            aph ^= 1u;
+        }
+    }
+    return true;
 }
 
 // Units [u_begin, u_end) of this CTA: a contiguous range, so that the tiles of
@@ -223,11 +358,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     uint64_t* b_empty = bars + kMaxB;                 // [kMaxB]
     uint64_t* a_full = bars + 2 * kMaxB;              // [kMaxA]
     uint64_t* a_empty = a_full + kMaxA;               // [kMaxA]
-    uint64_t* d_full = a_empty + kMaxA;
-    uint64_t* d_empty = d_full + 1;
-    uint64_t* drain = d_full + 2;
-    uint64_t* f_full = d_full + 3;                    // [2]
-    uint64_t* f_empty = d_full + 5;                   // [2]
+    uint64_t* d_full = a_empty + kMaxA;               // [2]
+    uint64_t* d_empty = d_full + 2;                   // [2]
+    uint64_t* drain = d_full + 4;
+    uint64_t* f_full = d_full + 5;                    // [2]
+    uint64_t* f_empty = d_full + 7;                   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -248,8 +383,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             mbar_init(&a_full[b], 128);
             mbar_init(&a_empty[b], 1);
         }
-        mbar_init(d_full, 1);
-        mbar_init(d_empty, 256);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&d_full[b], 1);
+            mbar_init(&d_empty[b], 256);
+        }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&f_full[b], 1);
             mbar_init(&f_empty[b], 128);
@@ -323,11 +460,18 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            MmaCtx ctx{b_full, b_empty, a_full, a_empty, d_full, d_empty, abort_flag, tmem_base, smem_u32(bblk)};
+            MmaCtx ctx{b_full,    b_empty,        a_full,   a_empty, d_full, d_empty, abort_flag, tmem_base,
+                       smem_u32(bblk), smem_u32(smem + a.a_off)};
             const int kq = a.Ks >> 4;
-            const bool ok = a.XT == 1   ? mma_role_x<1>(kq, a, ctx, u_begin, u_end)
-                            : a.XT == 2 ? mma_role_x<2>(kq, a, ctx, u_begin, u_end)
-                                        : mma_role_x<4>(kq, a, ctx, u_begin, u_end);
+            bool ok;
+            if (a.a_smem)
+                ok = a.XT == 1   ? mma_role_x<1, true>(kq, a, ctx, u_begin, u_end)
+                     : a.XT == 2 ? mma_role_x<2, true>(kq, a, ctx, u_begin, u_end)
+                                 : mma_role_x<4, true>(kq, a, ctx, u_begin, u_end);
+            else
+                ok = a.XT == 1   ? mma_role_x<1, false>(kq, a, ctx, u_begin, u_end)
+                     : a.XT == 2 ? mma_role_x<2, false>(kq, a, ctx, u_begin, u_end)
+                                 : mma_role_x<4, false>(kq, a, ctx, u_begin, u_end);
             if (!ok) {
                 report_timeout(a.status);
                 *abort_flag = 1;
@@ -360,12 +504,23 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 ++fe;
                 prev_c = t.c;
             }
+            if (a.a_smem) {
+                ok = build_a_tables(a, t, fwords + fb * a.f_words, smem + a.a_off, a_full, a_empty, abort_flag,
+                                    threadIdx.x - 64, ab, aph);
+                const bool last = u + 1 >= u_end || decode_unit(a, u + 1).c != t.c;
+                if (ok && last) mbar_arrive(&f_empty[fb]);
+                continue;
+            }
             // A_i[m][j] = F[i-p][j + e], e = xb - x0 + px - xl (the same for every sub-tile);
             // padded tap index t0 = e + kOff >= 0.
             const int t0 = t.xb - t.x0 + a.px - xl + kOff;
             const uint32_t* rowbase = fwords + fb * a.f_words + (t0 >> 1);
             const bool odd = (t0 & 1) != 0;
-            for (int i = 0; i < a.NI; ++i) {
+            // registers for the loop (its statements clobber memory)
+            const int NI = a.NI, KY = a.KY, kq = a.Ks >> 4, half_l = a.half_l;
+            const uint32_t a_base = tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0);
+            const uint32_t a_cols = static_cast<uint32_t>(a.a_cols);
+            for (int i = 0; i < NI; ++i) {
                 const uint32_t b = ab;
                 if (!mbar_wait(&a_empty[b], aph ^ 1u, abort_flag)) {
                     ok = false;
@@ -373,10 +528,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 }
                 tc_fence_after();
                 const int ry = i - p;
-                const uint32_t taddr =
-                    tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0) + b * static_cast<uint32_t>(a.a_cols);
-                const bool nonzero = ry >= 0 && ry < a.KY;
-                store_a(a.Ks >> 4, taddr, rowbase + (nonzero ? ry : 0) * a.half_l, odd, nonzero);
+                const uint32_t taddr = a_base + b * a_cols;
+                const bool nonzero = ry >= 0 && ry < KY;
+                store_a(kq, taddr, rowbase + (nonzero ? ry : 0) * half_l, odd, nonzero);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&a_full[b]);
@@ -400,8 +554,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         const int quarter = warp & 3;
         const int half = (warp - 6) >> 2;
         const int m = quarter * 32 + lane;
-        const int p = m / a.TW;
-        const int xl = m % a.TW;
+        // row m of the accumulator: output row phase p and column xl (see build_a_tables
+        // for the order of the rows when A is in shared memory)
+        const int R = 8 / a.P;
+        const int p = a.a_smem ? (m & 7) / R : m / a.TW;
+        const int xl = a.a_smem ? R * (15 - (m >> 3)) + (m & 7) % R : m % a.TW;
+        const uint32_t set_cols = static_cast<uint32_t>(a.XT * ncol_sub);
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
         const int hcols = (a.XT * ncol_sub) >> 1;   // columns per half: at most 128
         const int nch = hcols >> 5;                  // 32-column chunks per half: 1 .. 4
@@ -415,7 +573,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         bool ok = true;
         for (int u = u_begin; u < u_end; ++u) {
             const Unit t = decode_unit(a, u);
-            const bool w = mbar_wait(d_full, ub & 1u, abort_flag);
+            const uint32_t acc = a.nacc == 2 ? (ub & 1u) : 0u;
+            const uint32_t use = a.nacc == 2 ? (ub >> 1) : ub;
+            const bool w = mbar_wait(&d_full[acc], use & 1u, abort_flag);
             // with staging boxes the half's 128 threads meet at named barriers, so they agree
             // on whether to go on
             if (a.tma_epi ? !named_barrier_and(1 + half, 128, w) : !w) {
@@ -428,7 +588,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             for (int cc = 0; cc < 4; ++cc) {
                 if (cc < nch) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(half * hcols + cc * 32), v);
+                    tmem_ld_32x32b_x32(
+                        tmem_base + lane_addr + acc * set_cols + static_cast<uint32_t>(half * hcols + cc * 32), v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
@@ -437,7 +598,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(d_empty);   // the accumulator may be overwritten now
+            mbar_arrive(&d_empty[acc]);   // the accumulator may be overwritten now
             if (a.tma_epi) {
                 // P = 2, one sub-tile: the 128 threads of this half hold every row m = (p, xl)
                 // of their 32-column chunks, i.e. 8 output rows (4 h' x 2 phases) x 8 images
@@ -819,6 +980,11 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     // DGRAD_TC_EPI=store keeps the epilogue's direct 16-bit stores (testing and tuning).
     const char* epi = dgrad::tuning_env("DGRAD_TC_EPI");
     const bool no_tma_epi = epi && strcmp(epi, "store") == 0;
+    // DGRAD_TC_A=tmem keeps A_i in tensor memory, written by the builders; DGRAD_TC_A=smem takes
+    // the shared-memory tables whenever they fit (testing and tuning).
+    const char* amode = dgrad::tuning_env("DGRAD_TC_A");
+    const bool no_a_smem = amode && strcmp(amode, "tmem") == 0;
+    const bool force_a_smem = amode && strcmp(amode, "smem") == 0;
     if (const char* ft = dgrad::tuning_env("DGRAD_TC_TILE"))
         if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
@@ -869,45 +1035,69 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             p.a_cols = ((p.Ks / 2) + 31) & ~31;
             const int ncols_d = p.XT * 8 * p.NH;
             if (ncols_d > 256 || (ncols_d / 2) % 32 != 0) continue;
+            // The planar kernel keeps A_i in shared memory (tables of core matrices, see
+            // build_a_tables) for P = 2 when a table has at most 32*kMaxAPairs blocks, a
+            // layout with two or more tables fits and a tile runs at least 16 shift steps;
+            // tensor memory then holds two accumulator sets.  Otherwise A_i goes to tensor
+            // memory after one accumulator set.  Measured on B200 (bench suite): 31x31 (32
+            // steps) 109.6 us with tables against 113.4 us in tensor memory, 51x5 and 5x51 (6
+            // steps) 60.9 us against 59.6 us.
+            p.a_slots = 16 + p.P * (p.Ks / 8 - 1);
+            p.a_bytes = static_cast<uint32_t>(p.a_slots) * 128u;
             p.a_col0 = ncols_d;
-            p.na = (static_cast<int>(kTmemCols) - p.a_col0) / p.a_cols;
-            if (p.na < 2) continue;
-            if (p.na > kMaxA) p.na = kMaxA;
+            const int na_tmem = std::min((static_cast<int>(kTmemCols) - p.a_col0) / p.a_cols, 4);
             p.panel_bytes = static_cast<uint32_t>(p.NR) * 1024u;
             p.b_bytes = static_cast<uint32_t>(p.npanels) * p.panel_bytes;
             bool fits = false;
             // The NHWC kernel keeps one B block (the cluster refills it) and two filter
             // buffers, or one when two do not fit.  The planar kernel takes two B blocks when
             // they fit and, for P = 2 with one sub-tile, 16 KB of epilogue staging boxes when
-            // they fit as well.
-            // Then two filter-line buffers when they fit as well.
+            // they fit as well; then two filter-line buffers when they fit as well; with A in
+            // shared memory, 4, 3 or 2 tables.
             const bool stg_ok = !nhwc && p.P == 2 && p.XT == 1 && !no_tma_epi;
-            for (int opt = 0; opt < 8 && !fits; ++opt) {
-                int nbuf;
-                if (nhwc) {
-                    if (opt >= 2) break;
-                    p.NB = 1;
-                    p.nfb = 2 - opt;
-                    p.tma_epi = 0;
-                } else {
-                    nbuf = kMaxB - opt / 4;                 // B blocks: 2, then 1
-                    p.NB = nbuf;
-                    p.tma_epi = stg_ok && (opt / 2) % 2 == 0 ? 1 : 0;   // staging, then none
-                    p.nfb = opt % 2 == 0 ? 2 : 1;           // filter buffers: 2, then 1
-                    if (!stg_ok && (opt / 2) % 2 == 1) continue;   // the same layouts as the options before
+            const bool smem_a_ok = !nhwc && !no_a_smem && p.P == 2 && p.a_slots * 4 <= 128 * kMaxAPairs &&
+                                   (p.NI >= 16 || force_a_smem);
+            for (int amode = smem_a_ok ? 0 : 1; amode < 2 && !fits; ++amode) {
+                p.a_smem = amode == 0 ? 1 : 0;
+                p.nacc = p.a_smem ? 2 : 1;
+                p.na = na_tmem;
+                if (!p.a_smem && p.na < 2) break;
+                const int n_na = p.a_smem ? 3 : 1;
+                for (int opt = 0; opt < 8 * n_na && !fits; ++opt) {
+                    const int o = opt / n_na;
+                    if (nhwc) {
+                        if (o >= 2) break;
+                        p.NB = 1;
+                        p.nfb = 2 - o;
+                        p.tma_epi = 0;
+                    } else {
+                        p.NB = kMaxB - o / 4;                   // B blocks: 2, then 1
+                        p.tma_epi = stg_ok && (o / 2) % 2 == 0 ? 1 : 0;   // staging, then none
+                        p.nfb = o % 2 == 0 ? 2 : 1;             // filter buffers: 2, then 1
+                        if (!stg_ok && (o / 2) % 2 == 1) continue;   // the same layouts as the options before
+                        if (p.a_smem) p.na = 4 - opt % n_na;
+                    }
+                    p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
+                    p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
+                    size_t end = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16;
+                    p.a_off = 0;
+                    if (p.a_smem) {
+                        // plus slack, so that the descriptor's addresses would stay inside the
+                        // allocation even with its two strides exchanged
+                        p.a_off = static_cast<uint32_t>(round_up(end, 128));
+                        end = p.a_off + static_cast<size_t>(p.na) * p.a_bytes +
+                              128u * (p.P - 1) * static_cast<size_t>(std::max(0, 16 - p.Ks / 8));
+                    }
+                    p.stg_off = 0;
+                    if (p.tma_epi) {
+                        p.stg_off = static_cast<uint32_t>(round_up(end, 1024));
+                        end = p.stg_off + 2 * 8192;
+                    }
+                    // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
+                    p.smem = end + 1024;
+                    if (p.smem < 120 * 1024) p.smem = 120 * 1024;
+                    fits = p.smem <= 227 * 1024;
                 }
-                p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
-                p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
-                size_t end = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16;
-                p.stg_off = 0;
-                if (p.tma_epi) {
-                    p.stg_off = static_cast<uint32_t>(round_up(end, 1024));
-                    end = p.stg_off + 2 * 8192;
-                }
-                // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
-                p.smem = end + 1024;
-                if (p.smem < 120 * 1024) p.smem = 120 * 1024;
-                fits = p.smem <= 227 * 1024;
             }
             if (!fits) continue;
             const long long num_yt = (p.Yo + p.P * p.NH - 1) / (p.P * p.NH);
@@ -1045,6 +1235,11 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.a_col0 = p.a_col0;
         t.a_cols = p.a_cols;
         t.na = p.na;
+        t.a_smem = p.a_smem;
+        t.a_slots = p.a_slots;
+        t.a_off = p.a_off;
+        t.a_bytes = p.a_bytes;
+        t.nacc = p.nacc;
         t.f16 = a.f16 ? 1 : 0;
         t.panel_bytes = p.panel_bytes;
         t.b_bytes = p.b_bytes;
@@ -1061,11 +1256,9 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));
         if (e != cudaSuccess) return e;
         const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-        {
-            const cudaError_t le_ = launch_kernel(dw_toeplitz_kernel, dim3(grid), dim3(kThreadsT), p.smem, stream, 1,
-                                                 map_b, maps.tma_epi ? maps.d_store : map_b, t);
-            if (le_ != cudaSuccess) return le_;
-        }
+        e = launch_kernel(dw_toeplitz_kernel, dim3(grid), dim3(kThreadsT), p.smem, stream, 1, map_b,
+                          maps.tma_epi ? maps.d_store : map_b, t);
+        if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

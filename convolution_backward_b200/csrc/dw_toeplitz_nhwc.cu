@@ -300,32 +300,43 @@ __device__ __noinline__ bool mma_role_n(const ToepNArgs& a, const MmaCtxN& c, in
     for (int sx = 0; sx < 4; ++sx) d_tmem[sx] = c.tmem_base + static_cast<uint32_t>(sx * ncol_sub);
     const uint32_t a_first = c.tmem_base + static_cast<uint32_t>(a.a_col0);
     const uint32_t a_last = a_first + static_cast<uint32_t>((a.na - 1) * a.a_cols);
+    // The loop reads registers only: the MMA and commit statements clobber memory, so
+    // fields read through `a` or `c` would be loaded again after each of them, and this
+    // single thread's issue rate bounds the tensor pipe's.
+    const int NI = a.NI;
+    const uint32_t a_cols = static_cast<uint32_t>(a.a_cols), bblk_addr = c.bblk_addr;
+    uint64_t* const b_full = c.b_full;
+    uint64_t* const d_empty = c.d_empty;
+    uint64_t* const d_full = c.d_full;
+    uint64_t* const a_full = c.a_full;
+    uint64_t* const a_empty = c.a_empty;
+    uint64_t* const bfree = c.bfree;
+    const volatile int* const abort_flag = c.abort_flag;
     uint32_t ab = 0, aph = 0;
     uint32_t a_tmem = a_first;
     for (int t = 0; t < ntiles; ++t) {
         const uint32_t ph = static_cast<uint32_t>(t) & 1u;
-        if (!mbar_wait_remote(c.b_full, ph, c.abort_flag) || !mbar_wait(c.d_empty, ph ^ 1u, c.abort_flag))
-            return false;
+        if (!mbar_wait_remote(b_full, ph, abort_flag) || !mbar_wait(d_empty, ph ^ 1u, abort_flag)) return false;
         fence_proxy_async_smem();
         tc_fence_after();
-        uint64_t desc = sw128_desc(c.bblk_addr, 16, sbo);
-        for (int i = 0; i < a.NI; ++i) {
-            if (!mbar_wait(&c.a_full[ab], aph, c.abort_flag)) return false;
+        uint64_t desc = sw128_desc(bblk_addr, 16, sbo);
+        for (int i = 0; i < NI; ++i) {
+            if (!mbar_wait(&a_full[ab], aph, abort_flag)) return false;
             tc_fence_after();
             issue_step<KQ, XT>(d_tmem, a_tmem, desc, pb16, idesc, i == 0);
-            umma_commit(&c.a_empty[ab]);
+            umma_commit(&a_empty[ab]);
             desc += 64;   // next shift step: one 1024-byte atom
             if (a_tmem == a_last) {
                 a_tmem = a_first;
                 ab = 0;
                 aph ^= 1u;
             } else {
-                a_tmem += static_cast<uint32_t>(a.a_cols);
+                a_tmem += a_cols;
                 ++ab;
             }
         }
-        umma_commit(c.d_full);
-        umma_commit_mc(c.bfree, static_cast<uint16_t>((1u << kCluster) - 1u));
+        umma_commit(d_full);
+        umma_commit_mc(bfree, static_cast<uint16_t>((1u << kCluster) - 1u));
     }
     return true;
 }
@@ -406,7 +417,11 @@ __device__ __forceinline__ void abuild_role(const ToepNArgs& a, const KCtx& k, i
         const int t0 = tl.xb - tl.x0 + a.px - xl + kOff;
         const uint32_t* rowbase = fbuf + (t0 >> 1);
         const bool odd = (t0 & 1) != 0;
-        for (int i = 0; i < a.NI; ++i) {
+        // registers for the loop (its statements clobber memory)
+        const int NI = a.NI, KY = a.KY, kq = a.Ks >> 4, half_l = a.half_l;
+        const uint32_t a_base = tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0);
+        const uint32_t a_cols = static_cast<uint32_t>(a.a_cols);
+        for (int i = 0; i < NI; ++i) {
             const uint32_t b = ab;
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&a_empty[b], aph ^ 1u, abort_flag))) {
                 ok = false;
@@ -414,10 +429,9 @@ __device__ __forceinline__ void abuild_role(const ToepNArgs& a, const KCtx& k, i
             }
             tc_fence_after();
             const int ry = i - p;
-            const uint32_t taddr =
-                tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0) + b * static_cast<uint32_t>(a.a_cols);
-            const bool nonzero = ry >= 0 && ry < a.KY;
-            store_a(a.Ks >> 4, taddr, rowbase + (nonzero ? ry : 0) * a.half_l, odd, nonzero);
+            const uint32_t taddr = a_base + b * a_cols;
+            const bool nonzero = ry >= 0 && ry < KY;
+            store_a(kq, taddr, rowbase + (nonzero ? ry : 0) * half_l, odd, nonzero);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&a_full[b]);

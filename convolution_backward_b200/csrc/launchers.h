@@ -107,6 +107,8 @@ struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
     int P, TW, XT, NH, Ks, NR, NI, NB, nfb, npanels, half_l, f_words, a_col0, a_cols, na;
     int clip;   // one tile spans the row: K clipped to the input columns inside the image
+    int a_smem, a_slots, nacc;   // A_i as shared-memory tables of a_slots core matrices; accumulator sets
+    uint32_t a_off, a_bytes;     // offset of the first A table and the stride between them
     int tma_epi;          // the MMA epilogue stores staged boxes by TMA (needs ToepMaps::d_store)
     uint32_t stg_off;     // its staging boxes in shared memory
     uint32_t panel_bytes, b_bytes, f_off, bar_off;

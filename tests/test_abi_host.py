@@ -231,7 +231,10 @@ def test_depthwise_tc_validation_and_workspace_size():
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(empty), ctypes.byref(nb)) == OK and nb.value == 0
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 32, 32)),
                                           ctypes.byref(nb)) == OK
-    refused = [cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 6, 6),     # 64x64 at pad 6: K = 144, too large a tile
+    # 64x64 at pad 6 on 64x64 planes: the input rows are 13 columns wide, so K is clipped to 16
+    assert L.dgrad_depthwise_tc_workspace(ctypes.byref(cb.Problem(1, 64, 64, 32, 32, 64, 64, 1, 6, 6)),
+                                          ctypes.byref(nb)) == OK
+    refused = [cb.Problem(1, 128, 128, 32, 32, 64, 64, 1, 6, 6),   # 64x64 at pad 6, 128 wide: K = 144, no tile fits
                cb.Problem(1, 64, 64, 32, 32, 7, 7, 2, 3, 3),       # stride 2
                cb.Problem(1, 64, 64, 32, 64, 7, 7, 1, 3, 3),       # depth multiplier 2
                cb.Problem(1, 64, 64, 32, 32, 7, 7, 1, 7, 3)]       # pad beyond KH-1

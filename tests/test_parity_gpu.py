@@ -513,6 +513,71 @@ def test_depthwise_tensor_core_tile_shapes(tile, monkeypatch):
     cb.check_status()
 
 
+TC_A_TMEM = [q for q in TC_SMALL if q.name in ("tc31x31", "tc51x5", "tc5x51", "tc17x17_nonsame", "tc64x64",
+                                                 "tc11x9_c136_ragged_x", "tc31x31_f16")]
+
+
+_TILE_PROBLEM = P("tc_tile", "depthwise", "bf16", 9, 37, 41, 24, 24, 9, 7, 1, 4, 3, seed=160)
+TC_A_TMEM_CASES = [(q, "auto") for q in TC_A_TMEM] + [(_TILE_PROBLEM, t) for t in TC_TILES]
+
+
+@pytest.mark.parametrize("case", TC_A_TMEM_CASES, ids=[f"{q.name}-{t}" for q, t in TC_A_TMEM_CASES])
+def test_depthwise_tensor_core_a_in_tensor_memory(case, monkeypatch):
+    """The planar tensor-core kernel with its Toeplitz operand A_i written into tensor memory by the
+    builder warps (DGRAD_TC_A=tmem), the layout it falls back to when the shared-memory tables do not
+    fit: the default tile of several problems, and every tile shape on a ragged problem."""
+    p, tile = case
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_A", "tmem")
+    if tile != "auto":
+        monkeypatch.setenv("DGRAD_TC_TILE", tile)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/A in tensor memory, tile {tile}")
+    cb.check_status()
+
+
+# More than 8 images (two or more image groups, ragged), two row tiles, two B panels (K clipped
+# to 80), both orientations, f16.
+TC_MANY_IMAGES = [
+    P("tcn16_31x31", "depthwise", "bf16", 16, 20, 20, 16, 16, 31, 31, 1, 15, 15, seed=171),
+    P("tcn13_9x7", "depthwise", "bf16", 13, 28, 36, 24, 24, 9, 7, 1, 4, 3, seed=172),
+    P("tcn17_11x5_two_row_tiles", "depthwise", "bf16", 17, 100, 40, 8, 8, 11, 5, 1, 5, 2, seed=173),
+    P("tcn10_5x9_two_panels", "depthwise", "bf16", 10, 68, 64, 8, 8, 5, 9, 1, 2, 8, seed=174),
+    P("tcn12_51x5", "depthwise", "bf16", 12, 64, 64, 16, 16, 51, 5, 1, 25, 2, seed=175),
+    P("tcn12_5x51", "depthwise", "bf16", 12, 64, 64, 16, 16, 5, 51, 1, 2, 25, seed=176),
+    P("tcn11_17x17_f16", "depthwise", "f16", 11, 32, 48, 24, 24, 17, 17, 1, 8, 8, seed=177),
+    P("tcn9_3x3_c40", "depthwise", "bf16", 9, 16, 24, 40, 40, 3, 3, 1, 1, 1, seed=178),
+]
+
+
+@pytest.mark.parametrize("amode", ["smem", "tmem"])
+@pytest.mark.parametrize("p", TC_MANY_IMAGES, ids=[q.name for q in TC_MANY_IMAGES])
+def test_depthwise_tensor_core_many_images(p, amode, monkeypatch):
+    """The planar tensor-core kernel on problems with several image groups, with A_i as shared-memory
+    tables (DGRAD_TC_A=smem) and in tensor memory (DGRAD_TC_A=tmem), against the oracle on every
+    element; dX starts as NaN and a second call gives identical bits."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_A", amode)
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    out = torch.full(p.dx_shape, float("nan"), dtype=dy.dtype, device=dy.device)
+    cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, out=out)
+    again = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    cb.check_status()
+    assert torch.equal(out, again), f"{p.name}: two calls differ"
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/A in {amode}")
+
+
 TC_AUTO = [q for q in TC_SMALL if q.KH * q.KW > 49]
 
 
