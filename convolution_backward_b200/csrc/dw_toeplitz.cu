@@ -86,7 +86,7 @@ using namespace toep;
 
 constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxA = 6;         // A buffers (tensor memory: at most 4; shared memory: at most 6)
+constexpr int kMaxA = 4;         // A buffers: tensor-memory tiles or shared-memory tables
 constexpr int kMaxB = 2;         // B blocks in shared memory
 constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 9;   // + d_full[2], d_empty[2], drain, f_full[2], f_empty[2]
 

@@ -449,6 +449,29 @@ def test_grouped_and_f16_tensor_core(p):
     cb.check_status()
 
 
+# fp32 pointwise on both tile heights: 64-row tiles (>= 64 tiles: 4096 and 4160+5 rows) and
+# 16-row tiles (fewer tiles: 392 rows as in the small fp32 workload, and a ragged 77-row case)
+PW_F32_TILES = [P("pw_f32_tall", "pointwise", "f32", 4, 32, 32, 64, 48, seed=191),
+                P("pw_f32_tall_ragged", "pointwise", "f32", 5, 29, 29, 68, 36, seed=192),
+                P("pw_f32_392", "pointwise", "f32", 2, 14, 14, 64, 64, seed=193),
+                P("pw_f32_77", "pointwise", "f32", 1, 7, 11, 24, 20, seed=194)]
+
+
+@pytest.mark.parametrize("p", PW_F32_TILES, ids=[q.name for q in PW_F32_TILES])
+def test_pointwise_f32_tile_heights(p):
+    """The fp32 FMA pointwise kernel with 64-row and with 16-row tiles against the oracle, every element
+    within the fp32 bound."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    got = h.gpu_to_np(h.run_gpu(p, dy, w))
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=p.name)
+    cb.check_status()
+
+
 @pytest.mark.parametrize("shape", [(2, 13, 23, 264, 200), (1, 9, 11, 64, 512), (3, 7, 5, 8, 8)])
 def test_pointwise_f16(shape):
     """dgrad_pointwise with fp16 I/O (routed to the tap kernel with one 1x1 tap)."""
