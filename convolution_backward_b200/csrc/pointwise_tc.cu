@@ -571,10 +571,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     pw_tc_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_d, int M, int C, int K, int* status)
 {
-    pdl_wait();      // the previous kernel on the stream has finished
-    pdl_trigger();   // the next one may start its set-up
     using L = PwPairLayout<BN, STAGES>;
     constexpr int kPairStages = STAGES;
+    {
+        // While the previous kernel may still run, only L2 prefetches of this CTA's first
+        // stages of dY and W: L2 is the point of coherence, so the loads below still see
+        // that kernel's writes, and the DRAM reads overlap its tail.
+        const int num_n0 = (C + BN - 1) / BN;
+        const int pairs0 = static_cast<int>(gridDim.x >> 1);
+        const PwSched sched0(((M + 255) / 256) * num_n0, num_n0, pairs0, BN);
+        const int pair0 = static_cast<int>(blockIdx.x >> 1);
+        if (threadIdx.x == 0 && sched0.count(pair0) > 0) {
+            const uint32_t r0 = cluster_ctarank();
+            const PwUnit un = sched0.unit(pair0, 0, BN);
+            tma_prefetch_desc(&map_a);
+            tma_prefetch_desc(&map_b);
+            const int nkb = (K + kBK - 1) / kBK < kPairStages ? (K + kBK - 1) / kBK : kPairStages;
+            for (int kb = 0; kb < nkb; ++kb) {
+                tma_prefetch_l2_2d(&map_a, kb * kBK, un.m_blk * 256 + static_cast<int>(r0) * 128);
+                for (int j = 0; j < un.ncols / 128; ++j)
+                    tma_prefetch_l2_2d(&map_b, un.n0 + static_cast<int>(r0) * (un.ncols / 2) + j * 64, kb * kBK);
+            }
+        }
+    }
+    pdl_wait();      // the previous kernel on the stream has finished
+    pdl_trigger();   // the next one may start its set-up
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
