@@ -31,6 +31,16 @@ __global__ void __launch_bounds__(kThreads)
     constexpr int RT = TM / 16;
     constexpr int kLdA = TM * kTK / 4 / kThreads;    // float4 loads per thread of a dY slice
     constexpr int kLdB = kTK * kTC / 4 / kThreads;   // of a W slice
+    {
+        // While the previous kernel may still run, only L2 prefetches of the first slice this
+        // thread loads (L2 is the point of coherence, so the loads still see its writes).
+        const int m = blockIdx.x * TM + (threadIdx.x >> 4);
+        const int k = (threadIdx.x & 15) * 4;
+        if (m < M && k < K) asm volatile("prefetch.global.L2 [%0];" ::"l"(dY + static_cast<int64_t>(m) * K + k));
+        const int c = blockIdx.y * kTC + (threadIdx.x & 15) * 4;
+        if ((threadIdx.x >> 4) < K && c < C)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(W + static_cast<int64_t>(threadIdx.x >> 4) * C + c));
+    }
     pdl_wait();      // the previous kernel on the stream has finished
     pdl_trigger();   // the next one may start its set-up
     __shared__ __align__(16) float As[kTK][TM + 4];    // dY slice, stored k-major
