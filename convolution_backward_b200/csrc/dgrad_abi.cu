@@ -536,7 +536,7 @@ dgrad_status_t dgrad_depthwise_tc(const dgrad_problem_t* prob, dgrad_dtype_t dty
     dgrad::ToepMaps maps{};
     if (!encode_planar_bf16(&maps.b, workspace, static_cast<uint64_t>(plan.Xi), static_cast<uint64_t>(a.N),
                             static_cast<uint64_t>(plan.Yi), static_cast<uint64_t>(a.C),
-                            static_cast<uint64_t>(plan.Xsi), static_cast<unsigned>(plan.NR)))
+                            static_cast<uint64_t>(plan.Xsi), static_cast<unsigned>(plan.b_rows)))
         return cuda_fail(cudaErrorInvalidValue);
     // TMA transposes when every map encodes (DGRAD_TC_TRANSPOSE=cuda selects the CUDA-core ones)
     const void* dXp = static_cast<const uint8_t*>(workspace) + plan.ws_in;

@@ -31,7 +31,12 @@
 // atom.  Row (h', img) of B_i is row (2*h' + i, img), so B_i is that block seen
 // through a descriptor whose start moves by one atom per shift step and whose
 // row-group stride is two atoms: one TMA load of the planar input per 64
-// columns serves every shift.  A_i is Toeplitz along both of its axes at the
+// columns serves every shift.  When one tile spans the whole plane height, every
+// block has the same rows of zero padding above and below the image; the two
+// blocks then share the zero rows between them, which the kernel writes once, and
+// each TMA load brings only the image rows (31x31 on 64-row planes: 173 KB for
+// both blocks instead of 188 KB, which leaves room for six A tables instead of
+// three; 110.4 -> 106.4 us on B200).  A_i is Toeplitz along both of its axes at the
 // granularity of 8 x 8 core matrices when each 8-row group holds 4 columns of
 // both row phases, so for P = 2 it is stored as a table of a_slots distinct
 // 128-byte core matrices (3.75 KB at K = 64) that the MMA's no-swizzle
@@ -86,7 +91,7 @@ using namespace toep;
 
 constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxA = 4;         // A buffers: tensor-memory tiles or shared-memory tables
+constexpr int kMaxA = 6;         // A buffers: tensor-memory tiles (at most 4) or shared-memory tables
 constexpr int kMaxB = 2;         // B blocks in shared memory
 constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 9;   // + d_full[2], d_empty[2], drain, f_full[2], f_empty[2]
 
@@ -110,6 +115,13 @@ struct ToepArgs {
     int tma_epi;                 // the epilogue stages 8 x 8 x 64 boxes in shared memory and stores them by TMA
     uint32_t stg_off;            // two 8 KB staging boxes (one per epilogue half)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
+    // B blocks: b_stride bytes apart.  When a tile spans the whole plane height, the rows of
+    // zero padding above and below the image are written once, and neighbouring blocks share
+    // the zero rows between them; the TMA box then carries only the image rows: it starts
+    // b_zt rows into the block (b_ld_off bytes) and brings b_ld_bytes.
+    uint32_t b_stride, b_ld_off, b_ld_bytes;
+    int b_zt;
+    uint32_t z_off[3], z_len[3];  // the zero rows, written at the start
     long long dxp_bytes;         // size of the planar output (index checks of the debug build)
 };
 
@@ -194,7 +206,7 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
     // and this single thread's issue rate bounds the tensor pipe's.
     const int NI = a.NI;
     const uint32_t na = static_cast<uint32_t>(a.na), nb = static_cast<uint32_t>(a.NB);
-    const uint32_t a_cols = static_cast<uint32_t>(a.a_cols), b_bytes = a.b_bytes, bblk_addr = c.bblk_addr;
+    const uint32_t a_cols = static_cast<uint32_t>(a.a_cols), b_stride = a.b_stride, bblk_addr = c.bblk_addr;
     const bool two_acc = a.nacc == 2;
     uint64_t* const b_full = c.b_full;
     uint64_t* const b_empty = c.b_empty;
@@ -215,7 +227,7 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
         uint32_t d_set[4];
 #pragma unroll
         for (int sx = 0; sx < 4; ++sx) d_set[sx] = d_tmem[sx] + acc * set_cols;
-        uint64_t desc = sw128_desc(bblk_addr + bb * b_bytes, 16, sbo);
+        uint64_t desc = sw128_desc(bblk_addr + bb * b_stride, 16, sbo);
         uint64_t a_desc = a_desc0 + static_cast<uint64_t>(ab * a_buf16);
         for (int i = 0; i < NI; ++i) {
             if (!mbar_wait(&a_full[ab], aph, abort_flag)) return false;
@@ -396,6 +408,13 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) tma_prefetch_desc(&map_b);
+    // the shared zero rows of the B blocks, once; the tensor core reads them through the
+    // async proxy (the barrier below orders them before the first MMA)
+#pragma unroll
+    for (int z = 0; z < 3; ++z)
+        for (uint32_t o = 16u * threadIdx.x; o < a.z_len[z]; o += 16u * kThreadsT)
+            *reinterpret_cast<uint4*>(bblk + a.z_off[z] + o) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
@@ -435,11 +454,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&b_full[bb], a.b_bytes);
-                uint8_t* blk = bblk + bb * a.b_bytes;
+                mbar_arrive_expect_tx(&b_full[bb], a.b_ld_bytes);
+                uint8_t* blk = bblk + bb * a.b_stride + a.b_ld_off;
                 for (uint32_t pn = 0; pn < a.npanels; ++pn)
                     tma_load_4d(blk + pn * a.panel_bytes, &map_b, &b_full[bb], t.xb + 64 * static_cast<int>(pn),
-                                8 * t.g, t.Y0 - a.py, t.c);
+                                8 * t.g, t.Y0 - a.py + a.b_zt, t.c);
                 ++ub;
             }
             if (!ok) {
@@ -985,6 +1004,16 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     const char* amode = dgrad::tuning_env("DGRAD_TC_A");
     const bool no_a_smem = amode && strcmp(amode, "tmem") == 0;
     const bool force_a_smem = amode && strcmp(amode, "smem") == 0;
+    // DGRAD_TC_SHZ=0 gives every B block its own zero rows, loaded with the image rows (testing
+    // and tuning).
+    const char* shz = dgrad::tuning_env("DGRAD_TC_SHZ");
+    const bool no_shz = shz && strcmp(shz, "0") == 0;
+    // DGRAD_TC_NA=n takes at most n shared-memory tables; DGRAD_TC_NFB=1 one filter-line buffer
+    // (testing and tuning).
+    const char* nas = dgrad::tuning_env("DGRAD_TC_NA");
+    const int max_na = nas ? atoi(nas) : kMaxA;
+    const char* nfs = dgrad::tuning_env("DGRAD_TC_NFB");
+    const bool one_fb = nfs && strcmp(nfs, "1") == 0;
     if (const char* ft = dgrad::tuning_env("DGRAD_TC_TILE"))
         if (sscanf(ft, "%d,%d,%d,%d", &force[0], &force[1], &force[2], &force[3]) != 4) force[0] = -1;
     bool have = false;
@@ -1048,12 +1077,20 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
             const int na_tmem = std::min((static_cast<int>(kTmemCols) - p.a_col0) / p.a_cols, 4);
             p.panel_bytes = static_cast<uint32_t>(p.NR) * 1024u;
             p.b_bytes = static_cast<uint32_t>(p.npanels) * p.panel_bytes;
+            // When a tile spans the whole plane height, every B block holds the same zt = py
+            // rows of zero padding above the image rows and zb below them.  With two blocks
+            // those rows are written once, and the zero rows between the blocks serve both:
+            // [zt zeros][image rows][max(zt, zb) zeros][image rows][zb zeros].  For 31x31 on
+            // 64-row planes that is 173 KB instead of 188 KB, which leaves room for more A
+            // tables, and each TMA box carries 64 rows instead of 94.
+            const int zt = p.py, zb = p.NR - p.py - p.Yi;
+            const bool shz_ok = !nhwc && !no_shz && p.npanels == 1 && p.Yo <= p.P * p.NH && zt > 0 && zb > 0;
             bool fits = false;
             // The NHWC kernel keeps one B block (the cluster refills it) and two filter
             // buffers, or one when two do not fit.  The planar kernel takes two B blocks when
             // they fit and, for P = 2 with one sub-tile, 16 KB of epilogue staging boxes when
-            // they fit as well; then two filter-line buffers when they fit as well; with A in
-            // shared memory, 4, 3 or 2 tables.
+            // they fit as well; then, with A in shared memory, 6 down to 2 tables; then two
+            // filter-line buffers when they fit as well.
             const bool stg_ok = !nhwc && p.P == 2 && p.XT == 1 && !no_tma_epi;
             const bool smem_a_ok = !nhwc && !no_a_smem && p.P == 2 && p.a_slots * 4 <= 128 * kMaxAPairs &&
                                    (p.NI >= 16 || force_a_smem);
@@ -1062,9 +1099,14 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
                 p.nacc = p.a_smem ? 2 : 1;
                 p.na = na_tmem;
                 if (!p.a_smem && p.na < 2) break;
-                const int n_na = p.a_smem ? 3 : 1;
+                const int n_na = p.a_smem ? kMaxA - 1 : 1;
                 for (int opt = 0; opt < 8 * n_na && !fits; ++opt) {
-                    const int o = opt / n_na;
+                    // o: B blocks (o / 4), staging (o / 2 % 2), filter buffers (o % 2); with tables,
+                    // their count runs between the (B blocks, staging) groups and the filter
+                    // buffers: more tables before a second filter buffer (31x31 on B200: 6 tables
+                    // with one buffer 106.4 us, 4 tables with two 107.0 us, 4 with one 108.3 us)
+                    const int rem = opt % (2 * n_na);
+                    const int o = (opt / (2 * n_na)) * 2 + rem % 2;
                     if (nhwc) {
                         if (o >= 2) break;
                         p.NB = 1;
@@ -1075,9 +1117,28 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
                         p.tma_epi = stg_ok && (o / 2) % 2 == 0 ? 1 : 0;   // staging, then none
                         p.nfb = o % 2 == 0 ? 2 : 1;             // filter buffers: 2, then 1
                         if (!stg_ok && (o / 2) % 2 == 1) continue;   // the same layouts as the options before
-                        if (p.a_smem) p.na = 4 - opt % n_na;
+                        if (p.a_smem) p.na = kMaxA - rem / 2;
+                        if ((p.a_smem && p.na > max_na) || (one_fb && p.nfb == 2)) continue;
                     }
+                    p.b_zt = 0;
+                    p.b_rows = p.NR;
+                    p.b_stride = p.b_bytes;
+                    for (int z = 0; z < 3; ++z) p.z_off[z] = p.z_len[z] = 0;
                     p.f_off = static_cast<uint32_t>(p.NB) * p.b_bytes;
+                    if (shz_ok && p.NB == 2) {
+                        const uint32_t D = static_cast<uint32_t>(p.Yi), ut = static_cast<uint32_t>(zt),
+                                       ub = static_cast<uint32_t>(zb), um = std::max(ut, ub);
+                        p.b_zt = zt;
+                        p.b_rows = p.Yi;
+                        p.b_stride = (D + um) * 1024u;
+                        p.z_off[0] = 0;
+                        p.z_len[0] = ut * 1024u;
+                        p.z_off[1] = (ut + D) * 1024u;
+                        p.z_len[1] = um * 1024u;
+                        p.z_off[2] = (ut + 2u * D + um) * 1024u;
+                        p.z_len[2] = ub * 1024u;
+                        p.f_off = (ut + 2u * D + um + ub) * 1024u;
+                    }
                     p.bar_off = static_cast<uint32_t>(round_up(p.f_off + 4ull * p.nfb * p.f_words, 16));
                     size_t end = p.bar_off + (nhwc ? kNumBarsNhwc : kNumBars) * 8 + 16;
                     p.a_off = 0;
@@ -1243,6 +1304,14 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.f16 = a.f16 ? 1 : 0;
         t.panel_bytes = p.panel_bytes;
         t.b_bytes = p.b_bytes;
+        t.b_stride = p.b_stride;
+        t.b_zt = p.b_zt;
+        t.b_ld_off = static_cast<uint32_t>(p.b_zt) * 1024u;
+        t.b_ld_bytes = static_cast<uint32_t>(p.b_rows) * 1024u * static_cast<uint32_t>(p.npanels);
+        for (int z = 0; z < 3; ++z) {
+            t.z_off[z] = p.z_off[z];
+            t.z_len[z] = p.z_len[z];
+        }
         t.npanels = static_cast<uint32_t>(p.npanels);
         t.f_words = static_cast<uint32_t>(p.f_words);
         t.f_bytes = static_cast<uint32_t>(p.f_words) * 4u;

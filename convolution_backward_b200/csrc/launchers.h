@@ -101,7 +101,7 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 // the plane orientation and tile and returns false when the problem does not
 // fit; the launch needs a workspace of ws_in + ws_out + ws_f bytes (planar dY,
 // planar dX, packed filter lines) and map_b, a 4-D bf16 map of the planar dY
-// [C][Yi][N][Xsi] with dims (Xi, N, Yi, C), box (64, 8, NR, 1), 128-byte
+// [C][Yi][N][Xsi] with dims (Xi, N, Yi, C), box (64, 8, b_rows, 1), 128-byte
 // swizzle, zero fill.
 struct ToepPlan {
     int orient, KY, KX, py, px, Yi, Xi, Xsi, Yo, Xo, Xso;
@@ -112,6 +112,11 @@ struct ToepPlan {
     int tma_epi;          // the MMA epilogue stores staged boxes by TMA (needs ToepMaps::d_store)
     uint32_t stg_off;     // its staging boxes in shared memory
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
+    // B blocks b_stride bytes apart; the TMA box brings b_rows rows starting b_zt rows into a
+    // block (b_rows = NR, b_zt = 0 unless the blocks share their zero rows, which the kernel
+    // writes once at z_off / z_len)
+    int b_zt, b_rows;
+    uint32_t b_stride, z_off[3], z_len[3];
     size_t smem, ws_in, ws_out, ws_f;
 };
 // Tensor maps of one call: b as above; for the transposes (when tma_transpose),

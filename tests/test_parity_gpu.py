@@ -601,6 +601,42 @@ def test_depthwise_tensor_core_many_images(p, amode, monkeypatch):
     h.check(p, got, ref, absref, what=f"{p.name}/A in {amode}")
 
 
+# B-block layouts of the planar kernel: by default the blocks share the rows of zero padding
+# above and below the image (written once by the kernel); DGRAD_TC_SHZ=0 gives each block its
+# own, loaded by the TMA with the image rows.  Fewer shared-memory tables (DGRAD_TC_NA), with one or
+# two filter-line buffers (DGRAD_TC_NFB), are the other layouts the planner can reach.
+TC_LAYOUT_PROBLEMS = [q for q in TC_SMALL if q.name in ("tc31x31", "tc31x31_c40", "tc51x5", "tc17x17_nonsame",
+                                                        "tc7x7_nonsame", "tc41x41")] + \
+    [q for q in TC_MANY_IMAGES if q.name in ("tcn16_31x31", "tcn13_9x7", "tcn12_5x51")]
+TC_LAYOUTS = {"own_zero_rows": {"DGRAD_TC_SHZ": "0"},
+              "4_tables": {"DGRAD_TC_NA": "4"},
+              "5_tables": {"DGRAD_TC_NA": "5"},
+              "one_filter_buffer_4_tables": {"DGRAD_TC_NFB": "1", "DGRAD_TC_NA": "4"}}
+
+
+@pytest.mark.parametrize("layout", list(TC_LAYOUTS))
+@pytest.mark.parametrize("p", TC_LAYOUT_PROBLEMS, ids=[q.name for q in TC_LAYOUT_PROBLEMS])
+def test_depthwise_tensor_core_b_layouts(p, layout, monkeypatch):
+    """The planar tensor-core kernel with each B-block and table layout, against the oracle on every
+    element; the workspace starts as NaN, and a call with the default layout gives identical bits."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    nb = cb.depthwise_tc_workspace_bytes(p.N, p.H, p.W, p.C, p.KH, p.KW, p.pad_h, p.pad_w)
+    ws = torch.full((nb // 2 + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    base = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w)
+    for k, v in TC_LAYOUTS[layout].items():
+        monkeypatch.setenv(k, v)
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=ws)
+    cb.check_status()
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/{layout}")
+    assert torch.equal(out, base), f"{p.name}: {layout} differs from the default layout"
+
+
 TC_AUTO = [q for q in TC_SMALL if q.KH * q.KW > 49]
 
 
