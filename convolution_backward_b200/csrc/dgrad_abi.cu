@@ -625,12 +625,16 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
         e = dgrad::launch_dw_tile(a, map, cs);
     } else if (mode == DGRAD_DW_ROTATED) {
         e = dgrad::launch_dw_rotated(a, cs);
-    } else if (env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box)) {
-        CUtensorMap map;
+    } else if (unsigned box_dx[4]; env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box, box_dx)) {
+        CUtensorMap map, dx_map;
         if (!encode_nhwc_h16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box, a.f16))
             return cuda_fail(cudaErrorInvalidValue);
-        e = dgrad::launch_dw_rowstream_fast(a, map, 0, cs);
+        // the output map is optional: without it the kernel stores dX directly
+        const bool dx_ok = aligned16(dX) && encode_nhwc_h16(&dx_map, dX, static_cast<uint64_t>(prob->N),
+                                                            static_cast<uint64_t>(prob->H), static_cast<uint64_t>(prob->W),
+                                                            static_cast<uint64_t>(prob->C), box_dx, a.f16);
+        e = dgrad::launch_dw_rowstream_fast(a, map, dx_ok ? &dx_map : nullptr, 0, cs);
     } else {
         e = dgrad::launch_dw_rowstream(a, cs);
     }

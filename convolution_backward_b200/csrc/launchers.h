@@ -145,12 +145,15 @@ cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);
 
 // Register-blocked row-streaming kernel for the compiled (KH, KW, S) set, bf16
 // or f16.  dy_map covers dY as a 4-D 16-bit tensor (C, Wo, Ho, N innermost first)
-// with no swizzle.  Returns cudaErrorNotSupported when no instantiation fits.
-cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, int G, cudaStream_t stream);
+// with no swizzle; dx_map (or null) covers dX the same way (C, W, H, N), and the
+// register-ring kernel then stores its final rows through it.  Returns
+// cudaErrorNotSupported when no instantiation fits.
+cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map, int G,
+                                     cudaStream_t stream);
 
-// Box (inner first) the fast row-streaming kernel loads from dY, or false when
-// the problem has no fast instantiation.
-bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4]);
+// Boxes (inner first) the fast row-streaming kernel loads from dY and stores into
+// dX, or false when the problem has no fast instantiation.
+bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4]);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -43,6 +43,8 @@ CASES = [
     (P("dw_tile_3x3", "depthwise", "bf16", 2, 17, 19, 40, 40, 3, 3, 1, 1, 1, seed=504), {}, "rotated"),
     (P("dw_rot_13x9_f32", "depthwise", "f32", 1, 21, 17, 36, 36, 13, 9, 1, 6, 4, seed=505), {}, "rotated"),
     (P("dw_rs_reg_7x7s2", "depthwise", "bf16", 2, 23, 29, 40, 40, 7, 7, 2, 3, 3, seed=506), {}, "rowstream"),
+    (P("dw_rs_reg_7x7s2_direct", "depthwise", "bf16", 2, 23, 29, 40, 40, 7, 7, 2, 3, 3, seed=506),
+     {"DGRAD_RS_STORE": "direct"}, "rowstream"),
     (P("dw_rs_smem_5x5s2", "depthwise", "bf16", 1, 19, 21, 24, 24, 5, 5, 2, 2, 2, seed=507),
      {"DGRAD_RS_KERNEL": "smem"}, "rowstream"),
     (P("dw_rs_generic_s3", "depthwise", "f16", 1, 17, 16, 16, 16, 5, 4, 3, 2, 1, seed=508),

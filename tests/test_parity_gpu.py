@@ -299,16 +299,19 @@ RS_FAST = [
 ]
 
 
-RS_VARIANTS = [("0", "reg", ""), ("0", "reg", "q4"), ("0", "smem", ""), ("0", "smem", "alt"), ("1", "", "")]
+RS_VARIANTS = [("0", "reg", ""), ("0", "reg", "q4"), ("0", "reg", "direct"), ("0", "smem", ""), ("0", "smem", "alt"),
+               ("1", "", "")]
 
 
 @pytest.mark.parametrize("generic,kern,g", RS_VARIANTS,
-                         ids=["reg-ring", "reg-ring-q4", "smem-ring", "smem-ring-altG", "generic"])
+                         ids=["reg-ring", "reg-ring-q4", "reg-ring-direct-stores", "smem-ring", "smem-ring-altG",
+                              "generic"])
 @pytest.mark.parametrize("p", RS_FAST, ids=[p.name for p in RS_FAST])
 def test_rowstream_paths(p, generic, kern, g, monkeypatch):
     """Strided depthwise through every row-streaming kernel: accumulator ring in
-    registers (two and four output columns per thread), ring in shared memory (both
-    step depths G), and the generic one."""
+    registers (two and four output columns per thread; final rows stored by TMA from
+    shared memory, or stored directly), ring in shared memory (both step depths G), and
+    the generic one."""
     h = _h()
     monkeypatch.setenv("DGRAD_RS_GENERIC", generic)
     if kern:
@@ -317,6 +320,8 @@ def test_rowstream_paths(p, generic, kern, g, monkeypatch):
         monkeypatch.setenv("DGRAD_RS_G", {7: "1", 5: "1", 3: "2"}[p.KH])
     if g == "q4":
         monkeypatch.setenv("DGRAD_RS_Q", "4")
+    if g == "direct":
+        monkeypatch.setenv("DGRAD_RS_STORE", "direct")
     inp = synthetic.make_inputs(p)
     dy, w = h.to_dev(inp)
     got = h.gpu_to_np(h.run_gpu(p, dy, w))
