@@ -112,6 +112,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     return true;
 }
 
+// Bounded wait until a flag in global memory that another CTA sets (flag_set_gpu)
+// is non-zero, with acquire at GPU scope.  Returns false when the budget runs out
+// or the abort flag is raised.
+__device__ __forceinline__ bool flag_wait_gpu(const int* flag, const volatile int* abort = nullptr)
+{
+    const long long t0 = clock64();
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v != 0) return true;
+        if (abort && *abort) return false;
+        if (clock64() - t0 > kWaitCycles) return false;
+        __nanosleep(64);
+    }
+}
+
+// Sets a flag in global memory with release at GPU scope (after the caller's writes).
+__device__ __forceinline__ void flag_set_gpu(int* flag)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+
 // Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity)
 {
@@ -305,6 +327,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar)
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Warp-collective load of 8 consecutive 32-bit columns (as the x32 form below).
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&v)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr)
+                 : "memory");
+}
 
 // Warp-collective load of 32 consecutive 32-bit columns: lane i of the warp
 // receives TMEM lane (taddr.lane + i), columns taddr.col .. taddr.col + 31.

@@ -93,7 +93,7 @@ constexpr int kThreadsT = 448;   // 14 warps: producer, MMA, 4 A builders, 8 epi
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxA = 6;         // A buffers: tensor-memory tiles (at most 4) or shared-memory tables
 constexpr int kMaxB = 2;         // B blocks in shared memory
-constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 9;   // + d_full[2], d_empty[2], drain, f_full[2], f_empty[2]
+constexpr int kNumBars = 2 * kMaxB + 2 * kMaxA + 10;   // + d_full[2], d_empty[2], drain, f_full[2], f_empty[2], d_init
 
 
 struct ToepArgs {
@@ -122,6 +122,13 @@ struct ToepArgs {
     uint32_t b_stride, b_ld_off, b_ld_bytes;
     int b_zt;
     uint32_t z_off[3], z_len[3];  // the zero rows, written at the start
+    // split: the CTAs take equal ranges of shift steps instead of whole tiles.  A tile whose
+    // steps two CTAs share is started by the higher CTA, which writes its fp32 partial sum
+    // to part[its block] ([set_cols][128], column-major) and sets part_flag[its block]; the
+    // lower CTA ends with the tile's first steps, adds that partial and stores the result.
+    int split;
+    float* part;
+    int* part_flag;
     long long dxp_bytes;         // size of the planar output (index checks of the debug build)
 };
 
@@ -156,6 +163,7 @@ struct MmaCtx {
     uint32_t tmem_base;
     uint32_t bblk_addr;
     uint32_t a_addr;             // A table 0 (A in shared memory)
+    uint64_t* d_init;            // split: the partial is in the last unit's accumulator set
 };
 
 // The MMAs of one shift step with A_i in shared memory: as issue_step, with the
@@ -183,7 +191,8 @@ __device__ __forceinline__ void issue_step_ss(const uint32_t (&d_tmem)[4], uint6
 // indices and phases advance incrementally and the B descriptor moves by one
 // swizzle atom per step.  Returns false when a wait gave up.
 template <int KQ, int XT, bool AS>
-__device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
+__device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end, int i_first,
+                                      int i_last)
 {
     const int ncol_sub = 8 * a.NH;
     const uint32_t idesc =
@@ -205,6 +214,7 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
     // memory, so fields read through `a` or `c` would be loaded again after each of them,
     // and this single thread's issue rate bounds the tensor pipe's.
     const int NI = a.NI;
+    const bool split = a.split != 0;
     const uint32_t na = static_cast<uint32_t>(a.na), nb = static_cast<uint32_t>(a.NB);
     const uint32_t a_cols = static_cast<uint32_t>(a.a_cols), b_stride = a.b_stride, bblk_addr = c.bblk_addr;
     const bool two_acc = a.nacc == 2;
@@ -227,15 +237,25 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
         uint32_t d_set[4];
 #pragma unroll
         for (int sx = 0; sx < 4; ++sx) d_set[sx] = d_tmem[sx] + acc * set_cols;
-        uint64_t desc = sw128_desc(bblk_addr + bb * b_stride, 16, sbo);
+        // shift steps [ib, ie) of this unit (all of them unless the CTAs split it); when this
+        // CTA ends inside its last unit, that unit's accumulator starts from the partial of
+        // the unit's last steps (written by the epilogue warps), so its MMAs all accumulate
+        const int ib = u == u_begin ? i_first : 0;
+        const int ie = u == u_end - 1 ? i_last : NI;
+        const bool from_partial = split && ie < NI;
+        if (from_partial) {
+            if (!mbar_wait(c.d_init, 0, abort_flag)) return false;
+            tc_fence_after();
+        }
+        uint64_t desc = sw128_desc(bblk_addr + bb * b_stride, 16, sbo) + 64u * static_cast<uint32_t>(ib);
         uint64_t a_desc = a_desc0 + static_cast<uint64_t>(ab * a_buf16);
-        for (int i = 0; i < NI; ++i) {
+        for (int i = ib; i < ie; ++i) {
             if (!mbar_wait(&a_full[ab], aph, abort_flag)) return false;
             tc_fence_after();
             if (AS)
-                issue_step_ss<KQ, XT>(d_set, a_desc, desc, pb16, a_q16, idesc, i == 0);
+                issue_step_ss<KQ, XT>(d_set, a_desc, desc, pb16, a_q16, idesc, i == ib && !from_partial);
             else
-                issue_step<KQ, XT>(d_set, a_tmem, desc, pb16, idesc, i == 0);
+                issue_step<KQ, XT>(d_set, a_tmem, desc, pb16, idesc, i == ib && !from_partial);
             umma_commit(&a_empty[ab]);   // A buffer free once these MMAs have read it
             desc += 64;                   // next shift step: one 1024-byte atom
             if (++ab == na) {
@@ -259,18 +279,19 @@ __device__ __noinline__ bool mma_role(const ToepArgs& a, const MmaCtx& c, int u_
 }
 
 template <int XT, bool AS>
-__device__ __forceinline__ bool mma_role_x(int kq, const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end)
+__device__ __forceinline__ bool mma_role_x(int kq, const ToepArgs& a, const MmaCtx& c, int u_begin, int u_end,
+                                           int i_first, int i_last)
 {
     switch (kq) {
-    case 1: return mma_role<1, XT, AS>(a, c, u_begin, u_end);
-    case 2: return mma_role<2, XT, AS>(a, c, u_begin, u_end);
-    case 3: return mma_role<3, XT, AS>(a, c, u_begin, u_end);
-    case 4: return mma_role<4, XT, AS>(a, c, u_begin, u_end);
-    case 5: return mma_role<5, XT, AS>(a, c, u_begin, u_end);
-    case 6: return mma_role<6, XT, AS>(a, c, u_begin, u_end);
-    case 7: return mma_role<7, XT, AS>(a, c, u_begin, u_end);
-    case 8: return mma_role<8, XT, AS>(a, c, u_begin, u_end);
-    default: return mma_role<9, XT, AS>(a, c, u_begin, u_end);
+    case 1: return mma_role<1, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 2: return mma_role<2, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 3: return mma_role<3, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 4: return mma_role<4, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 5: return mma_role<5, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 6: return mma_role<6, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 7: return mma_role<7, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    case 8: return mma_role<8, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
+    default: return mma_role<9, XT, AS>(a, c, u_begin, u_end, i_first, i_last);
     }
 }
 
@@ -299,7 +320,8 @@ __device__ __forceinline__ uint4 load_window(const uint32_t* src, bool odd)
 
 __device__ __forceinline__ bool build_a_tables(const ToepArgs& a, const Unit& t, const uint32_t* lines,
                                                uint8_t* tables, uint64_t* a_full, uint64_t* a_empty,
-                                               const volatile int* abort_flag, int tb, uint32_t& ab, uint32_t& aph)
+                                               const volatile int* abort_flag, int tb, uint32_t& ab, uint32_t& aph,
+                                               int ib, int ie)
 {
     const int c0 = t.xb - t.x0 + a.px;
     const int npairs = 4 * a.a_slots;
@@ -317,9 +339,11 @@ __device__ __forceinline__ bool build_a_tables(const ToepArgs& a, const Unit& t,
         wo[k] = t0 >> 1;
         odd[k] = (t0 & 1) != 0;
         off[k] = 128 * sl + 16 * xr;
-        prev[k] = make_uint4(0u, 0u, 0u, 0u);          // line -1
+        prev[k] = make_uint4(0u, 0u, 0u, 0u);          // line ib - 1 (none when ib = 0)
+        if (ib > 0 && ib - 1 < KY && q < npairs) prev[k] = load_window(lines + (ib - 1) * half_l + wo[k], odd[k]);
     }
-    for (int i = 0; i < NI; ++i) {
+    (void)NI;
+    for (int i = ib; i < ie; ++i) {
         uint4 cur[kMaxAPairs];
 #pragma unroll
         for (int k = 0; k < kMaxAPairs; ++k) {
@@ -354,6 +378,61 @@ __device__ __forceinline__ void unit_range(const ToepArgs& a, int* u_begin, int*
     *u_end = static_cast<int>((static_cast<long long>(blockIdx.x + 1) * a.num_units) / gridDim.x);
 }
 
+// Split tiles (ToepArgs::split), one epilogue thread: its accumulator row (TMEM lane)
+// in the nch 32-column chunks from taddr, against a partial laid out [column][128 rows]
+// from `out` / `in` (this thread's row and first column already applied).  Eight
+// columns at a time, so that these rare paths need few registers beside the drain's.
+__device__ __forceinline__ void partial_out(uint32_t taddr, int nch, float* out)
+{
+#pragma unroll 1
+    for (int c8 = 0; c8 < 4 * nch; ++c8) {
+        uint32_t v[8];
+        tmem_ld_32x32b_x8(taddr + 8u * static_cast<uint32_t>(c8), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) __stcg(out + (8 * c8 + k) * 128, __uint_as_float(v[k]));
+    }
+}
+
+__device__ __forceinline__ void partial_init(uint32_t taddr, int nch, const float* in)
+{
+#pragma unroll 1
+    for (int h = 0; h < 2 * nch; ++h) {
+        // 16 loads issued together (16 KB in flight per SM), then two 8-column stores
+        uint32_t q[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) q[k] = __float_as_uint(__ldcg(in + (16 * h + k) * 128));
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            uint32_t v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = q[8 * g + k];
+            tmem_st_32x32b_x8(taddr + 16u * static_cast<uint32_t>(h) + 8u * static_cast<uint32_t>(g), v);
+        }
+    }
+    tmem_wait_st();
+}
+
+// With split: the steps [sb, se) of this CTA in the sequence of all units' shift
+// steps; units [u_begin, u_end), the first from step i_first, the last up to step
+// i_last (exclusive).  Without split: whole units, i_first = 0, i_last = NI.
+__device__ __forceinline__ void step_range(const ToepArgs& a, int* u_begin, int* u_end, int* i_first, int* i_last)
+{
+    if (!a.split) {
+        unit_range(a, u_begin, u_end);
+        *i_first = 0;
+        *i_last = a.NI;
+        return;
+    }
+    const long long total = static_cast<long long>(a.num_units) * a.NI;
+    const long long sb = (static_cast<long long>(blockIdx.x) * total) / gridDim.x;
+    const long long se = (static_cast<long long>(blockIdx.x + 1) * total) / gridDim.x;
+    *u_begin = static_cast<int>(sb / a.NI);
+    *i_first = static_cast<int>(sb - static_cast<long long>(*u_begin) * a.NI);
+    *u_end = static_cast<int>((se + a.NI - 1) / a.NI);
+    *i_last = static_cast<int>(se - static_cast<long long>(*u_end - 1) * a.NI);
+}
+
 __global__ void __launch_bounds__(kThreadsT, 1)
     dw_toeplitz_kernel(const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_d,
                        const __grid_constant__ ToepArgs a)
@@ -375,6 +454,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     uint64_t* drain = d_full + 4;
     uint64_t* f_full = d_full + 5;                    // [2]
     uint64_t* f_empty = d_full + 7;                   // [2]
+    uint64_t* d_init = d_full + 9;                    // split: the last unit's accumulator holds the partial
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -383,8 +463,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     const uint32_t na = static_cast<uint32_t>(a.na);
     const uint32_t nb = static_cast<uint32_t>(a.NB);
     const int ncol_sub = 8 * a.NH;                    // accumulator columns per sub-tile
-    int u_begin, u_end;
-    unit_range(a, &u_begin, &u_end);
+    int u_begin, u_end, i_first, i_last;
+    step_range(a, &u_begin, &u_end, &i_first, &i_last);
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < kMaxB; ++b) {
@@ -404,6 +484,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             mbar_init(&f_empty[b], 128);
         }
         mbar_init(drain, 1);
+        mbar_init(d_init, 256);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -480,17 +561,17 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             MmaCtx ctx{b_full,    b_empty,        a_full,   a_empty, d_full, d_empty, abort_flag, tmem_base,
-                       smem_u32(bblk), smem_u32(smem + a.a_off)};
+                       smem_u32(bblk), smem_u32(smem + a.a_off), d_init};
             const int kq = a.Ks >> 4;
             bool ok;
             if (a.a_smem)
-                ok = a.XT == 1   ? mma_role_x<1, true>(kq, a, ctx, u_begin, u_end)
-                     : a.XT == 2 ? mma_role_x<2, true>(kq, a, ctx, u_begin, u_end)
-                                 : mma_role_x<4, true>(kq, a, ctx, u_begin, u_end);
+                ok = a.XT == 1   ? mma_role_x<1, true>(kq, a, ctx, u_begin, u_end, i_first, i_last)
+                     : a.XT == 2 ? mma_role_x<2, true>(kq, a, ctx, u_begin, u_end, i_first, i_last)
+                                 : mma_role_x<4, true>(kq, a, ctx, u_begin, u_end, i_first, i_last);
             else
-                ok = a.XT == 1   ? mma_role_x<1, false>(kq, a, ctx, u_begin, u_end)
-                     : a.XT == 2 ? mma_role_x<2, false>(kq, a, ctx, u_begin, u_end)
-                                 : mma_role_x<4, false>(kq, a, ctx, u_begin, u_end);
+                ok = a.XT == 1   ? mma_role_x<1, false>(kq, a, ctx, u_begin, u_end, i_first, i_last)
+                     : a.XT == 2 ? mma_role_x<2, false>(kq, a, ctx, u_begin, u_end, i_first, i_last)
+                                 : mma_role_x<4, false>(kq, a, ctx, u_begin, u_end, i_first, i_last);
             if (!ok) {
                 report_timeout(a.status);
                 *abort_flag = 1;
@@ -523,9 +604,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 ++fe;
                 prev_c = t.c;
             }
+            const int ib = u == u_begin ? i_first : 0;
+            const int ie = u == u_end - 1 ? i_last : a.NI;
             if (a.a_smem) {
                 ok = build_a_tables(a, t, fwords + fb * a.f_words, smem + a.a_off, a_full, a_empty, abort_flag,
-                                    threadIdx.x - 64, ab, aph);
+                                    threadIdx.x - 64, ab, aph, ib, ie);
                 const bool last = u + 1 >= u_end || decode_unit(a, u + 1).c != t.c;
                 if (ok && last) mbar_arrive(&f_empty[fb]);
                 continue;
@@ -536,10 +619,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             const uint32_t* rowbase = fwords + fb * a.f_words + (t0 >> 1);
             const bool odd = (t0 & 1) != 0;
             // registers for the loop (its statements clobber memory)
-            const int NI = a.NI, KY = a.KY, kq = a.Ks >> 4, half_l = a.half_l;
+            const int KY = a.KY, kq = a.Ks >> 4, half_l = a.half_l;
             const uint32_t a_base = tmem_base + lane_addr + static_cast<uint32_t>(a.a_col0);
             const uint32_t a_cols = static_cast<uint32_t>(a.a_cols);
-            for (int i = 0; i < NI; ++i) {
+            for (int i = ib; i < ie; ++i) {
                 const uint32_t b = ab;
                 if (!mbar_wait(&a_empty[b], aph ^ 1u, abort_flag)) {
                     ok = false;
@@ -590,16 +673,87 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         const int64_t hrow_stride = static_cast<int64_t>(a.P) * a.N * a.Xso;
         uint32_t ub = 0;
         bool ok = true;
+        const int part_row_i = m + half * hcols * 128;
+        // split, CTA ending inside its last unit: that unit's accumulator set is freed by the
+        // drain of the unit two before it (or is unused); the partial of the last unit's
+        // remaining steps (the next CTA's first unit, ready long before) is written into it
+        // right after that drain (after the first unit's, when the CTA has only two), while
+        // the next unit's MMAs run, and the issuer waits for it.  A CTA sets its own flag
+        // before it waits for the next CTA's, so the waits never form a chain.
+        const bool init_last = a.split && i_last < a.NI;
+        const int init_after = max(u_end - 3, u_begin);
+        auto write_last_partial = [&]() -> bool {
+            bool fw = true;
+            if (warp == 6 && lane == 0) fw = flag_wait_gpu(a.part_flag + blockIdx.x + 1, abort_flag);
+            if (!named_barrier_and(3, 256, fw)) return false;
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            const uint32_t acc_last = static_cast<uint32_t>(u_end - 1 - u_begin) & 1u;
+            partial_init(tmem_base + lane_addr + acc_last * set_cols + static_cast<uint32_t>(half * hcols), nch,
+                         a.part + static_cast<size_t>(blockIdx.x + 1) * 128 * set_cols + part_row_i);
+            tc_fence_before();
+            mbar_arrive(d_init);
+            return true;
+        };
         for (int u = u_begin; u < u_end; ++u) {
             const Unit t = decode_unit(a, u);
             const uint32_t acc = a.nacc == 2 ? (ub & 1u) : 0u;
             const uint32_t use = a.nacc == 2 ? (ub >> 1) : ub;
             const bool w = mbar_wait(&d_full[acc], use & 1u, abort_flag);
-            // with staging boxes the half's 128 threads meet at named barriers, so they agree
-            // on whether to go on
-            if (a.tma_epi ? !named_barrier_and(1 + half, 128, w) : !w) {
+            // with staging boxes the half's 128 threads meet at named barriers, and with split
+            // all 256 epilogue threads meet at barrier 3, so they agree on whether to go on
+            const bool go = a.split      ? named_barrier_and(3, 256, w)
+                            : a.tma_epi ? named_barrier_and(1 + half, 128, w)
+                                        : w;
+            if (!go) {
                 ok = false;
                 break;
+            }
+            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + a.stg_off + half * 8192);
+            const bool issuer = lane == 0 && (warp & 3) == 2;   // warps 6 and 10
+            // P = 2, one sub-tile, staging boxes: the 128 threads of this half hold every row
+            // m = (p, xl) of their 32-column chunk cc, i.e. 8 output rows (4 h' x 2 phases) x 8
+            // images x 64 columns of one channel's planes; they stage that box in shared memory
+            // and one thread stores it with TMA, which clips the ragged edges.
+            auto stage_chunk = [&](int cc, const uint32_t* q) {
+                if (issuer) bulk_wait_group_read<0>();   // the previous box has been read
+                named_barrier_sync(1 + half, 128);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int hp = (2 * k) >> 3;            // h' offset inside the chunk
+                    const int img = (2 * k) & 7;
+                    const uint32_t v = q[k];
+                    stg[((2 * hp + p) * 8 + img) * 64 + xl] = static_cast<uint16_t>(v & 0xFFFFu);
+                    stg[((2 * hp + p) * 8 + img + 1) * 64 + xl] = static_cast<uint16_t>(v >> 16);
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1 + half, 128);
+                if (issuer) {
+                    const int hp0 = (half * hcols + cc * 32) >> 3;
+                    tma_store_4d(&map_d, stg, t.x0, 8 * t.g, t.Y0 + 2 * hp0, t.c);
+                    bulk_commit_group();
+                }
+            };
+            // split: the first unit of a CTA that starts inside it holds the unit's last steps,
+            // whose fp32 partial goes to part[blockIdx.x] ([column][row m]); the last unit of a
+            // CTA that ends inside it started from part[blockIdx.x + 1] (below) and is drained
+            // and stored as usual.
+            const uint32_t tacc = tmem_base + lane_addr + acc * set_cols + static_cast<uint32_t>(half * hcols);
+            const size_t part_stride = static_cast<size_t>(128) * set_cols;
+            const size_t part_row = static_cast<size_t>(m) + static_cast<size_t>(half * hcols) * 128;
+            if (a.split && u == u_begin && i_first > 0) {
+                tc_fence_after();
+                partial_out(tacc, nch, a.part + static_cast<size_t>(blockIdx.x) * part_stride + part_row);
+                tc_fence_before();
+                mbar_arrive(&d_empty[acc]);
+                __threadfence();                 // every epilogue thread's partial is written ...
+                named_barrier_sync(3, 256);
+                if (warp == 6 && lane == 0) flag_set_gpu(a.part_flag + blockIdx.x);   // ... before the flag
+                if (init_last && u == init_after && !write_last_partial()) {
+                    ok = false;
+                    break;
+                }
+                ++ub;
+                continue;
             }
             tc_fence_after();
             uint32_t pk[64];
@@ -618,35 +772,14 @@ __global__ void __launch_bounds__(kThreadsT, 1)
             }
             tc_fence_before();
             mbar_arrive(&d_empty[acc]);   // the accumulator may be overwritten now
+            if (init_last && u == init_after && !write_last_partial()) {
+                ok = false;
+                break;
+            }
             if (a.tma_epi) {
-                // P = 2, one sub-tile: the 128 threads of this half hold every row m = (p, xl)
-                // of their 32-column chunks, i.e. 8 output rows (4 h' x 2 phases) x 8 images
-                // x 64 columns of one channel's planes; they stage that box in shared memory
-                // and one thread stores it with TMA, which clips the ragged edges.
-                uint16_t* stg = reinterpret_cast<uint16_t*>(smem + a.stg_off + half * 8192);
-                const bool issuer = lane == 0 && (warp & 3) == 2;   // warps 6 and 10
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    if (cc < nch) {
-                        if (issuer) bulk_wait_group_read<0>();   // the previous box has been read
-                        named_barrier_sync(1 + half, 128);
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int hp = (2 * k) >> 3;            // h' offset inside the chunk
-                            const int img = (2 * k) & 7;
-                            const uint32_t v = pk[cc * 16 + k];
-                            stg[((2 * hp + p) * 8 + img) * 64 + xl] = static_cast<uint16_t>(v & 0xFFFFu);
-                            stg[((2 * hp + p) * 8 + img + 1) * 64 + xl] = static_cast<uint16_t>(v >> 16);
-                        }
-                        fence_proxy_async_smem();
-                        named_barrier_sync(1 + half, 128);
-                        if (issuer) {
-                            const int hp0 = (half * hcols + cc * 32) >> 3;
-                            tma_store_4d(&map_d, stg, t.x0, 8 * t.g, t.Y0 + 2 * hp0, t.c);
-                            bulk_commit_group();
-                        }
-                    }
-                }
+                for (int cc = 0; cc < 4; ++cc)
+                    if (cc < nch) stage_chunk(cc, pk + cc * 16);
                 ++ub;
                 continue;
             }
@@ -752,9 +885,11 @@ __device__ __forceinline__ void pack_filter_block(const __nv_bfloat16* __restric
 
 __global__ void __launch_bounds__(kPackThreads)
     dw_filter_pack_kernel(const __nv_bfloat16* __restrict__ filt, uint32_t* __restrict__ dst, int C, int KH, int KW,
-                          int KY, int KX, int orient, int half_l, int f_words)
+                          int KY, int KX, int orient, int half_l, int f_words, int* part_flag, int nflags)
 {
     pdl_wait();      // the previous kernel on the stream has finished
+    if (blockIdx.x == 0 && blockIdx.y == 0)   // the split flags of the MMA kernel that follows
+        for (int i = threadIdx.x; i < nflags; i += blockDim.x) part_flag[i] = 0;
     pack_filter_block(filt, dst, C, KH, KW, KY, KX, orient, half_l, f_words, blockIdx.x, blockIdx.y);
 }
 
@@ -862,6 +997,8 @@ struct TrArgs {
     const __nv_bfloat16* filt;
     uint32_t* fpk;
     int C, KH, KW, KY, KX, half_l, f_words, pack_ncb;
+    int* part_flag;   // split flags of the MMA kernel that follows, cleared by the first packing CTA
+    int nflags;
 };
 
 __device__ __forceinline__ void tr_coords(const TrArgs& a, int t, bool nhwc_side, int (&c)[4])
@@ -892,6 +1029,8 @@ __global__ void __launch_bounds__(256)
     pdl_wait();      // the previous kernel on the stream has finished
     if (static_cast<int>(blockIdx.x) >= a.grid_tr) {   // the filter-packing CTAs of the dY launch
         const int b = static_cast<int>(blockIdx.x) - a.grid_tr;
+        if (b == 0)
+            for (int i = threadIdx.x; i < a.nflags; i += blockDim.x) a.part_flag[i] = 0;
         pack_filter_block(a.filt, a.fpk, a.C, a.KH, a.KW, a.KY, a.KX, a.orient, a.half_l, a.f_words, b % a.pack_ncb,
                           b / a.pack_ncb);
         return;
@@ -1008,6 +1147,9 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     // and tuning).
     const char* shz = dgrad::tuning_env("DGRAD_TC_SHZ");
     const bool no_shz = shz && strcmp(shz, "0") == 0;
+    // DGRAD_TC_SPLIT=0 keeps whole tiles per CTA (testing and tuning).
+    const char* spl = dgrad::tuning_env("DGRAD_TC_SPLIT");
+    const bool no_split = spl && strcmp(spl, "0") == 0;
     // DGRAD_TC_NA=n takes at most n shared-memory tables; DGRAD_TC_NFB=1 one filter-line buffer
     // (testing and tuning).
     const char* nas = dgrad::tuning_env("DGRAD_TC_NA");
@@ -1178,6 +1320,22 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     best.ws_in = round_up(static_cast<size_t>(a.C) * best.Yi * a.N * best.Xsi * 2, 256);
     best.ws_out = round_up(static_cast<size_t>(a.C) * best.Yo * a.N * best.Xso * 2, 256);
     best.ws_f = round_up(static_cast<size_t>(a.C) * best.f_words * 4, 256);
+    // Split: with A tables (two accumulator sets, so a partial's write overlaps the next
+    // tile's MMAs) the CTAs take equal ranges of shift steps, and the tiles two CTAs share
+    // pass an fp32 partial through the workspace: one [set_cols][128] slot and one flag
+    // per CTA, after the filter lines.
+    const long long units = static_cast<long long>((best.Xo + best.XT * best.TW - 1) / (best.XT * best.TW)) *
+                            ((best.Yo + best.P * best.NH - 1) / (best.P * best.NH)) * ((a.N + 7) / 8) * a.C;
+    best.split = best.a_smem && best.tma_epi && !no_split ? 1 : 0;   // the split path stores staged boxes
+    best.part_slots = best.split ? static_cast<int>(std::min<long long>(units, kPlanSms)) : 0;
+    best.part_off = best.ws_f;
+    if (best.split) {
+        const size_t set_cols = static_cast<size_t>(best.XT) * 8 * best.NH;
+        best.flag_off = best.part_off + round_up(static_cast<size_t>(best.part_slots) * 128 * set_cols * 4, 256);
+        best.ws_f = best.flag_off + round_up(static_cast<size_t>(best.part_slots) * 4, 256);
+    } else {
+        best.flag_off = best.ws_f;
+    }
     *out = best;
     return true;
 }
@@ -1186,6 +1344,23 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
                                cudaStream_t stream)
 {
     const CUtensorMap& map_b = maps.b;
+    // The MMA kernel's grid (one CTA per SM at most) and whether its CTAs split tiles:
+    // only with more tiles than CTAs, so that no tile is shared by more than two CTAs.
+    // DGRAD_TC_GRID=n caps the grid (testing: it makes small problems split).
+    const long long units = static_cast<long long>((p.Xo + p.XT * p.TW - 1) / (p.XT * p.TW)) *
+                            ((p.Yo + p.P * p.NH - 1) / (p.P * p.NH)) * ((a.N + 7) / 8) * a.C;
+    if (units > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    int mma_grid = static_cast<int>(units < num_sms ? units : num_sms);
+    if (const char* g = dgrad::tuning_env("DGRAD_TC_GRID")) {
+        const int v = atoi(g);
+        if (v > 0 && v < mma_grid) mma_grid = v;
+    }
+    const bool split = p.split && maps.tma_epi && units > mma_grid && mma_grid <= p.part_slots;
+    float* part = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + p.ws_in + p.ws_out + p.part_off)
+                        : nullptr;
+    int* part_flag = split ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + p.ws_in + p.ws_out + p.flag_off)
+                           : nullptr;
+    const int nflags = split ? mma_grid : 0;
     const int tr_smem = (kTrStages + 2) * 8192 + kTrStages * 8 + 1024;
     if (maps.tma_transpose) {
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_transpose_tma_kernel), tr_smem);
@@ -1219,6 +1394,8 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
             t.f_words = p.f_words;
             t.pack_ncb = (a.C + 31) / 32;
             pack_blocks = t.pack_ncb * p.KY;
+            t.part_flag = part_flag;
+            t.nflags = nflags;
         }
         {
             const cudaError_t le_ = launch_kernel(dw_transpose_tma_kernel, dim3(grid + pack_blocks), dim3(256), tr_smem, stream, 1,
@@ -1258,7 +1435,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
                 const cudaError_t le_ = launch_kernel(dw_filter_pack_kernel, dim3(fgrid), dim3(kPackThreads), 0, stream, 1,
                                                      static_cast<const __nv_bfloat16*>(a.filt), fpk,
                                                                     a.C, a.KH, a.KW, p.KY, p.KX, p.orient, p.half_l,
-                                                                    p.f_words);
+                                                                    p.f_words, part_flag, nflags);
                 if (le_ != cudaSuccess) return le_;
             }
             e = cudaGetLastError();
@@ -1290,9 +1467,10 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.num_xt = (p.Xo + p.XT * p.TW - 1) / (p.XT * p.TW);
         t.num_yt = (p.Yo + p.P * p.NH - 1) / (p.P * p.NH);
         t.num_g = (a.N + 7) / 8;
-        const long long units = static_cast<long long>(t.num_xt) * t.num_yt * t.num_g * a.C;
-        if (units > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
         t.num_units = static_cast<int>(units);
+        t.split = split ? 1 : 0;
+        t.part = part;
+        t.part_flag = part_flag;
         t.a_col0 = p.a_col0;
         t.a_cols = p.a_cols;
         t.na = p.na;
@@ -1324,8 +1502,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.dxp_bytes = static_cast<long long>(p.ws_out);
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));
         if (e != cudaSuccess) return e;
-        const int grid = static_cast<int>(units < num_sms ? units : num_sms);
-        e = launch_kernel(dw_toeplitz_kernel, dim3(grid), dim3(kThreadsT), p.smem, stream, 1, map_b,
+        e = launch_kernel(dw_toeplitz_kernel, dim3(mma_grid), dim3(kThreadsT), p.smem, stream, 1, map_b,
                           maps.tma_epi ? maps.d_store : map_b, t);
         if (e != cudaSuccess) return e;
         e = cudaGetLastError();

@@ -100,7 +100,7 @@ cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStrea
 // a sum of banded-Toeplitz GEMMs, one per filter line.  plan_dw_toeplitz picks
 // the plane orientation and tile and returns false when the problem does not
 // fit; the launch needs a workspace of ws_in + ws_out + ws_f bytes (planar dY,
-// planar dX, packed filter lines) and map_b, a 4-D bf16 map of the planar dY
+// planar dX, packed filter lines and the split partials) and map_b, a 4-D bf16 map of the planar dY
 // [C][Yi][N][Xsi] with dims (Xi, N, Yi, C), box (64, 8, b_rows, 1), 128-byte
 // swizzle, zero fill.
 struct ToepPlan {
@@ -117,6 +117,10 @@ struct ToepPlan {
     // writes once at z_off / z_len)
     int b_zt, b_rows;
     uint32_t b_stride, z_off[3], z_len[3];
+    // split: CTAs take equal ranges of shift steps; part_slots fp32 partial tiles at part_off
+    // and as many flags at flag_off, both offsets into the ws_f region
+    int split, part_slots;
+    size_t part_off, flag_off;
     size_t smem, ws_in, ws_out, ws_f;
 };
 // Tensor maps of one call: b as above; for the transposes (when tma_transpose),

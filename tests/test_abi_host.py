@@ -221,9 +221,10 @@ def test_depthwise_tc_validation_and_workspace_size():
     p31 = cb.Problem(16, 64, 64, 384, 384, 31, 31, 1, 15, 15)
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p31), ctypes.byref(nb)) == OK
     # planar dY + planar dX + packed filter lines (31 lines per channel of (Ks + 80) / 2 words,
-    # Ks <= 144 the tile's MMA depth)
+    # Ks <= 144 the tile's MMA depth) + the split partials (one fp32 128 x 256 tile and one flag
+    # per CTA, at most 148)
     planar = 2 * 384 * 64 * 16 * 64 * 2
-    assert planar < nb.value <= planar + 384 * 31 * 112 * 4
+    assert planar < nb.value <= planar + 384 * 31 * 112 * 4 + 148 * (128 * 256 * 4 + 4) + 512
     p51 = cb.Problem(8, 64, 64, 768, 768, 51, 5, 1, 25, 2)
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), ctypes.byref(nb)) == OK
     assert L.dgrad_depthwise_tc_workspace(ctypes.byref(p51), None) == INVALID

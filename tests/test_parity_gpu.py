@@ -614,6 +614,7 @@ TC_LAYOUT_PROBLEMS = [q for q in TC_SMALL if q.name in ("tc31x31", "tc31x31_c40"
                                                         "tc7x7_nonsame", "tc41x41")] + \
     [q for q in TC_MANY_IMAGES if q.name in ("tcn16_31x31", "tcn13_9x7", "tcn12_5x51")]
 TC_LAYOUTS = {"own_zero_rows": {"DGRAD_TC_SHZ": "0"},
+              "whole_tiles_per_cta": {"DGRAD_TC_SPLIT": "0"},
               "4_tables": {"DGRAD_TC_NA": "4"},
               "5_tables": {"DGRAD_TC_NA": "5"},
               "one_filter_buffer_4_tables": {"DGRAD_TC_NFB": "1", "DGRAD_TC_NA": "4"}}
@@ -640,6 +641,41 @@ def test_depthwise_tensor_core_b_layouts(p, layout, monkeypatch):
     absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
     h.check(p, got, ref, absref, what=f"{p.name}/{layout}")
     assert torch.equal(out, base), f"{p.name}: {layout} differs from the default layout"
+
+
+# Balanced shift-step ranges: with A tables the CTAs take equal ranges of shift steps, and a tile
+# two CTAs share passes an fp32 partial through the workspace.  DGRAD_TC_GRID caps the grid so that
+# these small problems have more tiles than CTAs and split at many different steps.
+TC_SPLIT_PROBLEMS = [q for q in TC_SMALL if q.name in ("tc31x31", "tc31x31_c40", "tc17x17_nonsame", "tc41x41",
+                                                       "tc31x31_f16")] + \
+    [q for q in TC_MANY_IMAGES if q.name in ("tcn16_31x31", "tcn11_17x17_f16")]
+
+
+@pytest.mark.parametrize("transpose", ["tma", "cuda"])
+@pytest.mark.parametrize("grid", [2, 3, 5, 7])
+@pytest.mark.parametrize("p", TC_SPLIT_PROBLEMS, ids=[q.name for q in TC_SPLIT_PROBLEMS])
+def test_depthwise_tensor_core_split_steps(p, grid, transpose, monkeypatch):
+    """The planar tensor-core kernel with tiles split between CTAs at shift-step boundaries (a few
+    CTAs for many tiles), through the TMA and the CUDA-core transposes (each clears the split flags),
+    against the oracle on every element; the workspace starts as NaN and a second call gives
+    identical bits."""
+    h = _h()
+    import convolution_backward_b200 as cb
+    monkeypatch.setenv("DGRAD_TC_GRID", str(grid))
+    if transpose == "cuda":
+        monkeypatch.setenv("DGRAD_TC_TRANSPOSE", "cuda")
+    inp = synthetic.make_inputs(p)
+    dy, w = h.to_dev(inp)
+    nb = cb.depthwise_tc_workspace_bytes(p.N, p.H, p.W, p.C, p.KH, p.KW, p.pad_h, p.pad_w)
+    ws = torch.full((nb // 2 + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=ws)
+    again = cb.depthwise_tc(dy, w, H=p.H, Wd=p.W, pad_h=p.pad_h, pad_w=p.pad_w, workspace=ws)
+    cb.check_status()
+    assert torch.equal(out, again), f"{p.name}: two calls differ"
+    got = h.gpu_to_np(out)
+    ref = h.oracle_full(p, inp.dy, inp.w)
+    absref = h.oracle_full(p, np.abs(inp.dy), np.abs(inp.w))
+    h.check(p, got, ref, absref, what=f"{p.name}/split over {grid} CTAs ({transpose} transposes)")
 
 
 TC_AUTO = [q for q in TC_SMALL if q.KH * q.KW > 49]
