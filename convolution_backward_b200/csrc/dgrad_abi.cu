@@ -616,13 +616,17 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
             if (e != cudaErrorNotSupported) return e == cudaSuccess ? DGRAD_OK : cuda_fail(e);
         }
     }
-    if (mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box)) {
+    if (unsigned tbox_dx[4]; mode == DGRAD_DW_ROTATED && !force_line && dgrad::dw_tile_box(a, box, tbox_dx)) {
         // small filters: one halo tile per CTA
-        CUtensorMap map;
+        CUtensorMap map, dx_map;
         if (!encode_nhwc_h16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box, a.f16))
             return cuda_fail(cudaErrorInvalidValue);
-        e = dgrad::launch_dw_tile(a, map, cs);
+        // the output map is optional: without it the kernel stores dX directly
+        const bool dx_ok = aligned16(dX) && encode_nhwc_h16(&dx_map, dX, static_cast<uint64_t>(prob->N),
+                                                            static_cast<uint64_t>(prob->H), static_cast<uint64_t>(prob->W),
+                                                            static_cast<uint64_t>(prob->C), tbox_dx, a.f16);
+        e = dgrad::launch_dw_tile(a, map, dx_ok ? &dx_map : nullptr, cs);
     } else if (mode == DGRAD_DW_ROTATED) {
         e = dgrad::launch_dw_rotated(a, cs);
     } else if (unsigned box_dx[4]; env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box, box_dx)) {

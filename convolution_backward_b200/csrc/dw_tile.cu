@@ -14,11 +14,15 @@
 //     it walks the R+KH-1 input rows it needs once, converting each 16-bit pair
 //     to fp32 once, and applies every filter row that input row reaches
 //     (packed fma.rn.f32x2, the rotated filter held in registers);
-//   * results are rounded to the I/O format and stored straight to dX (16 threads write
-//     64 contiguous bytes).
+//   * results are rounded to the I/O format into an output tile [TH][TW][32] that
+//     replaces the halo tile in shared memory, and one TMA box stores it, clipping
+//     the ragged edges (3x3 on 8 x 56 x 56 x 128: 5.68 -> 5.16 us on B200 against
+//     direct 4-byte stores, which DGRAD_TILE_STORE=direct keeps for testing).
 #include "common.cuh"
 #include "host_util.h"
 #include "launchers.h"
+
+#include <cstring>
 
 namespace dgrad {
 namespace {
@@ -31,12 +35,14 @@ struct TileParams {
     int CS, RS;       // column and row slots per CTA (threads = 16 * CS * RS)
     int TH, TW;       // output tile
     int nX, nY, nC;
+    int tma_out;          // the output tile is staged in shared memory and stored with one TMA box
     long long dx_bytes;   // size of dX (index checks of the debug build)
 };
 
 template <int KH, int KW, int R, int TAT, int EK>
 __global__ void __launch_bounds__(256)
-    dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const TileParams p)
+    dw_tile_kernel(const __grid_constant__ CUtensorMap dy_map, const __grid_constant__ CUtensorMap dx_map,
+                   const TileParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -132,6 +138,25 @@ __global__ void __launch_bounds__(256)
             }
     }
 
+    if (p.tma_out) {
+        // The output tile [TH][TW][32 channels] replaces the halo tile in shared memory and
+        // one TMA box stores it; the box clips rows, columns and channels past dX.
+        __syncthreads();   // every thread has read the halo tile
+        uint32_t* out_t = reinterpret_cast<uint32_t*>(smem);
+#pragma unroll
+        for (int ro = 0; ro < R; ++ro)
+#pragma unroll
+            for (int j = 0; j < TAT; ++j)
+                out_t[((row0 + ro) * p.TW + col0 + j) * 16 + cp] = float2_to_h16x2<EK>(acc[ro][j].x, acc[ro][j].y);
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&dx_map, smem, c0, w0, h0, n);
+            bulk_commit_group();
+            bulk_wait_group<0>();   // the tile has been read and written before the CTA ends
+        }
+        return;
+    }
     if (!c_ok) return;
     const long long row_elems = static_cast<long long>(p.W) * p.C;
     uint16_t* obase = p.dX + static_cast<long long>(n) * p.H * row_elems + c;
@@ -180,9 +205,12 @@ TileParams plan_tile(const DwArgs& a)
 }
 
 template <int KH, int KW, int R, int TAT>
-cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t stream)
+cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, const CUtensorMap* dx_map, cudaStream_t stream)
 {
-    const TileParams p = plan_tile<KH, KW, R, TAT>(a);
+    TileParams p = plan_tile<KH, KW, R, TAT>(a);
+    // DGRAD_TILE_STORE=direct keeps the direct 4-byte stores of dX (testing and tuning)
+    const char* ts = dgrad::tuning_env("DGRAD_TILE_STORE");
+    p.tma_out = dx_map != nullptr && !(ts && strcmp(ts, "direct") == 0) ? 1 : 0;
     const long long blocks = static_cast<long long>(a.N) * p.nC * p.nY * p.nX;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
@@ -193,7 +221,7 @@ cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
     if (e != cudaSuccess) return e;
     {
         const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(16 * p.CS * p.RS), smem, stream, 1,
-                                             map, p);
+                                             map, p.tma_out ? *dx_map : map, p);
         if (le_ != cudaSuccess) return le_;
     }
     return cudaGetLastError();
@@ -206,7 +234,7 @@ cudaError_t launch_tile(const DwArgs& a, const CUtensorMap& map, cudaStream_t st
 
 }  // namespace
 
-bool dw_tile_box(const DwArgs& a, unsigned box[4])
+bool dw_tile_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4])
 {
     if (!(a.bf16 || a.f16) || a.S != 1) return false;
 #define DGRAD_TILE_BOX(kh, kw, r, tat)                                                              \
@@ -214,6 +242,8 @@ bool dw_tile_box(const DwArgs& a, unsigned box[4])
         const TileParams p = plan_tile<kh, kw, r, tat>(a);                                          \
         box[0] = 32; box[1] = static_cast<unsigned>(p.TW + kw - 1);                                  \
         box[2] = static_cast<unsigned>(p.TH + kh - 1); box[3] = 1;                                   \
+        box_dx[0] = 32; box_dx[1] = static_cast<unsigned>(p.TW);                                    \
+        box_dx[2] = static_cast<unsigned>(p.TH); box_dx[3] = 1;                                     \
         return true;                                                                                \
     }
     DGRAD_TILE_SET(DGRAD_TILE_BOX)
@@ -221,11 +251,11 @@ bool dw_tile_box(const DwArgs& a, unsigned box[4])
     return false;
 }
 
-cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream)
+cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map, cudaStream_t stream)
 {
     if (!(a.bf16 || a.f16) || a.S != 1) return cudaErrorNotSupported;
 #define DGRAD_TILE_LAUNCH(kh, kw, r, tat) \
-    if (a.KH == kh && a.KW == kw) return launch_tile<kh, kw, r, tat>(a, dy_map, stream);
+    if (a.KH == kh && a.KW == kw) return launch_tile<kh, kw, r, tat>(a, dy_map, dx_map, stream);
     DGRAD_TILE_SET(DGRAD_TILE_LAUNCH)
 #undef DGRAD_TILE_LAUNCH
     return cudaErrorNotSupported;

@@ -92,9 +92,11 @@ cudaError_t launch_dw_rotated(const DwArgs& a, cudaStream_t stream);
 
 // Stride-1 depthwise for small filters (3x3, 5x5, 7x7; bf16 or f16): one TMA halo
 // tile per CTA.  dy_map covers dY as a 4-D 16-bit tensor (C, Wo, Ho, N innermost first)
-// with the box dw_tile_box returns.  cudaErrorNotSupported when not compiled.
-bool dw_tile_box(const DwArgs& a, unsigned box[4]);
-cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, cudaStream_t stream);
+// with the box dw_tile_box returns; dx_map (or null) covers dX the same way (C, W, H, N)
+// with box_dx, and the kernel then stores each output tile through it.
+// cudaErrorNotSupported when not compiled.
+bool dw_tile_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4]);
+cudaError_t launch_dw_tile(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map, cudaStream_t stream);
 
 // Stride-1 depthwise on the tcgen05 tensor cores (bf16): each channel plane as
 // a sum of banded-Toeplitz GEMMs, one per filter line.  plan_dw_toeplitz picks

@@ -41,6 +41,8 @@ CASES = [
     (P("pw_f32", "pointwise", "f32", 2, 7, 9, 44, 20, seed=502), {}, "auto"),
     (P("pw_f16_taps", "pointwise", "f16", 1, 9, 11, 40, 72, seed=503), {}, "auto"),
     (P("dw_tile_3x3", "depthwise", "bf16", 2, 17, 19, 40, 40, 3, 3, 1, 1, 1, seed=504), {}, "rotated"),
+    (P("dw_tile_3x3_direct", "depthwise", "bf16", 2, 17, 19, 40, 40, 3, 3, 1, 1, 1, seed=504),
+     {"DGRAD_TILE_STORE": "direct"}, "rotated"),
     (P("dw_rot_13x9_f32", "depthwise", "f32", 1, 21, 17, 36, 36, 13, 9, 1, 6, 4, seed=505), {}, "rotated"),
     (P("dw_rs_reg_7x7s2", "depthwise", "bf16", 2, 23, 29, 40, 40, 7, 7, 2, 3, 3, seed=506), {}, "rowstream"),
     (P("dw_rs_reg_7x7s2_direct", "depthwise", "bf16", 2, 23, 29, 40, 40, 7, 7, 2, 3, 3, seed=506),

@@ -156,11 +156,14 @@ ROT_SMALL = [
 ]
 
 
-@pytest.mark.parametrize("kernel", ["tile", "line"])
+@pytest.mark.parametrize("kernel", ["tile", "tile-direct-stores", "line"])
 @pytest.mark.parametrize("p", ROT_SMALL, ids=[p.name for p in ROT_SMALL])
 def test_rotated_small_filter_kernels(p, kernel, monkeypatch):
     """Small stride-1 filters through the halo-tile kernel and the line kernel."""
     h = _h()
+    if kernel == "tile-direct-stores":
+        monkeypatch.setenv("DGRAD_TILE_STORE", "direct")   # the tile kernel without its TMA-stored output tile
+        kernel = "tile"
     monkeypatch.setenv("DGRAD_ROT_KERNEL", kernel)
     inp = synthetic.make_inputs(p)
     dy, w = h.to_dev(inp)
