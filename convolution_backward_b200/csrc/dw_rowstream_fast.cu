@@ -571,6 +571,9 @@ FastParams plan_fast(const DwArgs& a, const void* kern = nullptr, size_t (*smem_
             nb_best = nb;
         }
     }
+    // DGRAD_RS_BANDS=n forces the band count (testing and tuning)
+    if (const char* eb = dgrad::tuning_env("DGRAD_RS_BANDS"))
+        if (atoi(eb) >= 1 && kern) nb_best = std::min(atoi(eb), max_nb);
     int bh = (a.H + nb_best - 1) / nb_best;
     bh = ((bh + nf - 1) / nf) * nf;
     p.BH = bh;

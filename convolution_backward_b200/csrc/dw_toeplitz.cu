@@ -113,7 +113,8 @@ struct ToepArgs {
     int clip;                    // one tile spans the row: B starts at input column 0 (xb = 0)
     int nfb;                     // filter-line buffers: 2 when they fit, so the next channel's lines load early
     int tma_epi;                 // the epilogue stages 8 x 8 x 64 boxes in shared memory and stores them by TMA
-    uint32_t stg_off;            // two 8 KB staging boxes (one per epilogue half)
+    uint32_t stg_off;            // 8 KB staging boxes: one or two per epilogue half
+    int nstg;                    // staging boxes per half (two: a box is staged while the last one is read)
     uint32_t panel_bytes, b_bytes, npanels, f_bytes, f_words, f_off, bar_off;
     // B blocks: b_stride bytes apart.  When a tile spans the whole plane height, the rows of
     // zero padding above and below the image are written once, and neighbouring blocks share
@@ -674,6 +675,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         uint32_t ub = 0;
         bool ok = true;
         const int part_row_i = m + half * hcols * 128;
+        uint32_t stg_seq = 0;   // staged boxes of this half so far
         // split, CTA ending inside its last unit: that unit's accumulator set is freed by the
         // drain of the unit two before it (or is unused); the partial of the last unit's
         // remaining steps (the next CTA's first unit, ready long before) is written into it
@@ -708,14 +710,24 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                 ok = false;
                 break;
             }
-            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + a.stg_off + half * 8192);
+            uint16_t* stg0 = reinterpret_cast<uint16_t*>(smem + a.stg_off + half * a.nstg * 8192);
             const bool issuer = lane == 0 && (warp & 3) == 2;   // warps 6 and 10
             // P = 2, one sub-tile, staging boxes: the 128 threads of this half hold every row
             // m = (p, xl) of their 32-column chunk cc, i.e. 8 output rows (4 h' x 2 phases) x 8
             // images x 64 columns of one channel's planes; they stage that box in shared memory
             // and one thread stores it with TMA, which clips the ragged edges.
             auto stage_chunk = [&](int cc, const uint32_t* q) {
-                if (issuer) bulk_wait_group_read<0>();   // the previous box has been read
+                (void)cc;
+                uint16_t* stg = stg0 + (a.nstg == 2 ? (stg_seq & 1u) * 4096u : 0u);
+                ++stg_seq;   // boxes alternate between the buffers in the order they are staged
+                // the box staged in this buffer before has been read (with two buffers the
+                // last box may still be in flight)
+                if (issuer) {
+                    if (a.nstg == 2)
+                        bulk_wait_group_read<1>();
+                    else
+                        bulk_wait_group_read<0>();
+                }
                 named_barrier_sync(1 + half, 128);
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
@@ -1150,6 +1162,9 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
     // DGRAD_TC_SPLIT=0 keeps whole tiles per CTA (testing and tuning).
     const char* spl = dgrad::tuning_env("DGRAD_TC_SPLIT");
     const bool no_split = spl && strcmp(spl, "0") == 0;
+    // DGRAD_TC_STG=1 keeps one epilogue staging box per half (testing and tuning).
+    const char* stgs = dgrad::tuning_env("DGRAD_TC_STG");
+    const bool one_stg = stgs && strcmp(stgs, "1") == 0;
     // DGRAD_TC_NA=n takes at most n shared-memory tables; DGRAD_TC_NFB=1 one filter-line buffer
     // (testing and tuning).
     const char* nas = dgrad::tuning_env("DGRAD_TC_NA");
@@ -1292,9 +1307,15 @@ bool plan_dw_toeplitz(const DwArgs& a, ToepPlan* out, bool nhwc)
                               128u * (p.P - 1) * static_cast<size_t>(std::max(0, 16 - p.Ks / 8));
                     }
                     p.stg_off = 0;
+                    p.nstg = 1;
                     if (p.tma_epi) {
                         p.stg_off = static_cast<uint32_t>(round_up(end, 1024));
                         end = p.stg_off + 2 * 8192;
+                        // a second staging box per half when it fits beside everything else
+                        if (end + 2 * 8192 + 1024 <= 227 * 1024 && !one_stg) {
+                            p.nstg = 2;
+                            end += 2 * 8192;
+                        }
                     }
                     // At least 120 KB, so that one CTA runs per SM (each allocates all 512 TMEM columns).
                     p.smem = end + 1024;
@@ -1498,6 +1519,7 @@ cudaError_t launch_dw_toeplitz(const DwArgs& a, const ToepPlan& p, const ToepMap
         t.clip = p.clip;
         t.tma_epi = p.tma_epi && maps.tma_epi ? 1 : 0;
         t.stg_off = p.stg_off;
+        t.nstg = p.nstg;
         t.bar_off = p.bar_off;
         t.dxp_bytes = static_cast<long long>(p.ws_out);
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(dw_toeplitz_kernel), static_cast<int>(p.smem));

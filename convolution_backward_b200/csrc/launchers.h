@@ -113,6 +113,7 @@ struct ToepPlan {
     uint32_t a_off, a_bytes;     // offset of the first A table and the stride between them
     int tma_epi;          // the MMA epilogue stores staged boxes by TMA (needs ToepMaps::d_store)
     uint32_t stg_off;     // its staging boxes in shared memory
+    int nstg;             // staging boxes per epilogue half (1 or 2)
     uint32_t panel_bytes, b_bytes, f_off, bar_off;
     // B blocks b_stride bytes apart; the TMA box brings b_rows rows starting b_zt rows into a
     // block (b_rows = NR, b_zt = 0 unless the blocks share their zero rows, which the kernel

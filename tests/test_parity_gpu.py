@@ -618,6 +618,7 @@ TC_LAYOUT_PROBLEMS = [q for q in TC_SMALL if q.name in ("tc31x31", "tc31x31_c40"
     [q for q in TC_MANY_IMAGES if q.name in ("tcn16_31x31", "tcn13_9x7", "tcn12_5x51")]
 TC_LAYOUTS = {"own_zero_rows": {"DGRAD_TC_SHZ": "0"},
               "whole_tiles_per_cta": {"DGRAD_TC_SPLIT": "0"},
+              "one_staging_box_per_half": {"DGRAD_TC_STG": "1"},
               "4_tables": {"DGRAD_TC_NA": "4"},
               "5_tables": {"DGRAD_TC_NA": "5"},
               "one_filter_buffer_4_tables": {"DGRAD_TC_NFB": "1", "DGRAD_TC_NA": "4"}}
