@@ -629,8 +629,9 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
         e = dgrad::launch_dw_tile(a, map, dx_ok ? &dx_map : nullptr, cs);
     } else if (mode == DGRAD_DW_ROTATED) {
         e = dgrad::launch_dw_rotated(a, cs);
-    } else if (unsigned box_dx[4]; env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box, box_dx)) {
-        CUtensorMap map, dx_map;
+    } else if (unsigned box_dx[4], rows8 = 1;
+               env_int("DGRAD_RS_GENERIC", 0) == 0 && dgrad::dw_rowstream_fast_box(a, box, box_dx, &rows8)) {
+        CUtensorMap map, dx_map, dx_map8;
         if (!encode_nhwc_h16(&map, dY, static_cast<uint64_t>(prob->N), static_cast<uint64_t>(Ho),
                              static_cast<uint64_t>(Wo), static_cast<uint64_t>(prob->C), box, a.f16))
             return cuda_fail(cudaErrorInvalidValue);
@@ -638,7 +639,11 @@ dgrad_status_t dgrad_depthwise(const dgrad_problem_t* prob, dgrad_dtype_t dtype,
         const bool dx_ok = aligned16(dX) && encode_nhwc_h16(&dx_map, dX, static_cast<uint64_t>(prob->N),
                                                             static_cast<uint64_t>(prob->H), static_cast<uint64_t>(prob->W),
                                                             static_cast<uint64_t>(prob->C), box_dx, a.f16);
-        e = dgrad::launch_dw_rowstream_fast(a, map, dx_ok ? &dx_map : nullptr, 0, cs);
+        const unsigned box_dx8[4] = {box_dx[0], box_dx[1], rows8, 1};
+        const bool dx8_ok = dx_ok && encode_nhwc_h16(&dx_map8, dX, static_cast<uint64_t>(prob->N),
+                                                     static_cast<uint64_t>(prob->H), static_cast<uint64_t>(prob->W),
+                                                     static_cast<uint64_t>(prob->C), box_dx8, a.f16);
+        e = dgrad::launch_dw_rowstream_fast(a, map, dx8_ok ? &dx_map : nullptr, dx8_ok ? &dx_map8 : nullptr, 0, cs);
     } else {
         e = dgrad::launch_dw_rowstream(a, cs);
     }

@@ -40,7 +40,8 @@
 //     store per output instead of an address computation, a bounds test and a
 //     global store (7x7 stride 2, 32 x 112 x 112 x 96 on B200: 43.0 us with direct
 //     stores, 41.0 us with one thread issuing every box, 37.4 us with the boxes
-//     spread over the warps).
+//     spread over the warps, 35.8 us with one box of all of a step's rows when they
+//     all lie in the band).
 #include "common.cuh"
 #include "host_util.h"
 #include "launchers.h"
@@ -344,7 +345,7 @@ __device__ __forceinline__ void rs_reg_stage(float2 (&acc)[RS][Q], const float2 
 template <int KH, int KW, int S, int Q, int RS, int GT, int EK>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     dw_rs_reg_kernel(const __grid_constant__ CUtensorMap dy_map, const __grid_constant__ CUtensorMap dx_map,
-                     const FastParams p)
+                     const __grid_constant__ CUtensorMap dx_map8, const FastParams p)
 {
     constexpr int NTMAX = (KW + S - 1) / S;
     extern __shared__ uint8_t smem_raw[];
@@ -482,12 +483,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
         __syncthreads();
         if (storer) {
-            // the stage's final rows hb .. hb + GT*S - 1 that lie in this band, one row box each
-            // (TMA clips columns past W and channels past C)
+            // the stage's final rows hb .. hb + GT*S - 1 that lie in this band: one box of all
+            // of them when they all do (thread 0), else one row box each (TMA clips columns
+            // past W and channels past C)
+            if (hb >= h0 && hb + GT * S <= h1) {
+                if (warp == 0) tma_store_4d(&dx_map8, stg, c0, x0, hb, n);
+            } else {
 #pragma unroll 1
-            for (int r = warp; r < GT * S; r += nwarps) {
-                const int h = hb + r;
-                if (h >= h0 && h < h1) tma_store_4d(&dx_map, stg + r * row_words, c0, x0, h, n);
+                for (int r = warp; r < GT * S; r += nwarps) {
+                    const int h = hb + r;
+                    if (h >= h0 && h < h1) tma_store_4d(&dx_map, stg + r * row_words, c0, x0, h, n);
+                }
             }
             bulk_commit_group();
         }
@@ -612,11 +618,12 @@ static bool rs_direct_store()
 }
 
 template <int KH, int KW, int S, int Q, int RS, int GT>
-cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, const CUtensorMap* dx_map, cudaStream_t stream)
+cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, const CUtensorMap* dx_map,
+                       const CUtensorMap* dx_map8, cudaStream_t stream)
 {
     // plan as the shared-ring kernel with G = GT (band rows a multiple of S*GT)
     auto kern = a.f16 ? dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kF16> : dw_rs_reg_kernel<KH, KW, S, Q, RS, GT, kBF16>;
-    const bool tma_out = dx_map != nullptr && !rs_direct_store();
+    const bool tma_out = dx_map != nullptr && dx_map8 != nullptr && !rs_direct_store();
     auto smem_tma = [](int lw, int nthreads) { return reg_smem(GT, lw, S, (nthreads / 16) * Q); };
     auto smem_direct = [](int lw, int) { return reg_smem(GT, lw); };
     FastParams p = plan_fast<KH, KW, S, Q, GT>(a, reinterpret_cast<const void*>(kern),
@@ -631,7 +638,7 @@ cudaError_t launch_reg(const DwArgs& a, const CUtensorMap& map, const CUtensorMa
     if (e != cudaSuccess) return e;
     {
         const cudaError_t le_ = launch_kernel(kern, dim3(static_cast<unsigned>(blocks)), dim3(nthreads), smem, stream, 1,
-                                             map, tma_out ? *dx_map : map, p);
+                                             map, tma_out ? *dx_map : map, tma_out ? *dx_map8 : map, p);
         if (le_ != cudaSuccess) return le_;
     }
     return cudaGetLastError();
@@ -683,16 +690,18 @@ static int alt_g()
     return e && *e ? atoi(e) : 0;
 }
 
-bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4])
+bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4], unsigned* rows_dx8)
 {
     if (!(a.bf16 || a.f16)) return false;
     box_dx[0] = 32; box_dx[1] = 1; box_dx[2] = 1; box_dx[3] = 1;
+    *rows_dx8 = 1;
     if (use_reg_ring()) {
 #define DGRAD_RS_REG_BOX(kh, kw, s, q, rs, gt)                                                     \
         if (a.KH == kh && a.KW == kw && a.S == s) {                                                 \
             const FastParams p = plan_fast<kh, kw, s, q, gt>(a);                                    \
             box[0] = 32; box[1] = static_cast<unsigned>(p.LW); box[2] = gt; box[3] = 1;            \
             box_dx[1] = static_cast<unsigned>(p.TX);                                                \
+            *rows_dx8 = static_cast<unsigned>(gt * s);                                              \
             return true;                                                                            \
         }
         if (reg_q4()) { DGRAD_RS_REG_Q4_SET(DGRAD_RS_REG_BOX) }
@@ -714,14 +723,14 @@ bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4])
 }
 
 // Returns cudaErrorNotSupported when no specialised instantiation serves the problem.
-cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map, int G,
-                                     cudaStream_t stream)
+cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map,
+                                     const CUtensorMap* dx_map8, int G, cudaStream_t stream)
 {
     (void)G;
     if (!(a.bf16 || a.f16)) return cudaErrorNotSupported;
     if (use_reg_ring()) {
 #define DGRAD_RS_REG_LAUNCH(kh, kw, s, q, rs, gt) \
-        if (a.KH == kh && a.KW == kw && a.S == s) return launch_reg<kh, kw, s, q, rs, gt>(a, dy_map, dx_map, stream);
+        if (a.KH == kh && a.KW == kw && a.S == s) return launch_reg<kh, kw, s, q, rs, gt>(a, dy_map, dx_map, dx_map8, stream);
         if (reg_q4()) { DGRAD_RS_REG_Q4_SET(DGRAD_RS_REG_LAUNCH) }
         DGRAD_RS_REG_SET(DGRAD_RS_REG_LAUNCH)
 #undef DGRAD_RS_REG_LAUNCH

@@ -152,15 +152,17 @@ cudaError_t launch_dw_rowstream(const DwArgs& a, cudaStream_t stream);
 
 // Register-blocked row-streaming kernel for the compiled (KH, KW, S) set, bf16
 // or f16.  dy_map covers dY as a 4-D 16-bit tensor (C, Wo, Ho, N innermost first)
-// with no swizzle; dx_map (or null) covers dX the same way (C, W, H, N), and the
-// register-ring kernel then stores its final rows through it.  Returns
-// cudaErrorNotSupported when no instantiation fits.
-cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map, int G,
-                                     cudaStream_t stream);
+// with no swizzle; dx_map and dx_map8 (or null) cover dX the same way (C, W, H, N),
+// with boxes of one row and of rows_dx8 rows, and the register-ring kernel then
+// stores its final rows through them.  Returns cudaErrorNotSupported when no
+// instantiation fits.
+cudaError_t launch_dw_rowstream_fast(const DwArgs& a, const CUtensorMap& dy_map, const CUtensorMap* dx_map,
+                                     const CUtensorMap* dx_map8, int G, cudaStream_t stream);
 
 // Boxes (inner first) the fast row-streaming kernel loads from dY and stores into
-// dX, or false when the problem has no fast instantiation.
-bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4]);
+// dX (box_dx one row high; rows_dx8 the rows of the taller box), or false when the
+// problem has no fast instantiation.
+bool dw_rowstream_fast_box(const DwArgs& a, unsigned box[4], unsigned box_dx[4], unsigned* rows_dx8);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
